@@ -1,0 +1,210 @@
+"""Pins of the oracle's quantizers (no GPU).
+
+* Exact round trip: a tensor built as fp4 x block_scale x global_scale with
+  global scale 0.00390625 (the value in Figure 1 of "Accelerating large
+  language models with NVFP4 quantization") and block scales on the E4M3
+  grid must come back with those very codes, scales and global scale, and
+  reconstruct exactly ("NVFP4 Explained", "How NVFP4 Represents a Value").
+  A wrong 6 * 448 constant, a wrong block-scale formula or a wrong
+  reconstruction fails it.
+* Storage: 4 bits per value plus one 8-bit scale per 16 values plus one FP32
+  per tensor = 4.5 bits/value ("W4A8 vs NVFP4 quantization on GPUs", "Scale
+  layout changes the real storage cost"); 16/4.5 and 8/4.5 match the ~3.5x and
+  ~1.8x of "NVFP4 Explained", "Memory and Accuracy".
+* Outliers: per-16 block scales give lower error than one scale per tensor
+  on outlier-laden data ("NVFP4 Explained", "Why Blocks of 16 Improve
+  Accuracy").
+* Element rounding: each code is the E2M1 value nearest to x * r.
+* 2D blocks ("What is NVFP4?", "Why does scaling matter so much?") reduce to
+  1D blocks when a tile's 16 rows are equal; grouped quantization equals
+  independent quantization of each group.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+
+GRID = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+
+
+def _facts(golden_dir):
+    with open(os.path.join(golden_dir, "format_facts.json")) as f:
+        return {k: v["value"] for k, v in json.load(f).items() if not k.startswith("_")}
+
+
+def _build_exact(rng, rows, k, g, block_rows=1):
+    """x = v * s * g with v on the E2M1 grid (every block holds a +-6) and s an
+    E4M3 value; one block uses s = 448 so amax = 6 * 448 * g."""
+    nb_r, nb_c = rows // block_rows, k // 16
+    s_codes = rng.integers(1, 0x7E, size=(nb_r, nb_c)).astype(np.uint8)
+    s_codes[rng.integers(nb_r), rng.integers(nb_c)] = 0x7E
+    mag_idx = rng.integers(1, 8, size=(rows, k))          # no zeros: avoids the +-0 ambiguity
+    sign = rng.integers(0, 2, size=(rows, k))
+    for br in range(nb_r):
+        for bc in range(nb_c):
+            r = br * block_rows + rng.integers(block_rows)
+            mag_idx[r, bc * 16 + rng.integers(16)] = 7   # a +-6 in every block
+    v = GRID[mag_idx] * np.where(sign == 1, -1.0, 1.0)
+    s = np.array([O.e4m3_decode(c) for c in range(256)])[s_codes]
+    s_el = np.repeat(np.repeat(s, block_rows, axis=0), 16, axis=1)
+    x = v * s_el * g
+    xb = W.to_bf16_bits(x.astype(np.float32))
+    assert np.array_equal(W.bf16_bits_to_f32(xb).astype(np.float64), x), "construction must be exact in BF16"
+    codes = (mag_idx | (sign << 3)).astype(np.uint8)
+    return xb, x, codes, s_codes
+
+
+def _unpack(codes):
+    lo, hi = codes & 0xF, codes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(codes.shape[0], -1)
+
+
+def test_exact_round_trip_1d_fig1_global_scale(golden_dir):
+    g_fig1 = _facts(golden_dir)["example_global_scale"]
+    rng = np.random.default_rng(1)
+    rows, k = 160, 96                                   # 2 scale row tiles, ragged columns
+    xb, x, want_codes, want_s = _build_exact(rng, rows, k, g_fig1)
+    codes, sf, g = O.quantize_1d(xb)
+    assert g == g_fig1
+    assert np.array_equal(_unpack(codes), want_codes)
+    # element 2i in the low nibble of byte i
+    assert np.array_equal(codes, (want_codes[:, 0::2] | (want_codes[:, 1::2] << 4)).astype(np.uint8))
+    for r in range(rows):
+        for b in range(k // 16):
+            assert sf[O.sf_offset(r, b, k)] == want_s[r, b]
+    assert np.array_equal(O.dequantize(codes, sf, g), x)
+
+
+def test_exact_round_trip_2d_fig1_global_scale(golden_dir):
+    g_fig1 = _facts(golden_dir)["example_global_scale"]
+    rng = np.random.default_rng(2)
+    rows, k = 48, 64
+    xb, x, want_codes, want_s = _build_exact(rng, rows, k, g_fig1, block_rows=16)
+    codes, sf, g, sfc = O.quantize_2d(xb, compact=True)
+    assert g == g_fig1
+    assert np.array_equal(_unpack(codes), want_codes)
+    assert np.array_equal(sfc, want_s)
+    for r in range(rows):
+        for b in range(k // 16):
+            assert sf[O.sf_offset(r, b, k)] == want_s[r // 16, b]
+    assert np.array_equal(O.dequantize(codes, sf, g), x)
+
+
+def test_storage_is_4p5_bits_per_value(golden_dir):
+    f = _facts(golden_dir)
+    for rows, k in [(128, 64), (256, 4096), (8192, 4096)]:
+        n = rows * k
+        code_bytes = rows * k // 2
+        scale_bytes = O.scale_rows(rows) * O.scale_cols(k)
+        total_bits = 8 * (code_bytes + scale_bytes) + f["tensor_scale_bits"]
+        assert scale_bytes * 8 == n // f["block_size_1d"] * f["scale_bits_per_block"]
+        assert (total_bits - f["tensor_scale_bits"]) / n == f["bits_per_value"]
+    ratio16, ratio8 = 16 / f["bits_per_value"], 8 / f["bits_per_value"]
+    # 16/4.5 = 3.56 reads as "~3.5x"; 8/4.5 = 1.78 reads as "~1.8x"
+    assert f["memory_ratio_vs_fp16"] <= ratio16 < f["memory_ratio_vs_fp16"] + 0.1
+    assert abs(ratio8 - f["memory_ratio_vs_fp8"]) < 0.05
+
+
+@pytest.mark.parametrize("which", ["tiny", "laplace"])
+def test_block_scaling_beats_single_scale_on_outliers(which):
+    if which == "tiny":
+        xb, _ = W.tiny(0)
+    else:
+        xb = W.laplace_outliers_bf16((512, 1024), 0, 3)
+    x = O.bf16_to_f64(xb)
+    codes, sf, g = O.quantize_1d(xb)
+    xh = O.dequantize(codes, sf, g)
+    xs = O.single_scale_fp4(xb)
+    e_blk = (x - xh) ** 2
+    e_one = (x - xs) ** 2
+    assert e_blk.mean() <= e_one.mean()
+    per_blk = e_blk.reshape(-1, 16).sum(1)
+    per_one = e_one.reshape(-1, 16).sum(1)
+    assert np.mean(per_blk <= per_one) >= 0.95
+
+
+def test_codes_are_nearest_e2m1_of_scaled_input():
+    xb = W.laplace_outliers_bf16((256, 512), 0, 3, outlier_frac=0.01)
+    codes, sf, g = O.quantize_1d(xb)
+    rows, k = xb.shape
+    x = W.bf16_bits_to_f32(xb)
+    sfb = np.array([[sf[O.sf_offset(r, b, k)] for b in range(k // 16)] for r in range(rows)])
+    dec_s = np.array([O.e4m3_decode(c) for c in range(256)], np.float32)[sfb]
+    d = (dec_s * np.float32(g)).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        r = np.where(d == 0, np.float32(0), np.float32(1) / d).astype(np.float32)
+    y = (x * np.repeat(r, 16, axis=1)).astype(np.float32)
+    dec = np.array([O.e2m1_decode(c) for c in range(16)])[_unpack(codes)]
+    # nearest grid magnitude, ties to the even code, saturating at 6
+    ay = np.abs(y.astype(np.float64))
+    dist = np.abs(ay[..., None] - GRID)
+    best = dist.min(-1)
+    assert np.all(np.abs(np.abs(dec) - ay) == best)
+    # a block whose scale is a normal E4M3 value reaches the top code 6
+    normal_blocks = sfb >= 0x08
+    top = np.abs(dec).reshape(rows, k // 16, 16).max(-1)
+    assert np.all(top[normal_blocks] == 6.0)
+
+
+def test_2d_reduces_to_1d_when_tile_rows_are_equal():
+    base = W.gaussian_bf16((4, 128), 0, 11, 0.02)
+    xb = np.repeat(base, 16, axis=0)                   # every 16-row tile has equal rows
+    c1, s1, g1 = O.quantize_1d(xb)
+    c2, s2, g2 = O.quantize_2d(xb)
+    assert g1 == g2 and np.array_equal(c1, c2) and np.array_equal(s1, s2)
+
+
+def test_2d_scale_replicated_over_tile_rows():
+    xb = W.gaussian_bf16((64, 256), 0, 12, 0.02)
+    codes, sf, g, sfc = O.quantize_2d(xb, compact=True)
+    for r in range(64):
+        for b in range(16):
+            assert sf[O.sf_offset(r, b, 256)] == sfc[r // 16, b]
+
+
+def test_grouped_equals_independent_groups():
+    rng = np.random.default_rng(3)
+    sizes = [0, 5, 128, 130, 0, 1, 257]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    xb = W.gaussian_bf16((int(off[-1]), 64), 0, 13, 1.0, outlier_frac=0.01)
+    codes, sf, g = O.quantize_1d_grouped(xb, off)
+    C = O.scale_cols(64)
+    row0 = 0
+    for e, n in enumerate(sizes):
+        a, b = off[e], off[e + 1]
+        if n:
+            c1, s1, g1 = O.quantize_1d(xb[a:b])
+            assert g[e] == g1
+            assert np.array_equal(codes[a:b], c1)
+            assert np.array_equal(sf[row0 * C:(row0 + O.scale_rows(n)) * C], s1)
+        else:
+            assert g[e] == 1.0
+        row0 += O.scale_rows(n)
+    assert sf.size == row0 * C
+
+
+def test_zero_tensor_and_signed_zero():
+    xb = np.zeros((3, 32), np.uint16)
+    xb[1, 3] = 0x8000                                  # BF16 -0.0
+    codes, sf, g = O.quantize_1d(xb)
+    assert g == 1.0 and not sf.any()
+    u = _unpack(codes)
+    assert u[1, 3] == 0x8 and (u.sum() == 0x8)
+
+
+def test_nonfinite_input_rejected():
+    xb = np.zeros((1, 16), np.uint16)
+    xb[0, 5] = 0x7F80                                  # +inf
+    with pytest.raises(ValueError):
+        O.quantize_1d(xb)
+
+
+def test_scale_layout_is_a_bijection():
+    for rows, k in [(128, 64), (200, 80), (1, 16)]:
+        R, C = O.scale_rows(rows), O.scale_cols(k)
+        offs = {O.sf_offset(r, c, k) for r in range(R) for c in range(C)}
+        assert offs == set(range(R * C))
