@@ -1,0 +1,561 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 W4A4 hot path on B200.
+
+One step = one pass of the whole path over one batch: dynamic NVFP4
+quantization of the BF16 activations (tensor amax, block scales, E2M1 codes)
+followed by the block-scaled FP4 x FP4 GEMM against pre-quantized NVFP4
+weights, BF16 output.  Default workload (the prefill-shaped GEMM):
+A bf16 [4096, 4096] quantized per call, W nvfp4 [14336, 4096] (2D-quantized
+once, outside the timed region), C bf16 [4096, 14336].
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload prefill|quant|decode|moe] [--decode-m M]
+
+Prints one JSON line.  `value` is whole-job throughput (TFLOP/s of 2*M*N*K
+per step, summed over ranks, divided by the slowest rank's time).  L2 is
+flushed (a 256 MiB write) before every timed step and outside its events.
+Timing: CUDA events on the launching stream around each step; per-kernel
+durations come from separate event-timed loops of the GEMM and of the
+quantizer alone on the same inputs.  N > 1 runs N independent replicas (the
+path needs no exchange between GPUs), one process per GPU.
+
+--impl reference times the CPU oracle (plain C, binary64 GEMM) on a bounded
+sample of the same workload: rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+FP4_PER_BF16 = 4.0            # dense FP4 / dense BF16 nominal ratio (9 / 2.25 PFLOP/s)
+METRIC = "W4A4 NVFP4 GEMM TFLOPS (% dense FP4 peak); quantize GB/s (% HBM peak)"
+
+
+def quant_bytes(rows: int, k: int, groups: int = 1) -> int:
+    """Algorithmic bytes of one quantizer call: read BF16 once, write packed
+    codes and one E4M3 scale per 16 values, and the FP32 global scale(s)."""
+    n = rows * k
+    return 2 * n + n // 2 + n // 16 + 4 * groups
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": FALLBACK_HBM_GBS, "bf16_tflops": FALLBACK_BF16_TFLOPS,
+                "bf16_tflops_sustained": FALLBACK_BF16_TFLOPS, "source": "fallback"}
+
+
+# ---- clocks sampled during the timed region (NVML, read only) -------------------------
+
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+            0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, torch_device_index: int):
+        self.samples = []
+        self._stop = threading.Event()
+        self._thr = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            import torch
+            uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+            h = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                hi = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(hi)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                    h = hi
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.h = h
+            self.nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001 - clocks are reported as unavailable
+            self.err = str(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                try:
+                    rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                except AttributeError:
+                    rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+            time.sleep(0.02)
+
+    def stop(self):
+        if self._thr:
+            self._stop.set()
+            self._thr.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": f"NVML unavailable: {self.err}"}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        if not inside:   # very short timed region: nearest samples after it
+            inside = [s for s in self.samples if s[0] >= t0][:5] or self.samples[-5:]
+        mask = 0
+        for s in inside:
+            mask |= int(s[2])
+        reasons = [name for bit, name in _REASONS.items() if mask & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(s[1] for s in inside), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ---- distributed plumbing (replicas; the only collective is the timing reduction) -----
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def reduce_max(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---- workloads ----------------------------------------------------------------------------
+
+class Prefill:
+    name = "prefill"
+
+    def __init__(self, nv, torch, dev, m=4096, n=14336, k=4096):
+        import workloads as W
+        self.m, self.n, self.k = m, n, k
+        a, w = W.prefill(0, m, n, k)
+        self.a_host = a
+        self.a = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        wdev = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.w = nv.quantize_weight_2d(wdev)          # offline: pre-quantized weights
+        del wdev
+        self.c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        self.nv = nv
+        self.flops = 2.0 * m * n * k
+        self.qa = nv.quantize_act(self.a)
+        self.qbytes = quant_bytes(m, k)
+        self.launches_per_step = 3                    # amax, quantize, GEMM
+
+    def quantize(self):
+        self.nv.quantize_act(self.a, out=self.qa)
+
+    def gemm(self):
+        self.nv.gemm(self.qa, self.w, out=self.c)
+
+    def step(self):
+        self.quantize()
+        self.gemm()
+
+    def config(self):
+        return {"workload": f"prefill W4A4: A bf16 [{self.m},{self.k}] dynamically quantized (1D blocks) x "
+                            f"W nvfp4 [{self.n},{self.k}] (2D blocks, pre-quantized) -> C bf16 [{self.m},{self.n}]",
+                "m": self.m, "n": self.n, "k": self.k}
+
+
+class Decode(Prefill):
+    name = "decode"
+
+    def __init__(self, nv, torch, dev, m=64):
+        import workloads as W
+        self.m, self.n, self.k = m, 25600, 5120
+        a, w = W.decode(m)
+        self.a_host = a
+        self.a = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        wdev = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.w = nv.quantize_weight_2d(wdev)
+        del wdev
+        self.c = torch.empty((m, self.n), dtype=torch.bfloat16, device=dev)
+        self.nv = nv
+        self.flops = 2.0 * m * self.n * self.k
+        self.qa = nv.quantize_act(self.a)
+        self.qbytes = quant_bytes(m, self.k)
+        self.wbytes = self.n * self.k // 2 + nv.nvfp4_scale_bytes(self.n, self.k)
+        self.launches_per_step = 3
+
+    def config(self):
+        return {"workload": f"decode W4A4: A bf16 [{self.m},{self.k}] quantized per call x W nvfp4 "
+                            f"[{self.n},{self.k}] -> C bf16 [{self.m},{self.n}]", "m": self.m, "n": self.n, "k": self.k}
+
+
+class Quant:
+    name = "quant"
+
+    def __init__(self, nv, torch, dev):
+        import workloads as W
+        self.rows, self.k = 8192, 4096
+        x = W.quant_act(0)
+        self.a_host = x
+        self.a = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.nv = nv
+        self.qa = nv.quantize_act(self.a)
+        self.qbytes = quant_bytes(self.rows, self.k)
+        self.flops = 0.0
+        self.launches_per_step = 2
+
+    def quantize(self):
+        self.nv.quantize_act(self.a, out=self.qa)
+
+    step = quantize
+
+    def config(self):
+        return {"workload": "activation quantizer: bf16 [8192,4096] Laplace(0,1) + 0.1% +-U[50,200] -> nvfp4 "
+                            "(1D 16-element blocks)", "rows": self.rows, "k": self.k}
+
+
+class Moe:
+    name = "moe"
+
+    def __init__(self, nv, torch, dev):
+        import workloads as W
+        a, off, w = W.moe(0)
+        E, N, K = w.shape
+        self.E, self.n, self.k, self.rows = E, N, K, a.shape[0]
+        self.a_host = a
+        self.a = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.off = torch.from_numpy(off).to(dev)
+        wdev = torch.from_numpy(w.reshape(E * N, K).view(np.int16)).to(dev).view(torch.bfloat16)
+        tw = [nv.quantize_weight_2d(wdev[e * N:(e + 1) * N]) for e in range(E)]
+        del wdev
+        self.b_codes = torch.stack([t.codes for t in tw])
+        self.b_scales = torch.cat([t.scales for t in tw])
+        self.b_global = torch.cat([t.global_scale for t in tw])
+        del tw
+        self.c = torch.empty((self.rows, N), dtype=torch.bfloat16, device=dev)
+        self.nv = nv
+        self.flops = 2.0 * self.rows * N * K
+        self.qa = nv.quantize_act(self.a, self.off)
+        self.qbytes = quant_bytes(self.rows, K, E)
+        self.launches_per_step = 3
+
+    def quantize(self):
+        self.nv.quantize_act(self.a, self.off, out=self.qa)
+
+    def gemm(self):
+        self.nv.grouped_gemm(self.qa, self.b_codes, self.b_scales, self.b_global, self.n, out=self.c)
+
+    def step(self):
+        self.quantize()
+        self.gemm()
+
+    def config(self):
+        return {"workload": f"MoE grouped W4A4: {self.rows // 8} tokens top-8 of {self.E} experts, A bf16 "
+                            f"[{self.rows},{self.k}] quantized per expert group x W nvfp4 {self.E}x[{self.n},{self.k}] "
+                            f"-> C bf16 [{self.rows},{self.n}]", "rows": self.rows, "n": self.n, "k": self.k,
+                "experts": self.E}
+
+
+# ---- timing helpers -------------------------------------------------------------------------
+
+def timed_loop(torch, fn, iters, flush):
+    """Per-iteration CUDA-event times (seconds) of fn, L2 flushed before each."""
+    s = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for i in range(iters):
+        flush(i)
+        evs[i][0].record(s)
+        fn()
+        evs[i][1].record(s)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) * 1e-3 for a, b in evs]
+
+
+def cpu_baseline_prefill(wl, max_seconds=12.0):
+    """The oracle as it stands on the host cores: dynamic quantization of the
+    whole A plus the binary64 GEMM of a sample of rows (W reconstructed once,
+    outside the timing)."""
+    import oracle as O
+    import workloads as W
+    a_host = wl.a_host
+    w_bits = W.prefill(0, wl.m, wl.n, wl.k)[1] if wl.name == "prefill" else W.decode(wl.m)[1]
+    wc, wsf, gw = O.quantize_2d(w_bits)
+    wh = O.dequantize(wc, wsf, gw)
+    t = time.perf_counter()
+    ac, asf, ga = O.quantize_1d(a_host)
+    ah = O.dequantize(ac, asf, ga)
+    tq = time.perf_counter() - t
+    t = time.perf_counter()
+    O.gemm_f64_rows(ah, wh, np.arange(min(4, wl.m)))
+    t_row = (time.perf_counter() - t) / min(4, wl.m)
+    rows = int(max(1, min(wl.m, (max_seconds - tq) / max(t_row, 1e-6))))
+    sel = np.linspace(0, wl.m - 1, rows).astype(np.int64)
+    t = time.perf_counter()
+    ac, asf, ga = O.quantize_1d(a_host)
+    ah = O.dequantize(ac, asf, ga)
+    O.gemm_f64_rows(ah, wh, sel)
+    dt = time.perf_counter() - t
+    flops = 2.0 * rows * wl.n * wl.k
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"dynamic quantization of the whole A [{wl.m},{wl.k}] + binary64 GEMM of {rows} of "
+                      f"{wl.m} rows against W [{wl.n},{wl.k}] ({dt:.1f} s)"}
+
+
+def cpu_baseline_quant(wl, max_seconds=12.0):
+    import oracle as O
+    t = time.perf_counter()
+    O.quantize_1d(wl.a_host)
+    dt = time.perf_counter() - t
+    return {"value": wl.qbytes / dt / 1e9, "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"one full quantization of [{wl.rows},{wl.k}] ({dt:.2f} s)"}
+
+
+# ---- the two arms ------------------------------------------------------------------------------
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle as O
+    import workloads as W
+    if args.workload == "quant":
+        x = W.quant_act(0)
+        unit = "GB/s"
+        work = quant_bytes(8192, 4096)
+        cfg = Quant.config(type("Q", (), {"rows": 8192, "k": 4096})())
+
+        def step():
+            O.quantize_1d(x)
+        sample = "one full quantization of [8192,4096] per step"
+    else:
+        m, n, k = (4096, 14336, 4096) if args.workload == "prefill" else (args.decode_m, 25600, 5120)
+        a, w = W.prefill(0, m, n, k) if args.workload == "prefill" else W.decode(m)
+        wc, wsf, gw = O.quantize_2d(w)
+        wh = O.dequantize(wc, wsf, gw)
+        rows = min(m, args.ref_rows)
+        sel = np.linspace(0, m - 1, rows).astype(np.int64)
+        unit = "TFLOP/s"
+        work = 2.0 * rows * n * k
+        cfg = {"workload": f"{args.workload} W4A4 m={m} n={n} k={k}", "m": m, "n": n, "k": k}
+
+        def step():
+            ac, asf, ga = O.quantize_1d(a)
+            O.gemm_f64_rows(O.dequantize(ac, asf, ga), wh, sel)
+        sample = (f"per step: dynamic quantization of the whole A [{m},{k}] + binary64 GEMM of {rows} of {m} "
+                  f"rows against W [{n},{k}]")
+    for _ in range(args.warmup):
+        step()
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t
+    value = work * args.steps / dt / (1e12 if unit == "TFLOP/s" else 1e9)
+    line = {"metric": METRIC, "value": value, "unit": unit, "n_gpus": 0, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+            "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": unit, "kind": "oracle", "cores": O.num_threads(),
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        from nvfp4_w4a4_quantized_05_b200 import build as B
+        entry = t.get(kernel)
+        if entry and entry.get("src_hash") == B._src_hash():
+            return entry.get("bytes_per_launch")
+    except (OSError, ValueError, ImportError):
+        pass
+    return None
+
+
+def run_ours(args):
+    import torch
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        print(json.dumps({"metric": METRIC, "error": "no CUDA device"}))
+        return 1
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    import nvfp4_w4a4_quantized_05_b200 as nv
+    nv.lib()
+    peaks = load_peaks()
+    wl = {"prefill": Prefill, "decode": Decode, "quant": Quant, "moe": Moe}[args.workload]
+    wl = wl(nv, torch, dev, m=args.decode_m) if args.workload == "decode" else wl(nv, torch, dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush(i):
+        flush_buf.fill_(i & 0xFF)
+
+    # warm-up
+    for i in range(max(3, args.warmup)):
+        flush(i)
+        wl.step()
+    torch.cuda.synchronize()
+    nv.check_device_error()
+
+    # ---- timed region: exactly K steps ----
+    sampler = ClockSampler(local)
+    sampler.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    step_times = timed_loop(torch, wl.step, args.steps, flush)
+    torch.cuda.synchronize()
+    barrier(world)
+    t1 = time.perf_counter()
+    sampler.stop()
+    nv.check_device_error()
+    total = reduce_max(sum(step_times), world, dev)
+    clocks = sampler.summary(t0, t1)
+
+    # ---- per-kernel times on the same inputs (separate event-timed loops) ----
+    kiters = max(10, min(args.steps, 200))
+    q_times = timed_loop(torch, wl.quantize, kiters, flush)
+    q_avg = statistics.mean(q_times)
+    g_avg = None
+    if hasattr(wl, "gemm"):
+        g_times = timed_loop(torch, wl.gemm, kiters, flush)
+        g_avg = statistics.mean(g_times)
+    nv.check_device_error()
+
+    # ---- end to end through the public API from pinned host memory ----
+    e2e = None
+    if not args.no_e2e:
+        a_pinned = torch.from_numpy(wl.a_host.view(np.int16)).pin_memory()
+        out_dev = wl.c if hasattr(wl, "c") else wl.qa.codes
+        out_pinned = torch.empty(out_dev.shape, dtype=out_dev.dtype).pin_memory()
+
+        def e2e_step():
+            wl.a.view(torch.int16).copy_(a_pinned, non_blocking=True)
+            wl.step()
+            src = wl.c if hasattr(wl, "c") else wl.qa.codes
+            out_pinned.copy_(src, non_blocking=True)
+        for i in range(2):
+            e2e_step()
+        e_times = timed_loop(torch, e2e_step, max(5, min(args.steps, 50)), flush)
+        e_avg = reduce_max(statistics.mean(e_times), world, dev)
+        h2d = a_pinned.numel() * a_pinned.element_size()
+        d2h = out_pinned.numel() * out_pinned.element_size()
+        if wl.flops:
+            ev, eu = world * wl.flops / e_avg / 1e12, "TFLOP/s"
+        else:
+            ev, eu = world * wl.qbytes / e_avg / 1e9, "GB/s"
+        e2e = {"value": ev, "unit": eu, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    ms = total / args.steps * 1e3
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    q_gbs = wl.qbytes / q_avg / 1e9
+    line = {"metric": METRIC}
+    if wl.flops:
+        value = world * wl.flops * args.steps / total / 1e12
+        line.update({"value": value, "unit": "TFLOP/s"})
+    else:
+        value = world * wl.qbytes * args.steps / total / 1e9
+        line.update({"value": value, "unit": "GB/s"})
+    line.update({"n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                 "dtype": "fp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate)",
+                 "data": "synthetic (seeded; see workloads/)"})
+    cfg = wl.config()
+    cfg.update({"l2": "flushed before every timed step (256 MiB write, outside the step's events)",
+                "parallelism": f"replicas x{world}" if world > 1 else "single GPU"})
+    line["config"] = cfg
+    if g_avg is not None:
+        g_tflops = wl.flops / g_avg / 1e12
+        line["roofline"] = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 mxf4nvf4)",
+                            "achieved": g_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
+                            "frac": g_tflops / fp4_peak, "traffic": load_traffic(f"gemm_{wl.name}"),
+                            "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_PER_BF16} "
+                                         "(dense FP4 / BF16 nominal ratio)",
+                            "avg_launch_ms": g_avg * 1e3}
+    else:
+        line["roofline"] = {"bound": "hbm", "kernel": "amax_kernel + quant1d_kernel", "achieved": q_gbs,
+                            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_gbs / peaks["hbm_gbs"],
+                            "traffic": load_traffic(f"quant_{wl.name}"),
+                            "peak_note": f"{peaks['source']} HBM copy bandwidth", "avg_launch_ms": q_avg * 1e3}
+    line["quantize"] = {"gbs": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"], "avg_ms": q_avg * 1e3,
+                        "algorithmic_bytes": wl.qbytes}
+    if isinstance(wl, Decode):
+        line["weight_stream"] = {"gbs": wl.wbytes / g_avg / 1e9, "frac_hbm": wl.wbytes / g_avg / 1e9 / peaks["hbm_gbs"],
+                                 "bytes": wl.wbytes}
+    line["e2e"] = e2e
+    line["gpu_launches"] = wl.launches_per_step * args.steps
+    line["clocks"] = clocks
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = (cpu_baseline_quant(wl) if wl.name == "quant" else
+                                cpu_baseline_prefill(wl) if wl.name in ("prefill", "decode") else None)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["prefill", "quant", "decode", "moe"], default="prefill")
+    ap.add_argument("--decode-m", type=int, default=64)
+    ap.add_argument("--ref-rows", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,213 @@
+/*
+ * nvfp4.h -- C ABI of libnvfp4.so: NVFP4 W4A4 inference on NVIDIA B200
+ * (sm_100a).  Two stages: dynamic NVFP4 quantization of BF16 tensors, and a
+ * block-scaled FP4 x FP4 GEMM on the tcgen05 tensor cores.
+ *
+ * Format (all entry points):
+ *   Element: E2M1, 1 sign / 2 exponent / 1 mantissa bit, magnitudes
+ *     {0, 0.5, 1, 1.5, 2, 3, 4, 6} ("What is NVFP4? 4-bit AI inference on
+ *     NVIDIA Blackwell explained", "What does NVFP4 mean?").
+ *   Block scale: FP8 E4M3, one per 16 consecutive values along K (1D), or one
+ *     per 16 x 16 tile for weights (2D) (same page, "Why does scaling matter
+ *     so much?"; "NVFP4 Explained: NVIDIA's 4-Bit Format for Faster AI
+ *     Inference", "Why the Block Scale Uses FP8 E4M3").
+ *   Tensor scale: one FP32 per tensor (or per group), kept as a decode
+ *     multiplier:  reconstructed = fp4 x block_scale x global_scale
+ *     ("NVFP4 Explained", "How NVFP4 Represents a Value").
+ *   Readings where the pages are silent:
+ *     global_scale g = amax / (6 * 448), or 1 when amax == 0;
+ *     block scale   = E4M3_rne_satfinite(block_amax / (6 * g));
+ *     code          = E2M1_rne_satfinite(x * r), r = 1 / (block_scale * g),
+ *                     r = 0 when block_scale * g == 0; the sign bit of x is
+ *                     kept, also for zero codes.
+ *   Storage: codes [rows, k/2] bytes, row-major, element 2i in bits 3:0 and
+ *     element 2i+1 in bits 7:4 of byte i -- 4 bits per value; scales 1 byte
+ *     per 16 values; 4.5 bits per value plus 4 bytes per tensor ("W4A8 vs
+ *     NVFP4 quantization on GPUs", "Scale layout changes the real storage
+ *     cost").
+ *   Scale layout (not on the pages; the layout the tensor cores read):
+ *     rows padded to a multiple of 128, scale columns (k/16) padded to a
+ *     multiple of 4, stored as 512-byte tiles of 128 rows x 4 columns, tiles
+ *     ordered row-tile major, column-tile minor; inside a tile row r and
+ *     column c sit at byte (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4).
+ *     Pad bytes are written as zero.
+ *
+ * Conventions:
+ *   - Every buffer is owned by the caller.  Pointers marked "device" must be
+ *     device memory of the current device; all device pointers must be
+ *     16-byte aligned.  No entry point allocates device memory.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  All compute
+ *     entry points are asynchronous on it; argument errors are returned
+ *     before anything is launched.  Device-side failures (a bounded wait
+ *     that ran out) are reported by nvfp4_get_last_device_error.
+ *   - Global scales and group offsets stay on the device: no call waits on
+ *     the host for them.
+ *   - workspace: device scratch of nvfp4_workspace_bytes(...) bytes.  It must
+ *     be zero before its first use (nvfp4_workspace_init); every call that
+ *     returns NVFP4_OK leaves it zero again.  Calls sharing one workspace
+ *     must be ordered on one stream.
+ */
+#ifndef NVFP4_H
+#define NVFP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NVFP4_OK = 0,
+    NVFP4_ERR_INVALID_ARGUMENT = 1,  /* null pointer, negative size, bad group offsets count */
+    NVFP4_ERR_UNSUPPORTED_SHAPE = 2, /* k % 16 (quantize) or k % 64 (GEMM) != 0, n % 16 != 0 (2D), too large */
+    NVFP4_ERR_MISALIGNED = 3,        /* a device pointer or leading dimension breaks 16-byte alignment */
+    NVFP4_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, driver entry point) */
+    NVFP4_ERR_TIMEOUT = 5,           /* a kernel's bounded wait ran out; results are invalid */
+    NVFP4_ERR_NO_DEVICE = 6          /* no sm_100 device current */
+} nvfp4_status_t;
+
+/* Status code -> static string.  Never NULL. */
+const char* nvfp4_status_string(nvfp4_status_t status);
+
+/* Library version, "major.minor.patch". */
+const char* nvfp4_version(void);
+
+/* ---- sizes --------------------------------------------------------------- */
+
+/* Bytes of packed E2M1 codes for a [rows, k] tensor: rows * k / 2. */
+size_t nvfp4_codes_bytes(int64_t rows, int64_t k);
+
+/* Bytes of the tiled E4M3 scale buffer for a [rows, k] tensor:
+ * ceil(rows / 128) * 128 * ceil(k / 64) * 4. */
+size_t nvfp4_scale_bytes(int64_t rows, int64_t k);
+
+/* Upper bound of the scale buffer for grouped quantization of total_rows rows
+ * in num_groups groups: each group's scale rows start at a multiple of 128,
+ * so at most ((total_rows + 127 * num_groups) / 128) * 128 rows of scales. */
+size_t nvfp4_grouped_scale_bytes(int64_t total_rows, int num_groups, int64_t k);
+
+/* Workspace bytes an operation needs (operations below); 0 if none. */
+enum { NVFP4_OP_QUANTIZE_ACT = 0, NVFP4_OP_QUANTIZE_WEIGHT_2D = 1, NVFP4_OP_GEMM = 2,
+       NVFP4_OP_GROUPED_GEMM = 3 };
+size_t nvfp4_workspace_bytes(int op, int64_t rows, int64_t n, int64_t k, int num_groups);
+
+/* Zero a workspace before its first use (cudaMemsetAsync on stream). */
+nvfp4_status_t nvfp4_workspace_init(void* workspace, size_t bytes, void* stream);
+
+/* ---- stage 1: dynamic quantization ----------------------------------------
+ *
+ * nvfp4_quantize_act -- 1D 16-element blocks, global scale from the tensor
+ * amax computed in the same call (dynamic activation quantization: "NVFP4
+ * Dynamic Quantization in Practice", "The Meaning and Advantages of W4A4";
+ * "NVFP4 Explained", FAQ "Can NVFP4 quantize both weights and activations?").
+ *
+ *   x            device, BF16 [rows, k] with row stride ld elements (ld >= k,
+ *                ld % 8 == 0).  Finite values only (NaN/Inf: undefined codes).
+ *   rows, k      rows >= 0, k > 0, k % 16 == 0.
+ *   group_offsets NULL: one tensor.  Otherwise device int32 [num_groups + 1],
+ *                non-decreasing, offsets[0] >= 0, offsets[num_groups] <= rows:
+ *                rows [offsets[e], offsets[e+1]) form group e with its own
+ *                global scale; group e's scale rows start at
+ *                sum_{j<e} ceil128(offsets[j+1] - offsets[j]).  Rows outside
+ *                [offsets[0], offsets[num_groups]) are not touched.
+ *                The offsets are not validated on the device.
+ *   codes        device, nvfp4_codes_bytes(rows, k) bytes.
+ *   scales       device, nvfp4_scale_bytes(rows, k) bytes (one tensor) or
+ *                nvfp4_grouped_scale_bytes(rows, num_groups, k) (grouped);
+ *                every byte of each group's padded scale block is written.
+ *   global_scale device, FP32 [max(1, num_groups)].
+ *   workspace    nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_ACT, rows, 0, k, num_groups).
+ * Two kernels: a tensor-amax reduction, then the quantizer (launched with
+ * programmatic dependent launch so its start overlaps the reduction's end).
+ */
+nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                  const int32_t* group_offsets, int num_groups,
+                                  uint8_t* codes, uint8_t* scales, float* global_scale,
+                                  void* workspace, void* stream);
+
+/* nvfp4_quantize_weight_2d -- 16 x 16 blocks share one E4M3 scale ("What is
+ * NVFP4?", "Why does scaling matter so much?").  The tile's scale is written
+ * to the tiled scale layout for each of its 16 rows (so the GEMM reads it like
+ * 1D scales); scales_compact, if not NULL, receives it once per tile as a
+ * row-major [n/16, k/16] byte array.
+ *   w: device BF16 [n, k], row stride ld (ld >= k, ld % 8 == 0); n % 16 == 0,
+ *   k % 16 == 0.  Other arguments as nvfp4_quantize_act (one tensor). */
+nvfp4_status_t nvfp4_quantize_weight_2d(const void* w, int64_t n, int64_t k, int64_t ld,
+                                        uint8_t* codes, uint8_t* scales,
+                                        uint8_t* scales_compact, float* global_scale,
+                                        void* workspace, void* stream);
+
+/* ---- stage 2: block-scaled FP4 x FP4 GEMM ----------------------------------
+ *
+ * nvfp4_gemm -- C[m, n] = bf16_rn( (sum_k qa[m,k] sa[m,k/16] qb[n,k] sb[n,k/16])
+ *                                  * (a_global[0] * b_global[0]) )
+ * i.e. the product of the two reconstructed NVFP4 operands ("NVFP4 Explained",
+ * "How NVFP4 Represents a Value"), with FP32 accumulation on the tcgen05
+ * block-scaled tensor cores (native FP4 x FP4: "NVFP4 Dynamic Quantization in
+ * Practice", "Impact on the Open-Source Community and LLM Deployment
+ * Industry").  A is [m, k] activations, B is [n, k] weights, both K-major as
+ * written by the quantizers above ("TN").
+ *   a_codes, a_scales, a_global: device; output of nvfp4_quantize_act on [m, k].
+ *   b_codes, b_scales, b_global: device; output of either quantizer on [n, k].
+ *   c: device BF16 [m, n], row stride ldc elements (ldc >= n, ldc % 8 == 0).
+ *   m >= 0, n > 0, k > 0, k % 64 == 0.
+ *   workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, 0) bytes (may be
+ *   NULL when that is 0).
+ * For m <= 64 the kernel runs with the operands swapped (weights fill the
+ * 128-row MMA side; tokens fill the narrow N side), as decode is bound by
+ * streaming the weights ("W4A8 vs NVFP4 quantization on GPUs", "Batch size can
+ * change the winner"). */
+nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                          const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
+                          void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
+                          void* workspace, void* stream);
+
+/* nvfp4_grouped_gemm -- one GEMM per expert over row groups (mixture of
+ * experts: "NVFP4 Dynamic Quantization in Practice", "The Practical
+ * Significance of Full Gemma-4 Quantization Coverage").  For expert e, rows
+ * [offsets[e], offsets[e+1]) of A (quantized per group by nvfp4_quantize_act
+ * with the same offsets) multiply expert e's weights:
+ *   C[r, :] = bf16_rn( (A_e[r, :] . B_e^T) * a_global[e] * b_global[e] ).
+ *   a_codes [total_rows, k/2]; a_scales grouped layout (see nvfp4_quantize_act);
+ *   a_global [num_experts]; offsets device int32 [num_experts + 1] with
+ *   offsets[0] == 0 and offsets[num_experts] == total_rows;
+ *   b_codes [num_experts, n, k/2]; b_scales num_experts consecutive blocks of
+ *   nvfp4_scale_bytes(n, k) bytes; b_global [num_experts];
+ *   c BF16 [total_rows, n] (row stride n), rows in grouped order.
+ *   k % 64 == 0. */
+nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
+                                  const float* a_global, const int32_t* offsets, int num_experts,
+                                  const uint8_t* b_codes, const uint8_t* b_scales,
+                                  const float* b_global, void* c, int64_t n, int64_t k,
+                                  int64_t total_rows, void* workspace, void* stream);
+
+/* ---- diagnostics ------------------------------------------------------------ */
+
+/* Synchronizes stream, then returns NVFP4_ERR_TIMEOUT if any kernel of this
+ * library set its device error word since the last query (and clears it),
+ * NVFP4_ERR_CUDA if the stream holds a CUDA error, else NVFP4_OK. */
+nvfp4_status_t nvfp4_get_last_device_error(void* stream);
+
+/* Limit, in nanoseconds, of every bounded wait inside the GEMM kernels
+ * (mbarrier waits).  Default 2e9 (2 s).  Returns the previous limit.  Used by
+ * tests to make a wait run out quickly; not thread-safe. */
+uint64_t nvfp4_set_wait_limit_ns(uint64_t limit_ns);
+
+/* Hardware format probes: convert n FP32 values with the same conversion
+ * instructions the quantizer uses.  out_e2m1[i] = E2M1 code of in[i] (low
+ * nibble); out_e4m3[i] = E4M3 byte of |in[i]|.  Device pointers.  Used to pin
+ * the kernels' rounding against the CPU definition over wide sweeps. */
+nvfp4_status_t nvfp4_probe_cvt(const float* in, uint8_t* out_e2m1, uint8_t* out_e4m3,
+                               int64_t n, void* stream);
+
+/* Waits on a device flag that nothing sets, bounded by limit_ns, and reports
+ * the outcome like the GEMM kernels do (sets the device error word).  Lets a
+ * test check that a wait which runs out returns NVFP4_ERR_TIMEOUT through
+ * nvfp4_get_last_device_error instead of hanging. */
+nvfp4_status_t nvfp4_probe_bounded_wait(const uint32_t* flag, uint64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H */

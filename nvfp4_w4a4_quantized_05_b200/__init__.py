@@ -1,0 +1,291 @@
+"""NVFP4 W4A4 inference hot path for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI of ``libnvfp4.so`` (``include/nvfp4.h``):
+argument marshalling only.  Every step of the path runs in the library's CUDA
+kernels; PyTorch is used for device memory and streams.  There is no CPU
+fallback: if the library cannot be loaded, every call raises.
+
+Raw entry points keep the C names (``nvfp4_quantize_act``, ``nvfp4_gemm``, ...)
+and take integer device addresses.  The tensor-level helpers
+(``quantize_act``, ``quantize_weight_2d``, ``gemm``, ``grouped_gemm``)
+allocate outputs with torch on the input's device and run on torch's current
+stream.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+from typing import Optional
+
+__all__ = [
+    "lib", "Nvfp4Error", "NVFP4Tensor",
+    "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_grouped_scale_bytes", "nvfp4_workspace_bytes",
+    "nvfp4_workspace_init", "nvfp4_quantize_act", "nvfp4_quantize_weight_2d", "nvfp4_gemm",
+    "nvfp4_grouped_gemm", "nvfp4_get_last_device_error", "nvfp4_set_wait_limit_ns", "nvfp4_probe_cvt",
+    "nvfp4_probe_bounded_wait", "nvfp4_status_string", "nvfp4_version",
+    "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
+    "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4.so")
+
+OP_QUANTIZE_ACT, OP_QUANTIZE_WEIGHT_2D, OP_GEMM, OP_GROUPED_GEMM = 0, 1, 2, 3
+STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
+          5: "TIMEOUT", 6: "NO_DEVICE"}
+
+
+class Nvfp4Error(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({_status_string(status)})")
+
+
+_lib = None
+_lock = threading.Lock()
+_vp, _i64, _u64, _i32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int, ctypes.c_size_t
+
+_SIGNATURES = {
+    "nvfp4_status_string": (ctypes.c_char_p, [_i32]),
+    "nvfp4_version": (ctypes.c_char_p, []),
+    "nvfp4_codes_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_scale_bytes": (_sz, [_i64, _i64]),
+    "nvfp4_grouped_scale_bytes": (_sz, [_i64, _i32, _i64]),
+    "nvfp4_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
+    "nvfp4_workspace_init": (_i32, [_vp, _sz, _vp]),
+    "nvfp4_quantize_act": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nvfp4_quantize_weight_2d": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
+    "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "nvfp4_get_last_device_error": (_i32, [_vp]),
+    "nvfp4_set_wait_limit_ns": (_u64, [_u64]),
+    "nvfp4_probe_cvt": (_i32, [_vp, _vp, _vp, _i64, _vp]),
+    "nvfp4_probe_bounded_wait": (_i32, [_vp, _u64, _vp]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libnvfp4.so (building it first if the sources are newer)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    with _lock:
+        if _lib is None:
+            if os.environ.get("NVFP4_NO_AUTOBUILD") != "1":
+                from . import build as _build
+                if _build.needs_build():
+                    _build.build()
+            if not os.path.exists(LIB_PATH):
+                raise ImportError(f"libnvfp4.so not found at {LIB_PATH}; run "
+                                  "`python -m nvfp4_w4a4_quantized_05_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in _SIGNATURES.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _status_string(status: int) -> str:
+    try:
+        return lib().nvfp4_status_string(int(status)).decode()
+    except Exception:  # noqa: BLE001 - only used to format an error message
+        return "?"
+
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        raise Nvfp4Error(status, what)
+
+
+# ---- raw C ABI (integer addresses) ----------------------------------------------
+
+def nvfp4_status_string(status: int) -> str:
+    return lib().nvfp4_status_string(int(status)).decode()
+
+
+def nvfp4_version() -> str:
+    return lib().nvfp4_version().decode()
+
+
+def nvfp4_codes_bytes(rows: int, k: int) -> int:
+    return int(lib().nvfp4_codes_bytes(rows, k))
+
+
+def nvfp4_scale_bytes(rows: int, k: int) -> int:
+    return int(lib().nvfp4_scale_bytes(rows, k))
+
+
+def nvfp4_grouped_scale_bytes(total_rows: int, num_groups: int, k: int) -> int:
+    return int(lib().nvfp4_grouped_scale_bytes(total_rows, num_groups, k))
+
+
+def nvfp4_workspace_bytes(op: int, rows: int = 0, n: int = 0, k: int = 0, num_groups: int = 0) -> int:
+    return int(lib().nvfp4_workspace_bytes(op, rows, n, k, num_groups))
+
+
+def nvfp4_workspace_init(workspace: int, nbytes: int, stream: int = 0) -> int:
+    return lib().nvfp4_workspace_init(workspace, nbytes, stream)
+
+
+def nvfp4_quantize_act(x, rows, k, ld, group_offsets, num_groups, codes, scales, global_scale, workspace,
+                       stream=0) -> int:
+    return lib().nvfp4_quantize_act(x, rows, k, ld, group_offsets, num_groups, codes, scales, global_scale,
+                                    workspace, stream)
+
+
+def nvfp4_quantize_weight_2d(w, n, k, ld, codes, scales, scales_compact, global_scale, workspace, stream=0) -> int:
+    return lib().nvfp4_quantize_weight_2d(w, n, k, ld, codes, scales, scales_compact, global_scale, workspace,
+                                          stream)
+
+
+def nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k, workspace=None,
+               stream=0) -> int:
+    return lib().nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
+                            workspace, stream)
+
+
+def nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_codes, b_scales, b_global, c, n, k,
+                       total_rows, workspace=None, stream=0) -> int:
+    return lib().nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_codes, b_scales,
+                                    b_global, c, n, k, total_rows, workspace, stream)
+
+
+def nvfp4_get_last_device_error(stream=0) -> int:
+    return lib().nvfp4_get_last_device_error(stream)
+
+
+def nvfp4_set_wait_limit_ns(limit_ns: int) -> int:
+    return int(lib().nvfp4_set_wait_limit_ns(limit_ns))
+
+
+def nvfp4_probe_cvt(inp, out_e2m1, out_e4m3, n, stream=0) -> int:
+    return lib().nvfp4_probe_cvt(inp, out_e2m1, out_e4m3, n, stream)
+
+
+def nvfp4_probe_bounded_wait(flag, limit_ns, stream=0) -> int:
+    return lib().nvfp4_probe_bounded_wait(flag, limit_ns, stream)
+
+
+# ---- tensor-level helpers (torch for memory and streams) -----------------------------
+
+@dataclass
+class NVFP4Tensor:
+    """An NVFP4-quantized [rows, k] tensor living on the device."""
+    codes: "object"            # uint8 [rows, k/2]
+    scales: "object"           # uint8, tiled scale layout
+    global_scale: "object"     # float32 [groups]
+    rows: int
+    k: int
+    offsets: Optional["object"] = None   # int32 [groups+1] for grouped tensors
+
+
+_ws_cache: dict = {}
+
+
+def _stream_ptr(torch, device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _workspace(torch, device, op: int, groups: int = 0):
+    nbytes = nvfp4_workspace_bytes(op, 0, 0, 0, groups)
+    if nbytes == 0:
+        return None
+    key = (device.index, op, groups, torch.cuda.current_stream(device).cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def _ptr(t) -> int:
+    return 0 if t is None else int(t.data_ptr())
+
+
+def quantize_act(x, offsets=None, out: Optional[NVFP4Tensor] = None) -> NVFP4Tensor:
+    """Dynamic 1D NVFP4 quantization of a BF16 [rows, k] CUDA tensor (one
+    global scale, or one per row group when int32 ``offsets`` [G+1] is given).
+    ``out`` reuses the buffers of an earlier result of the same shape."""
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along k")
+    rows, k = x.shape
+    dev = x.device
+    groups = 0 if offsets is None else offsets.numel() - 1
+    sbytes = nvfp4_scale_bytes(rows, k) if offsets is None else nvfp4_grouped_scale_bytes(rows, groups, k)
+    if out is not None:
+        if out.rows != rows or out.k != k or out.scales.numel() < sbytes or out.global_scale.numel() < max(1, groups):
+            raise ValueError("out does not match the input shape")
+        codes, scales, g = out.codes, out.scales, out.global_scale
+    else:
+        codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty(sbytes, dtype=torch.uint8, device=dev)
+        g = torch.empty(max(1, groups), dtype=torch.float32, device=dev)
+    ws = _workspace(torch, dev, OP_QUANTIZE_ACT, groups)
+    st = nvfp4_quantize_act(_ptr(x), rows, k, x.stride(0), _ptr(offsets), groups, _ptr(codes), _ptr(scales),
+                            _ptr(g), _ptr(ws), _stream_ptr(torch, dev))
+    _check(st, "nvfp4_quantize_act")
+    if out is not None:
+        out.offsets = offsets
+        return out
+    return NVFP4Tensor(codes, scales, g, rows, k, offsets)
+
+
+def quantize_weight_2d(w, compact: bool = False):
+    """16x16-block NVFP4 quantization of a BF16 [n, k] CUDA tensor.  Returns
+    the NVFP4Tensor (and the [n/16, k/16] compact scales when asked)."""
+    import torch
+    if w.dtype != torch.bfloat16 or w.dim() != 2 or not w.is_cuda:
+        raise TypeError("w must be a 2-D bfloat16 CUDA tensor")
+    n, k = w.shape
+    dev = w.device
+    codes = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(nvfp4_scale_bytes(n, k), dtype=torch.uint8, device=dev)
+    sfc = torch.empty((n // 16, k // 16), dtype=torch.uint8, device=dev) if compact else None
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = _workspace(torch, dev, OP_QUANTIZE_WEIGHT_2D)
+    st = nvfp4_quantize_weight_2d(_ptr(w), n, k, w.stride(0), _ptr(codes), _ptr(scales), _ptr(sfc), _ptr(g),
+                                  _ptr(ws), _stream_ptr(torch, dev))
+    _check(st, "nvfp4_quantize_weight_2d")
+    t = NVFP4Tensor(codes, scales, g, n, k)
+    return (t, sfc) if compact else t
+
+
+def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out=None):
+    """C[m, n] = A * B^T of two NVFP4 tensors, BF16 output."""
+    import torch
+    if a.k != b.k:
+        raise ValueError("k mismatch")
+    dev = a.codes.device
+    c = out if out is not None else torch.empty((a.rows, b.rows), dtype=torch.bfloat16, device=dev)
+    st = nvfp4_gemm(_ptr(a.codes), _ptr(a.scales), _ptr(a.global_scale), _ptr(b.codes), _ptr(b.scales),
+                    _ptr(b.global_scale), _ptr(c), c.stride(0), a.rows, b.rows, a.k, None, _stream_ptr(torch, dev))
+    _check(st, "nvfp4_gemm")
+    return c
+
+
+def grouped_gemm(a: NVFP4Tensor, b_codes, b_scales, b_global, n: int, out=None):
+    """Per-expert GEMM: rows of ``a`` grouped by ``a.offsets`` times expert
+    weights ``b_codes`` [E, n, k/2] (scales: E blocks of nvfp4_scale_bytes(n, k))."""
+    import torch
+    if a.offsets is None:
+        raise ValueError("a must be a grouped NVFP4 tensor")
+    dev = a.codes.device
+    E = a.offsets.numel() - 1
+    c = out if out is not None else torch.empty((a.rows, n), dtype=torch.bfloat16, device=dev)
+    st = nvfp4_grouped_gemm(_ptr(a.codes), _ptr(a.scales), _ptr(a.global_scale), _ptr(a.offsets), E,
+                            _ptr(b_codes), _ptr(b_scales), _ptr(b_global), _ptr(c), n, a.k, a.rows, None,
+                            _stream_ptr(torch, dev))
+    _check(st, "nvfp4_grouped_gemm")
+    return c
+
+
+def check_device_error(stream: int = 0) -> None:
+    """Raise if a kernel of the library reported a bounded wait that ran out."""
+    _check(nvfp4_get_last_device_error(stream), "device")

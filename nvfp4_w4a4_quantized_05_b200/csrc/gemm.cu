@@ -1,0 +1,566 @@
+// gemm.cu -- stage 2 of the W4A4 path: block-scaled FP4 x FP4 GEMM on the
+// sm_100a tcgen05 tensor cores.
+//
+//   C[m, n] = bf16_rn( (sum_k qa[m,k] sa[m,k/16] qb[n,k] sb[n,k/16]) * ga * gb )
+//
+// i.e. the product of the two reconstructed NVFP4 operands ("NVFP4 Explained:
+// NVIDIA's 4-Bit Format for Faster AI Inference", "How NVFP4 Represents a
+// Value"): the E2M1 codes and their E4M3 block scales go to the tensor core
+// unchanged (tcgen05.mma .kind::mxf4nvf4, 16-element scale blocks), FP32
+// accumulation stays in tensor memory, and the two FP32 tensor scales are
+// applied once in the epilogue.  No dequantization pass: on Blackwell FP4 x FP4
+// is a native tensor-core mode ("NVFP4 Dynamic Quantization in Practice",
+// "Impact on the Open-Source Community and LLM Deployment Industry"; "W4A8 vs
+// NVFP4 quantization on GPUs", "Dequantization can erase a four-bit win").
+//
+// Kernel structure (one CTA per SM, persistent over output tiles):
+//   warp 0     TMA producer: codes tiles by tensor-map copies (128-byte
+//              swizzle), scale tiles by bulk copies, into a STAGES-deep ring
+//              guarded by mbarriers.  No cluster multicast.
+//   warp 1     allocates tensor memory; one thread moves each stage's scale
+//              tiles to tensor memory (tcgen05.cp) and issues the MMAs
+//              (128 x BN x 64 each), then commits to the stage's "empty"
+//              barrier and, per tile, to the accumulator-full barrier.
+//   warps 2-5  epilogue: tcgen05.ld of the FP32 accumulator, x (ga * gb),
+//              round to BF16, store.
+// Every mbarrier wait is bounded (globaltimer); a wait that runs out sets the
+// library's device error word and the CTA winds down instead of hanging.
+//
+// Operand roles: the "A side" fills the 128-row MMA dimension, the "B side" the
+// BN-wide dimension.  Normally A side = activations, B side = weights; for
+// m <= 64 (decode) they swap so the weights stream through the 128-row side
+// and the few tokens sit in a narrow BN, and the epilogue stores transposed.
+// The grouped form walks (expert, m-tile, n-tile) triples built from the
+// device offsets array.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kSfCol = 256;      // first tensor-memory column of the scale buffers
+constexpr int kMaxStages = 8;
+constexpr int kMaxGroups = 256;
+
+struct GemmArgs {
+    const uint8_t* sfa;        // A-side scales, tiled layout
+    int64_t sfa_rb_stride;     // bytes per 128-row scale block
+    const uint8_t* sfb;        // B-side scales
+    int64_t sfb_rb_stride;
+    int64_t sfb_group_stride;  // bytes between groups' B scales (grouped)
+    int sfb_rb_per_group;      // 128-row scale blocks per B group
+    const float* ga;           // global scales (index = group)
+    const float* gb;
+    __nv_bfloat16* c;
+    int64_t ldc;
+    int rows_a;                // A-side rows (plain) / total rows (grouped)
+    int rows_b;                // B-side rows per group
+    int num_ks;                // k / 64
+    int num_kt;                // ceil(num_ks / 4): k-tiles of 256 elements
+    int tiles_m;               // plain: ceil(rows_a / 128)
+    int tiles_n;               // ceil(rows_b / BN)
+    const int32_t* offsets;    // grouped: [num_groups + 1]
+    int num_groups;
+    uint64_t wait_limit_ns;
+    unsigned int* err;
+};
+
+struct alignas(8) SmemTail {
+    uint64_t full[kMaxStages];
+    uint64_t empty[kMaxStages];
+    uint64_t tmem_full;
+    uint64_t tmem_empty;
+    uint32_t tmem_base;
+    volatile int abort_flag;
+    int total_tiles;
+    int pad_;
+    int tile_prefix[kMaxGroups + 1];
+    int blk_prefix[kMaxGroups + 1];
+};
+
+struct TileInfo {
+    int a_row0;   // tensor-map row of the first A-side row
+    int a_rows;   // valid A-side rows in this tile
+    int sfa_rb;   // A-side 128-row scale block
+    int b_row0;   // tensor-map row of the first B-side row
+    int b_col0;   // index of the first B-side row inside its group
+    int b_rows;   // valid B-side rows
+    int group;
+};
+
+template <int BN, bool GROUPED>
+__device__ __forceinline__ TileInfo tile_info(const GemmArgs& p, const SmemTail* tail, int t) {
+    TileInfo ti;
+    if constexpr (!GROUPED) {
+        const int tm = t % p.tiles_m, tn = t / p.tiles_m;
+        ti.a_row0 = tm * 128;
+        ti.a_rows = min(128, p.rows_a - ti.a_row0);
+        ti.sfa_rb = tm;
+        ti.b_col0 = tn * BN;
+        ti.b_row0 = ti.b_col0;
+        ti.b_rows = min(BN, p.rows_b - ti.b_col0);
+        ti.group = 0;
+    } else {
+        int lo = 0, hi = p.num_groups;   // largest e with tile_prefix[e] <= t
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tail->tile_prefix[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int e = lo;
+        const int r0 = p.offsets[e], n_e = p.offsets[e + 1] - r0;
+        const int mt = (n_e + 127) / 128;
+        const int local = t - tail->tile_prefix[e];
+        const int tm = local % mt, tn = local / mt;
+        ti.a_row0 = r0 + tm * 128;
+        ti.a_rows = min(128, n_e - tm * 128);
+        ti.sfa_rb = tail->blk_prefix[e] + tm;
+        ti.b_col0 = tn * BN;
+        ti.b_row0 = e * p.rows_b + ti.b_col0;
+        ti.b_rows = min(BN, p.rows_b - ti.b_col0);
+        ti.group = e;
+    }
+    return ti;
+}
+
+__device__ __forceinline__ void raise_abort(SmemTail* tail, unsigned int* err) {
+    tail->abort_flag = 1;
+    if (err) atomicOr(err, 1u);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int BN, int STAGES, bool SWAP, bool GROUPED>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+    constexpr int NRB = BN >= 128 ? BN / 128 : 1;          // 128-row scale blocks on the B side
+    constexpr uint32_t A_BYTES = 128 * 128;                  // 128 rows x 256 FP4
+    constexpr uint32_t B_BYTES = BN * 128;
+    constexpr uint32_t SFA_BYTES = 4 * 512;                  // 4 k-steps x (128 rows x 4 scales)
+    constexpr uint32_t SFB_BYTES = NRB * 4 * 512;
+    constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    constexpr uint32_t SF_COLS = 16 + 16 * NRB;              // tensor-memory columns per k-tile of scales
+    constexpr int CW = BN >= 32 ? 32 : 16;                   // epilogue column chunk
+    constexpr uint32_t IDESC = idesc_mxf4nvf4(128, BN);
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
+    static_assert(STAGES <= kMaxStages, "stages");
+    static_assert(kSfCol + 2 * SF_COLS <= kTmemCols, "tensor memory budget");
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static_assert(!(SWAP && GROUPED), "swap form is for the plain GEMM");
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + STAGES * STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&tail->full[s], 1);
+            mbar_init(&tail->empty[s], 1);
+        }
+        mbar_init(&tail->tmem_full, 1);
+        mbar_init(&tail->tmem_empty, 4);
+        tail->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tail->tmem_base, kTmemCols);
+        tmem_relinquish();
+    }
+    // Everything read below (codes, scales, global scales, offsets) may be
+    // written by the previous kernel in the stream.
+    pdl_wait();
+    if constexpr (GROUPED) {
+        if (warp == 2) {
+            const int E = p.num_groups;
+            const int per = (E + 31) / 32;
+            int t_loc = 0, b_loc = 0;
+            for (int i = 0; i < per; ++i) {
+                const int e = lane * per + i;
+                if (e < E) {
+                    const int mt = (p.offsets[e + 1] - p.offsets[e] + 127) / 128;
+                    t_loc += mt * p.tiles_n;
+                    b_loc += mt;
+                }
+            }
+            int t_inc = t_loc, b_inc = b_loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int tv = __shfl_up_sync(0xFFFFFFFFu, t_inc, o);
+                const int bv = __shfl_up_sync(0xFFFFFFFFu, b_inc, o);
+                if (lane >= o) {
+                    t_inc += tv;
+                    b_inc += bv;
+                }
+            }
+            int t_run = t_inc - t_loc, b_run = b_inc - b_loc;
+            for (int i = 0; i < per; ++i) {
+                const int e = lane * per + i;
+                if (e < E) {
+                    tail->tile_prefix[e] = t_run;
+                    tail->blk_prefix[e] = b_run;
+                    const int mt = (p.offsets[e + 1] - p.offsets[e] + 127) / 128;
+                    t_run += mt * p.tiles_n;
+                    b_run += mt;
+                }
+            }
+            if (lane == 31) {
+                tail->tile_prefix[E] = t_inc;
+                tail->blk_prefix[E] = b_inc;
+                tail->total_tiles = t_inc;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = tail->tmem_base;
+    const int total_tiles = GROUPED ? tail->total_tiles : p.tiles_m * p.tiles_n;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer ----------------
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+                const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
+                const uint8_t* sfa_src = p.sfa + (int64_t)ti.sfa_rb * p.sfa_rb_stride;
+                const uint8_t* sfb_src = p.sfb + (int64_t)ti.group * p.sfb_group_stride +
+                                         (int64_t)(ti.b_col0 / 128) * p.sfb_rb_stride;
+                const int nsfb = min(NRB, p.sfb_rb_per_group - ti.b_col0 / 128);
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    const int nat = min(4, p.num_ks - kt * 4);
+                    uint8_t* sA = smem + stage * STAGE_BYTES;
+                    uint8_t* sB = sA + A_BYTES;
+                    uint8_t* sSFA = sB + B_BYTES;
+                    uint8_t* sSFB = sSFA + SFA_BYTES;
+                    uint64_t* bar = &tail->full[stage];
+                    mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES + (uint32_t)nat * 512u * (1u + (uint32_t)nsfb));
+                    tma_load_2d(sA, &tmA, bar, kt * 128, ti.a_row0);
+                    tma_load_2d(sB, &tmB, bar, kt * 128, ti.b_row0);
+                    bulk_load(sSFA, sfa_src + (int64_t)kt * 2048, (uint32_t)nat * 512u, bar);
+                    for (int rb = 0; rb < nsfb; ++rb)
+                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * 2048,
+                                  (uint32_t)nat * 512u, bar);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) raise_abort(tail, p.err);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------- MMA issuer ----------------
+            uint32_t stage = 0, phase = 0, ktg = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
+                if (!mbar_wait(&tail->tmem_empty, (uint32_t)(it & 1) ^ 1u, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kt = 0; kt < p.num_kt; ++kt, ++ktg) {
+                    if (!mbar_wait(&tail->full[stage], phase, limit) || tail->abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nat = min(4, p.num_ks - kt * 4);
+                    const uint32_t sA = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t sB = sA + A_BYTES;
+                    const uint32_t sSFA = sB + B_BYTES;
+                    const uint32_t sSFB = sSFA + SFA_BYTES;
+                    const uint32_t sf = tmem + kSfCol + (ktg & 1u) * SF_COLS;
+                    for (int j = 0; j < nat; ++j) tmem_cp_32x128b_x4(sf + j * 4, sdesc_sf_block(sSFA + j * 512));
+                    for (int rb = 0; rb < NRB; ++rb)
+                        for (int j = 0; j < nat; ++j)
+                            tmem_cp_32x128b_x4(sf + 16 + j * 4 * NRB + rb * 4,
+                                               sdesc_sf_block(sSFB + rb * 2048 + j * 512));
+                    for (int j = 0; j < nat; ++j)
+                        mma_mxf4nvf4(tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32), IDESC,
+                                     sf + j * 4, sf + 16 + j * 4 * NRB, (kt > 0 || j > 0) ? 1u : 0u);
+                    tc_commit(&tail->empty[stage]);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (ok) tc_commit(&tail->tmem_full);
+            }
+            if (!ok) raise_abort(tail, p.err);
+        }
+    } else {
+        // ---------------- epilogue (warps 2..5) ----------------
+        const int q = warp & 3;                       // tensor-memory lane quarter of this warp
+        const int rloc = q * 32 + lane;               // A-side row inside the tile
+        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+        int it = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
+            const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
+            if (!mbar_wait(&tail->tmem_full, (uint32_t)(it & 1), limit) || tail->abort_flag) {
+                if (lane == 0) raise_abort(tail, p.err);
+                break;
+            }
+            tc_fence_after();
+            const float alpha = __fmul_rn(p.ga[ti.group], p.gb[ti.group]);
+            const bool a_ok = rloc < ti.a_rows;
+#pragma unroll 1
+            for (int ch = 0; ch < BN / CW; ++ch) {
+                uint32_t v[CW];
+                if constexpr (CW == 32) {
+                    tmem_ld_32x32b_x32(tq + ch * CW, v);
+                } else {
+                    tmem_ld_32x32b_x16(tq + ch * CW, v);
+                }
+                tmem_ld_wait();
+                if constexpr (!SWAP) {
+                    if (a_ok) {
+                        __nv_bfloat16* crow = p.c + (int64_t)(ti.a_row0 + rloc) * p.ldc + ti.b_col0 + ch * CW;
+                        const int ncols = ti.b_rows - ch * CW;
+                        if (ncols >= CW) {
+#pragma unroll
+                            for (int i = 0; i < CW; i += 8) {
+                                uint4 w;
+                                w.x = pack_bf16x2(__uint_as_float(v[i + 0]) * alpha, __uint_as_float(v[i + 1]) * alpha);
+                                w.y = pack_bf16x2(__uint_as_float(v[i + 2]) * alpha, __uint_as_float(v[i + 3]) * alpha);
+                                w.z = pack_bf16x2(__uint_as_float(v[i + 4]) * alpha, __uint_as_float(v[i + 5]) * alpha);
+                                w.w = pack_bf16x2(__uint_as_float(v[i + 6]) * alpha, __uint_as_float(v[i + 7]) * alpha);
+                                *reinterpret_cast<uint4*>(crow + i) = w;
+                            }
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < CW; ++i)
+                                if (i < ncols) crow[i] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
+                        }
+                    }
+                } else {
+                    if (a_ok) {
+                        const int n = ti.a_row0 + rloc;
+#pragma unroll
+                        for (int i = 0; i < CW; ++i) {
+                            const int m = ti.b_col0 + ch * CW + i;
+                            if (ch * CW + i < ti.b_rows)
+                                p.c[(int64_t)m * p.ldc + n] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tail->tmem_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ---- host side -----------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 2-D uint8 view [rows, row_bytes] of packed codes, 128-byte x box_rows boxes,
+// 128-byte swizzle, zero fill outside the tensor.
+bool make_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t row_bytes, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {128u, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES, bool SWAP, bool GROUPED>
+nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid, cudaStream_t s) {
+    constexpr int NRB = BN >= 128 ? BN / 128 : 1;
+    constexpr size_t stage = 128 * 128 + BN * 128 + 2048 + NRB * 2048;
+    constexpr size_t smem = 1024 + STAGES * stage + sizeof(SmemTail);
+    static_assert(smem <= 232448, "shared memory");
+    auto kern = gemm_kernel<BN, STAGES, SWAP, GROUPED>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    });
+    if (attr_err != cudaSuccess) return NVFP4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
+}
+
+bool ptr_ok(const void* p) { return p && aligned16(p); }
+
+}  // namespace
+}  // namespace nvfp4
+
+using namespace nvfp4;
+
+extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                                     const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c,
+                                     int64_t ldc, int64_t m, int64_t n, int64_t k, void* workspace, void* stream) {
+    (void)workspace;
+    if (m < 0 || n <= 0 || k <= 0 || ldc < n) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !c)
+        return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 64 != 0 || m >= ((int64_t)1 << 31) || n >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!ptr_ok(a_codes) || !ptr_ok(a_scales) || !ptr_ok(b_codes) || !ptr_ok(b_scales) || !ptr_ok(c) ||
+        (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(b_global) & 3u) || ldc % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (m == 0) return NVFP4_OK;
+    const int sms = num_sms();
+    if (sms <= 0) return NVFP4_ERR_NO_DEVICE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int64_t sf_rb_stride = 128 * (k / 16);
+    GemmArgs p = {};
+    p.num_ks = (int)(k / 64);
+    p.num_kt = (p.num_ks + 3) / 4;
+    p.c = reinterpret_cast<__nv_bfloat16*>(c);
+    p.ldc = ldc;
+    p.sfa_rb_stride = sf_rb_stride;
+    p.sfb_rb_stride = sf_rb_stride;
+    p.sfb_group_stride = 0;
+    p.offsets = nullptr;
+    p.num_groups = 1;
+    p.wait_limit_ns = wait_limit_ns();
+    p.err = device_error_word();
+    if (!p.err) return NVFP4_ERR_CUDA;
+    CUtensorMap ta, tb;
+    if (m <= 64) {
+        // decode: weights on the 128-row side, tokens on the narrow side
+        const int bn = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
+        if (!make_codes_map(&ta, b_codes, n, k / 2, 128) || !make_codes_map(&tb, a_codes, m, k / 2, bn))
+            return NVFP4_ERR_CUDA;
+        p.sfa = b_scales;
+        p.sfb = a_scales;
+        p.sfb_rb_per_group = (int)((m + 127) / 128);
+        p.ga = b_global;
+        p.gb = a_global;
+        p.rows_a = (int)n;
+        p.rows_b = (int)m;
+        p.tiles_m = (int)((n + 127) / 128);
+        p.tiles_n = 1;
+        const int grid = (int)std::min<int64_t>(p.tiles_m, sms);
+        if (bn == 16) return launch<16, 7, true, false>(ta, tb, p, grid, s);
+        if (bn == 32) return launch<32, 7, true, false>(ta, tb, p, grid, s);
+        return launch<64, 7, true, false>(ta, tb, p, grid, s);
+    }
+    constexpr int BN = 256;
+    if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN))
+        return NVFP4_ERR_CUDA;
+    p.sfa = a_scales;
+    p.sfb = b_scales;
+    p.sfb_rb_per_group = (int)((n + 127) / 128);
+    p.ga = a_global;
+    p.gb = b_global;
+    p.rows_a = (int)m;
+    p.rows_b = (int)n;
+    p.tiles_m = (int)((m + 127) / 128);
+    p.tiles_n = (int)((n + BN - 1) / BN);
+    const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
+    if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int grid = (int)std::min<int64_t>(tiles, sms);
+    return launch<BN, 4, false, false>(ta, tb, p, grid, s);
+}
+
+extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                                             const int32_t* offsets, int num_experts, const uint8_t* b_codes,
+                                             const uint8_t* b_scales, const float* b_global, void* c, int64_t n,
+                                             int64_t k, int64_t total_rows, void* workspace, void* stream) {
+    (void)workspace;
+    if (num_experts < 1 || n <= 0 || k <= 0 || total_rows < 0) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (!a_codes || !a_scales || !a_global || !offsets || !b_codes || !b_scales || !b_global || !c)
+        return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 64 != 0 || num_experts > kMaxGroups || total_rows >= ((int64_t)1 << 31) ||
+        n * (int64_t)num_experts >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!ptr_ok(a_codes) || !ptr_ok(a_scales) || !ptr_ok(b_codes) || !ptr_ok(b_scales) || !ptr_ok(c) ||
+        (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(b_global) & 3u) ||
+        (reinterpret_cast<uintptr_t>(offsets) & 3u) || n % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (total_rows == 0) return NVFP4_OK;
+    const int sms = num_sms();
+    if (sms <= 0) return NVFP4_ERR_NO_DEVICE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    constexpr int BN = 256;
+    const int64_t sf_rb_stride = 128 * (k / 16);
+    GemmArgs p = {};
+    p.num_ks = (int)(k / 64);
+    p.num_kt = (p.num_ks + 3) / 4;
+    p.c = reinterpret_cast<__nv_bfloat16*>(c);
+    p.ldc = n;
+    p.sfa = a_scales;
+    p.sfa_rb_stride = sf_rb_stride;
+    p.sfb = b_scales;
+    p.sfb_rb_stride = sf_rb_stride;
+    p.sfb_group_stride = (int64_t)nvfp4_scale_bytes(n, k);
+    p.sfb_rb_per_group = (int)((n + 127) / 128);
+    p.ga = a_global;
+    p.gb = b_global;
+    p.rows_a = (int)total_rows;
+    p.rows_b = (int)n;
+    p.tiles_m = 0;
+    p.tiles_n = (int)((n + BN - 1) / BN);
+    p.offsets = offsets;
+    p.num_groups = num_experts;
+    p.wait_limit_ns = wait_limit_ns();
+    p.err = device_error_word();
+    if (!p.err) return NVFP4_ERR_CUDA;
+    CUtensorMap ta, tb;
+    if (!make_codes_map(&ta, a_codes, total_rows, k / 2, 128) ||
+        !make_codes_map(&tb, b_codes, n * num_experts, k / 2, BN))
+        return NVFP4_ERR_CUDA;
+    // upper bound of the tile count: sum_e ceil(n_e / 128) <= total_rows / 128 + num_experts
+    const int64_t max_tiles = (total_rows / 128 + num_experts) * (int64_t)p.tiles_n;
+    const int grid = (int)std::min<int64_t>(max_tiles, sms);
+    return launch<BN, 4, false, true>(ta, tb, p, grid, s);
+}

@@ -1,0 +1,35 @@
+// internal.h -- host-side helpers shared by the translation units of libnvfp4.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "../../include/nvfp4.h"
+
+namespace nvfp4 {
+
+// Device address of this library's error word on the current device
+// (nonzero after a bounded wait in a kernel ran out).  nullptr on failure.
+unsigned int* device_error_word();
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+// Current limit of the bounded waits, in ns.
+uint64_t wait_limit_ns();
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+inline nvfp4_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+
+// Workspace layout of the quantizers (bytes):
+//   [0, 4)         CTA completion counter (uint32)
+//   [16, 16+4G)    per-group amax as FP32 bit patterns (uint32)
+//   [pad_off, +4(G+1))  per-group first scale row (int32), written each call
+inline int64_t quant_ws_amax_off() { return 16; }
+inline int64_t quant_ws_pad_off(int groups) { return round_up(16 + 4 * (int64_t)groups, 16); }
+inline int64_t quant_ws_bytes(int groups) { return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 256); }
+
+}  // namespace nvfp4

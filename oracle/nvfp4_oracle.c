@@ -12,6 +12,7 @@
  */
 #include "nvfp4_oracle.h"
 
+#include <float.h>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -136,6 +137,7 @@ static uint8_t quantize_block(const float* xv, int n, float bamax, float g, uint
     uint8_t sf = orc_e4m3_encode(bamax / k6);
     float d = (float)orc_e4m3_decode(sf) * g;      /* decoded block scale times g */
     float r = (d == 0.0f) ? 0.0f : 1.0f / d;
+    if (r > FLT_MAX) r = FLT_MAX;                   /* 1/d overflows only when g is subnormal */
     for (int i = 0; i < n; ++i) code_out[i] = orc_e2m1_encode(xv[i] * r);
     return sf;
 }

@@ -27,7 +27,7 @@
  * Readings where the pages are silent (each listed in the design notes):
  *   g  = amax / (6 * 448) as a decode multiplier (1.0 when amax == 0);
  *   sf = E4M3_RNE_satfinite(block_amax / (6 * g));
- *   d  = decode(sf) * g;  r = (d == 0) ? 0 : 1 / d;
+ *   d  = decode(sf) * g;  r = (d == 0) ? 0 : min(1 / d, FLT_MAX);
  *   code = E2M1_RNE_satfinite(x * r), sign bit kept (also for zero);
  *   element 2i in bits 3:0 of byte i, element 2i+1 in bits 7:4;
  *   scales stored in 128-row x 4-column tiles of 512 bytes (tensor-core

@@ -1,0 +1,170 @@
+"""GPU GEMM parity: the tcgen05 block-scaled GEMM against the binary64 oracle
+GEMM over the reconstructed operands, within the stated tolerance
+(relative Frobenius <= 2e-3, max |error| <= 1e-2 x row max |ref|).  Small
+cases compare every output; the full-size prefill / decode / MoE workloads
+compare sampled rows the oracle computes one by one."""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+import nvfp4_w4a4_quantized_05_b200 as nv
+from gpu_util import assert_gemm_close, bf16_to_device, nvfp4_from_host, to_host_f64
+
+pytestmark = pytest.mark.gpu
+
+
+def _sync():
+    import torch
+    torch.cuda.synchronize()
+    nv.check_device_error()
+
+
+def _oracle_operands(m, n, k, seed):
+    a = W.gaussian_bf16((m, k), seed, 300 + m, 1.0, outlier_frac=0.01)
+    w = W.gaussian_bf16((n, k), seed, 301 + n, 0.02)
+    qa = O.quantize_1d(a)
+    qw = O.quantize_2d(w) if n % 16 == 0 else O.quantize_1d(w)
+    return qa, qw
+
+
+def test_tiny_workload_end_to_end():
+    a, w = W.tiny(0)
+    ta = nv.quantize_act(bf16_to_device(a))
+    tw = nv.quantize_weight_2d(bf16_to_device(w))
+    c = nv.gemm(ta, tw)
+    _sync()
+    ac, asf, ga = O.quantize_1d(a)
+    wc, wsf, gw = O.quantize_2d(w)
+    assert np.array_equal(ta.codes.cpu().numpy(), ac) and np.array_equal(tw.codes.cpu().numpy(), wc)
+    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    got = to_host_f64(c)
+    assert_gemm_close(got, ref, "tiny")
+    # the exact integer sum, scaled, rounds to within one BF16 step of the output
+    exact = O.gemm_exact_i64(ac, asf, wc, wsf, 256).astype(np.float64) * 2.0 ** -20 * float(np.float32(ga) * np.float32(gw))
+    assert np.all(np.abs(got - exact) <= 2.0 ** -7 * np.abs(exact) + 1e-30)
+
+
+@pytest.mark.parametrize("m,n,k", [
+    (128, 256, 256),     # one full tile
+    (200, 320, 320),     # ragged m, ragged n tile, partial last k-tile
+    (256, 512, 1024),    # several tiles
+    (65, 200, 64),       # smallest k; just above the swap threshold
+    (64, 200, 128),      # swap path, BN 64
+    (33, 304, 192),      # swap path, BN 64 with 33 tokens
+    (17, 136, 64),       # swap path, BN 32
+    (16, 64, 256),       # swap path, BN 16
+    (1, 64, 320),        # single token
+    (300, 16, 448),      # narrow n
+])
+def test_gemm_matches_oracle(m, n, k):
+    (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 0)
+    c = nv.gemm(nvfp4_from_host(ac, asf, ga), nvfp4_from_host(wc, wsf, gw))
+    _sync()
+    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    assert_gemm_close(to_host_f64(c), ref, f"{m}x{n}x{k}")
+
+
+def test_gemm_output_row_stride():
+    import torch
+    (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(150, 96, 128, 1)
+    out = torch.full((150, 136), 7.0, dtype=torch.bfloat16, device="cuda")
+    nv.gemm(nvfp4_from_host(ac, asf, ga), nvfp4_from_host(wc, wsf, gw), out=out[:, :96])
+    _sync()
+    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    assert_gemm_close(to_host_f64(out[:, :96]), ref, "strided")
+    assert torch.all(out[:, 96:] == 7.0)                  # nothing written past n
+
+
+@pytest.fixture(scope="module")
+def prefill_case():
+    a, w = W.prefill(0)
+    return a, w, O.quantize_1d(a), O.quantize_2d(w)
+
+
+def test_prefill_workload_sampled_rows(prefill_case):
+    a, w, (ac, asf, ga), (wc, wsf, gw) = prefill_case
+    ta = nv.quantize_act(bf16_to_device(a))
+    tw = nv.quantize_weight_2d(bf16_to_device(w))
+    c = nv.gemm(ta, tw)
+    _sync()
+    rows = np.unique(np.concatenate([np.arange(0, 4096, 128), np.arange(127, 4096, 128)[::4], [1, 2049, 4095]]))
+    ah = O.dequantize(ac, asf, ga)[rows]
+    wh = O.dequantize(wc, wsf, gw)
+    ref = O.gemm_f64(ah, wh)
+    got = to_host_f64(c[rows.tolist()])
+    assert_gemm_close(got, ref, "prefill")
+
+
+@pytest.fixture(scope="module")
+def decode_weights():
+    _, w = W.decode(1)
+    wc, wsf, gw = O.quantize_2d(w)
+    return w, (wc, wsf, gw), O.dequantize(wc, wsf, gw)
+
+
+@pytest.mark.parametrize("m", [1, 8, 32, 64])
+def test_decode_workload_full(m, decode_weights):
+    w, (wc, wsf, gw), wh = decode_weights
+    a, _ = W.decode(m)
+    ac, asf, ga = O.quantize_1d(a)
+    ta = nv.quantize_act(bf16_to_device(a))
+    c = nv.gemm(ta, nvfp4_from_host(wc, wsf, gw))
+    _sync()
+    assert np.array_equal(ta.codes.cpu().numpy(), ac)
+    ref = O.gemm_f64(O.dequantize(ac, asf, ga), wh)
+    assert_gemm_close(to_host_f64(c), ref, f"decode m={m}")
+
+
+def test_grouped_gemm_ragged_experts():
+    sizes = [0, 5, 128, 130, 0, 1, 257, 64]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    k, n = 320, 200
+    a = W.gaussian_bf16((int(off[-1]), k), 0, 44, 1.0, outlier_frac=0.01)
+    ac, asf, ga = O.quantize_1d_grouped(a, off)
+    E = len(sizes)
+    wq = [O.quantize_1d(W.gaussian_bf16((n, k), 0, 500 + e, 0.02)) for e in range(E)]
+    wc = np.stack([q[0] for q in wq])
+    wsf = np.concatenate([q[1] for q in wq])
+    gw = np.array([q[2] for q in wq], np.float32)
+    ta = nvfp4_from_host(ac, np.concatenate([asf, np.zeros(nv.nvfp4_grouped_scale_bytes(int(off[-1]), E, k) - asf.size, np.uint8)]), ga, off)
+    from gpu_util import u8_to_device
+    import torch
+    c = nv.grouped_gemm(ta, u8_to_device(wc), u8_to_device(wsf), torch.tensor(gw, device="cuda"), n)
+    _sync()
+    ah = O.dequantize_grouped(ac, asf, ga, off)
+    got = to_host_f64(c)
+    for e in range(E):
+        r0, r1 = off[e], off[e + 1]
+        if r1 > r0:
+            ref = O.gemm_f64(ah[r0:r1], O.dequantize(wq[e][0], wq[e][1], wq[e][2]))
+            assert_gemm_close(got[r0:r1], ref, f"expert {e}")
+
+
+def test_moe_workload_sampled_rows():
+    import torch
+    a, off, w = W.moe(0)
+    E, N, K = w.shape
+    ta = nv.quantize_act(bf16_to_device(a), torch.from_numpy(off).cuda())
+    wdev = bf16_to_device(w.reshape(E * N, K))
+    tw = [nv.quantize_weight_2d(wdev[e * N:(e + 1) * N]) for e in range(E)]
+    b_codes = torch.stack([t.codes for t in tw])
+    b_scales = torch.cat([t.scales for t in tw])
+    b_global = torch.cat([t.global_scale for t in tw])
+    c = nv.grouped_gemm(ta, b_codes, b_scales, b_global, N)
+    _sync()
+    ac, asf, ga = O.quantize_1d_grouped(a, off)
+    assert np.array_equal(ta.codes.cpu().numpy(), ac)
+    wc_all, wsf_all, gw_all = b_codes.cpu().numpy(), b_scales.cpu().numpy(), b_global.cpu().numpy()
+    sbytes = nv.nvfp4_scale_bytes(N, K)
+    row0 = 0
+    got = to_host_f64(c)
+    for e in range(E):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        n_e = r1 - r0
+        if n_e:
+            sel = np.unique([r0, r0 + n_e // 2, r1 - 1, min(r1 - 1, r0 + 127), min(r1 - 1, r0 + 128)])
+            a_hat = O.dequantize(ac[r0:r1], asf, float(ga[e]), sf_row0=row0, k=K)[sel - r0]
+            w_hat = O.dequantize(wc_all[e], wsf_all[e * sbytes:(e + 1) * sbytes], float(gw_all[e]))
+            assert_gemm_close(got[sel], O.gemm_f64(a_hat, w_hat), f"moe expert {e}")
+        row0 += O.scale_rows(n_e)

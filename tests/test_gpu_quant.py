@@ -1,0 +1,194 @@
+"""GPU quantizer parity: codes, scale bytes (whole buffer, pads included) and
+global scales must equal the CPU oracle bit for bit on the same seeded
+inputs; the hardware conversions must equal the oracle's encoders over wide
+binary32 sweeps.  Calls go through the C ABI (via the thin binding)."""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+import nvfp4_w4a4_quantized_05_b200 as nv
+from gpu_util import bf16_to_device, device
+
+pytestmark = pytest.mark.gpu
+
+
+def _gpu_q1d(xb, offsets=None):
+    import torch
+    x = bf16_to_device(xb)
+    off = None if offsets is None else torch.from_numpy(np.asarray(offsets, np.int32)).to(device())
+    q = nv.quantize_act(x, off)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    return q.codes.cpu().numpy(), q.scales.cpu().numpy(), q.global_scale.cpu().numpy()
+
+
+def _assert_same_1d(xb):
+    c, s, g = _gpu_q1d(xb)
+    oc, osf, og = O.quantize_1d(xb)
+    assert np.float32(og).view(np.uint32) == g[0].view(np.uint32), (og, g[0])
+    assert s.size == osf.size
+    bad = np.nonzero(c != oc)
+    assert bad[0].size == 0, f"{bad[0].size} code bytes differ, first at {bad[0][0]},{bad[1][0]}"
+    badsf = np.nonzero(s != osf)[0]
+    assert badsf.size == 0, f"{badsf.size} scale bytes differ, first at {badsf[:4]}"
+
+
+# ---- hardware conversions vs the oracle's encoders ----------------------------------
+
+def _sweep_compare(lo_pattern, hi_pattern, step, which):
+    import torch
+    chunk = 1 << 26
+    for start in range(lo_pattern, hi_pattern, chunk * step):
+        stop = min(hi_pattern, start + chunk * step)
+        pats = np.arange(start, stop, step, dtype=np.uint64).astype(np.uint32)
+        vals = pats.view(np.float32)
+        x = torch.from_numpy(pats.view(np.int32)).to(device()).view(torch.float32)
+        out = torch.empty(vals.size, dtype=torch.uint8, device=device())
+        if which == "e2m1":
+            st = nv.nvfp4_probe_cvt(x.data_ptr(), out.data_ptr(), None, vals.size)
+            want = O.e2m1_encode_array(vals)
+        else:
+            st = nv.nvfp4_probe_cvt(x.data_ptr(), None, out.data_ptr(), vals.size)
+            want = O.e4m3_encode_array(np.abs(vals))
+        assert st == 0
+        got = out.cpu().numpy()
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, (f"{which}: {bad.size} mismatches in [{start:#x},{stop:#x}); first value "
+                               f"{vals[bad[0]]!r} hw {got[bad[0]]:#x} oracle {want[bad[0]]:#x}")
+
+
+def test_cvt_e2m1_every_pattern_below_8():
+    _sweep_compare(0, 0x41000001, 1, "e2m1")                    # every +0 .. 8.0
+    _sweep_compare(0x80000000, 0xC1000001, 1, "e2m1")          # every -0 .. -8.0
+
+
+def test_cvt_e2m1_large_and_sign_sample():
+    _sweep_compare(0x41000000, 0x7F800000, 257, "e2m1")        # 8 .. FLT_MAX, sampled
+    _sweep_compare(0xC1000000, 0xFF800000, 263, "e2m1")
+
+
+def test_cvt_e4m3_every_pattern_below_1024():
+    _sweep_compare(0, 0x44800001, 1, "e4m3")
+    _sweep_compare(0x44800000, 0x7F800000, 251, "e4m3")        # saturating range, sampled
+
+
+# ---- 1D activations ------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(16, 256), (1, 16), (3, 48), (130, 320), (257, 4112), (64, 5120), (1, 5120)])
+def test_quantize_act_matches_oracle(shape):
+    xb = W.gaussian_bf16(shape, 0, 100 + shape[0], 1.0, outlier_frac=0.01)
+    _assert_same_1d(xb)
+
+
+def test_quantize_act_full_activation_workload():
+    _assert_same_1d(W.quant_act(0))          # [8192, 4096] Laplace + 0.1% +-U[50,200]
+
+
+def test_quantize_act_prefill_activations():
+    a, _ = W.prefill(0, n=16)
+    _assert_same_1d(a)                       # [4096, 4096] N(0,1)
+
+
+@pytest.mark.parametrize("case", ["zeros", "signed_zeros", "constant", "subnormal", "huge", "tiny_and_huge"])
+def test_quantize_act_edge_values(case):
+    rng = np.random.default_rng(7)
+    shape = (40, 96)
+    n = shape[0] * shape[1]
+    if case == "zeros":
+        xb = np.zeros(shape, np.uint16)
+    elif case == "signed_zeros":
+        xb = (rng.integers(0, 2, size=shape) * 0x8000).astype(np.uint16)
+    elif case == "constant":
+        xb = np.full(shape, 0x3FC0, np.uint16)          # 1.5
+    elif case == "subnormal":
+        xb = (rng.integers(1, 0x80, size=n) | (rng.integers(0, 2, size=n) << 15)).astype(np.uint16).reshape(shape)
+    elif case == "huge":
+        xb = (rng.integers(0x7F00, 0x7F80, size=n) | (rng.integers(0, 2, size=n) << 15)).astype(np.uint16).reshape(shape)
+    else:
+        lo = rng.integers(1, 0x0100, size=n)
+        hi = rng.integers(0x7E00, 0x7F80, size=n)
+        pick = rng.random(n) < 0.02
+        xb = np.where(pick, hi, lo).astype(np.uint16).reshape(shape)
+    _assert_same_1d(xb)
+
+
+def test_quantize_act_strided_rows():
+    import torch
+    wide = W.gaussian_bf16((70, 384), 0, 41, 1.0, outlier_frac=0.01)
+    x = bf16_to_device(wide)[:, :320]                   # ld = 384 > k = 320
+    q = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    oc, osf, og = O.quantize_1d(np.ascontiguousarray(wide[:, :320]))
+    assert np.array_equal(q.codes.cpu().numpy(), oc)
+    assert np.array_equal(q.scales.cpu().numpy(), osf)
+    assert q.global_scale.cpu().numpy()[0] == np.float32(og)
+
+
+def test_workspace_left_zero_and_reusable():
+    import torch
+    xb = W.gaussian_bf16((300, 512), 0, 42, 1.0)
+    x = bf16_to_device(xb)
+    dev = device()
+    ws = torch.zeros(nv.nvfp4_workspace_bytes(nv.OP_QUANTIZE_ACT), dtype=torch.uint8, device=dev)
+    codes = torch.empty((300, 256), dtype=torch.uint8, device=dev)
+    scales = torch.empty(nv.nvfp4_scale_bytes(300, 512), dtype=torch.uint8, device=dev)
+    g = torch.empty(1, dtype=torch.float32, device=dev)
+    for _ in range(3):
+        st = nv.nvfp4_quantize_act(x.data_ptr(), 300, 512, 512, None, 0, codes.data_ptr(), scales.data_ptr(),
+                                   g.data_ptr(), ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert int(ws[:16].abs().sum()) == 0 and int(ws.sum()) == 0
+    oc, osf, og = O.quantize_1d(xb)
+    assert np.array_equal(codes.cpu().numpy(), oc) and np.array_equal(scales.cpu().numpy(), osf)
+
+
+# ---- grouped (MoE) ---------------------------------------------------------------------
+
+def _assert_same_grouped(xb, off):
+    c, s, g = _gpu_q1d(xb, off)
+    oc, osf, og = O.quantize_1d_grouped(xb, off)
+    assert np.array_equal(g.view(np.uint32), og.view(np.uint32))
+    assert np.array_equal(c, oc)
+    assert s.size >= osf.size
+    bad = np.nonzero(s[:osf.size] != osf)[0]
+    assert bad.size == 0, f"{bad.size} scale bytes differ, first at {bad[:4]}"
+
+
+def test_grouped_quantize_ragged_groups():
+    sizes = [0, 5, 128, 130, 0, 1, 257, 64]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    xb = W.gaussian_bf16((int(off[-1]), 2048), 0, 43, 1.0, outlier_frac=0.01)
+    _assert_same_grouped(xb, off)
+
+
+def test_grouped_quantize_moe_workload():
+    a, off, _ = W.moe(0, with_weights=False)        # [32768, 2048], 128 experts, top-8 routing
+    _assert_same_grouped(a, off)
+
+
+# ---- 2D weights --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("shape", [(64, 256), (16, 16), (48, 80), (272, 4112)])
+def test_quantize_weight_2d_matches_oracle(shape):
+    import torch
+    wb = W.gaussian_bf16(shape, 0, 200 + shape[0], 0.02)
+    t, sfc = nv.quantize_weight_2d(bf16_to_device(wb), compact=True)
+    torch.cuda.synchronize()
+    oc, osf, og, osfc = O.quantize_2d(wb, compact=True)
+    assert t.global_scale.cpu().numpy()[0] == np.float32(og)
+    assert np.array_equal(t.codes.cpu().numpy(), oc)
+    assert np.array_equal(t.scales.cpu().numpy(), osf)
+    assert np.array_equal(sfc.cpu().numpy(), osfc)
+
+
+def test_quantize_weight_2d_full_weight_workload():
+    import torch
+    wb = W.quant_weight(0)                          # [14336, 4096] N(0, 0.02)
+    t = nv.quantize_weight_2d(bf16_to_device(wb))
+    torch.cuda.synchronize()
+    oc, osf, og = O.quantize_2d(wb)
+    assert t.global_scale.cpu().numpy()[0] == np.float32(og)
+    assert np.array_equal(t.codes.cpu().numpy(), oc)
+    assert np.array_equal(t.scales.cpu().numpy(), osf)

@@ -23,6 +23,8 @@ Workloads (sizes from the LLM shapes the pages discuss):
 """
 from __future__ import annotations
 
+import os
+
 import numpy as np
 
 _GAMMA = np.uint64(0x9E3779B97F4A7C15)
@@ -51,21 +53,60 @@ def splitmix64(seed: int, stream: int, n: int, start: int = 0) -> np.ndarray:
         return _mix(s + ctr * _GAMMA)
 
 
-def uniform(seed: int, stream: int, n: int) -> np.ndarray:
-    """Uniform doubles in the open interval (0, 1)."""
-    z = splitmix64(seed, stream, n)
+_CHUNK = 1 << 20
+_POOL = None
+
+
+def _pool():
+    global _POOL
+    if _POOL is None:
+        from concurrent.futures import ThreadPoolExecutor
+        _POOL = ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1))
+    return _POOL
+
+
+def _chunked(n: int, fill) -> np.ndarray:
+    """out[i] for i in [0, n), computed chunk by chunk (counter-based, so the
+    result does not depend on the chunking) on a thread pool."""
+    out = np.empty(n, np.float64)
+    starts = range(0, n, _CHUNK)
+    list(_pool().map(lambda s0: fill(out, s0, min(n, s0 + _CHUNK)), starts))
+    return out
+
+
+def _uniform_at(seed: int, stream: int, start: int, count: int) -> np.ndarray:
+    z = splitmix64(seed, stream, count, start=start)
     return ((z >> np.uint64(11)).astype(np.float64) + 0.5) * (1.0 / 9007199254740992.0)
 
 
+def uniform(seed: int, stream: int, n: int) -> np.ndarray:
+    """Uniform doubles in the open interval (0, 1): u_i from counter i + 1."""
+    def fill(out, a, b):
+        out[a:b] = _uniform_at(seed, stream, a, b - a)
+    return _chunked(n, fill)
+
+
 def normal(seed: int, stream: int, n: int, std: float = 1.0) -> np.ndarray:
-    u = uniform(seed, stream, 2 * n)
-    u1, u2 = u[0::2], u[1::2]
-    return std * np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * np.pi * u2)
+    """Box-Muller on consecutive uniform pairs (u_2p, u_2p+1): outputs 2p and
+    2p+1 are R cos(theta) and R sin(theta)."""
+    def fill(out, a, b):                     # a is even (chunk boundaries are)
+        cnt = b - a
+        pairs = (cnt + 1) // 2
+        u = _uniform_at(seed, stream, a, 2 * pairs)
+        r = std * np.sqrt(-2.0 * np.log(u[0::2]))
+        t = 2.0 * np.pi * u[1::2]
+        v = np.empty(2 * pairs, np.float64)
+        v[0::2] = r * np.cos(t)
+        v[1::2] = r * np.sin(t)
+        out[a:b] = v[:cnt]
+    return _chunked(n, fill)
 
 
 def laplace(seed: int, stream: int, n: int, b: float = 1.0) -> np.ndarray:
-    u = uniform(seed, stream, n) - 0.5
-    return -b * np.sign(u) * np.log1p(-2.0 * np.abs(u))
+    def fill(out, a, e):
+        u = _uniform_at(seed, stream, a, e - a) - 0.5
+        out[a:e] = -b * np.sign(u) * np.log1p(-2.0 * np.abs(u))
+    return _chunked(n, fill)
 
 
 def distinct_positions(seed: int, stream: int, n: int, count: int) -> np.ndarray:
@@ -87,10 +128,16 @@ def distinct_positions(seed: int, stream: int, n: int, count: int) -> np.ndarray
 
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round to BF16 (nearest even) and return the uint16 bit patterns."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
-    lsb = (u >> np.uint32(16)) & np.uint32(1)
-    r = (u + np.uint32(0x7FFF) + lsb) >> np.uint32(16)
-    return r.astype(np.uint16)
+    u = np.ascontiguousarray(x, dtype=np.float32).reshape(-1).view(np.uint32)
+    out = np.empty(u.size, np.uint16)
+
+    def conv(a):
+        b = min(u.size, a + _CHUNK)
+        v = u[a:b]
+        lsb = (v >> np.uint32(16)) & np.uint32(1)
+        out[a:b] = ((v + np.uint32(0x7FFF) + lsb) >> np.uint32(16)).astype(np.uint16)
+    list(_pool().map(conv, range(0, u.size, _CHUNK)))
+    return out.reshape(np.shape(x))
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
