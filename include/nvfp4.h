@@ -126,6 +126,31 @@ nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_
                                   uint8_t* codes, uint8_t* scales, float* global_scale,
                                   void* workspace, void* stream);
 
+/* nvfp4_quantize_act_static -- nvfp4_quantize_act without the workspace
+ * argument: this entry point allocates nothing and takes no scratch from the
+ * caller.  The pages have no counterpart; it exists for callers that cannot
+ * allocate device memory where they quantize -- a plugin whose host engine
+ * owns every byte of device memory and hands out no allocator, or a
+ * latency-critical path that may not call cudaMalloc (it can synchronize the
+ * whole device).
+ *   Scratch: a fixed 8448-byte array in the library's device image (each GPU
+ *   that loads the library holds it until the process exits), enough for at
+ *   most 1024 row groups; num_groups > 1024 returns
+ *   NVFP4_ERR_UNSUPPORTED_SHAPE.
+ *   The first call on a device looks up the array's device address with that
+ *   device current; make that first call before any stream capture.
+ *   Each call first clears, with an asynchronous memset on stream, the part of
+ *   the array that must start at zero; otherwise it behaves exactly like
+ *   nvfp4_quantize_act (same arguments, results, errors).
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents: calls that overlap on the GPU (e.g. on two streams without an
+ *   ordering between them) race and produce wrong results.
+ *   It calls no cudaMalloc, cudaFree or other allocating routine. */
+nvfp4_status_t nvfp4_quantize_act_static(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                         const int32_t* group_offsets, int num_groups,
+                                         uint8_t* codes, uint8_t* scales, float* global_scale,
+                                         void* stream);
+
 /* nvfp4_quantize_weight_2d -- 16 x 16 blocks share one E4M3 scale ("What is
  * NVFP4?", "Why does scaling matter so much?").  The tile's scale is written
  * to the tiled scale layout for each of its 16 rows (so the GEMM reads it like

@@ -22,7 +22,8 @@ from typing import Optional
 __all__ = [
     "lib", "Nvfp4Error", "NVFP4Tensor",
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_grouped_scale_bytes", "nvfp4_workspace_bytes",
-    "nvfp4_workspace_init", "nvfp4_quantize_act", "nvfp4_quantize_weight_2d", "nvfp4_gemm",
+    "nvfp4_workspace_init", "nvfp4_quantize_act", "nvfp4_quantize_act_static", "nvfp4_quantize_weight_2d",
+    "nvfp4_gemm",
     "nvfp4_grouped_gemm", "nvfp4_get_last_device_error", "nvfp4_set_wait_limit_ns", "nvfp4_probe_cvt",
     "nvfp4_probe_bounded_wait", "nvfp4_status_string", "nvfp4_version",
     "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
@@ -56,6 +57,7 @@ _SIGNATURES = {
     "nvfp4_workspace_bytes": (_sz, [_i32, _i64, _i64, _i64, _i32]),
     "nvfp4_workspace_init": (_i32, [_vp, _sz, _vp]),
     "nvfp4_quantize_act": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp]),
+    "nvfp4_quantize_act_static": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_weight_2d": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
@@ -135,6 +137,14 @@ def nvfp4_quantize_act(x, rows, k, ld, group_offsets, num_groups, codes, scales,
                        stream=0) -> int:
     return lib().nvfp4_quantize_act(x, rows, k, ld, group_offsets, num_groups, codes, scales, global_scale,
                                     workspace, stream)
+
+
+def nvfp4_quantize_act_static(x, rows, k, ld, group_offsets, num_groups, codes, scales, global_scale,
+                              stream=0) -> int:
+    """nvfp4_quantize_act with the library's fixed device scratch instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    return lib().nvfp4_quantize_act_static(x, rows, k, ld, group_offsets, num_groups, codes, scales,
+                                           global_scale, stream)
 
 
 def nvfp4_quantize_weight_2d(w, n, k, ld, codes, scales, scales_compact, global_scale, workspace, stream=0) -> int:

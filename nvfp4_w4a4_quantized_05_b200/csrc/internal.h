@@ -20,7 +20,7 @@ uint64_t wait_limit_ns();
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+constexpr int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
 inline nvfp4_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
@@ -28,8 +28,8 @@ inline nvfp4_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NVF
 //   [0, 4)         CTA completion counter (uint32)
 //   [16, 16+4G)    per-group amax as FP32 bit patterns (uint32)
 //   [pad_off, +4(G+1))  per-group first scale row (int32), written each call
-inline int64_t quant_ws_amax_off() { return 16; }
-inline int64_t quant_ws_pad_off(int groups) { return round_up(16 + 4 * (int64_t)groups, 16); }
-inline int64_t quant_ws_bytes(int groups) { return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 256); }
+constexpr int64_t quant_ws_amax_off() { return 16; }
+constexpr int64_t quant_ws_pad_off(int groups) { return round_up(16 + 4 * (int64_t)groups, 16); }
+constexpr int64_t quant_ws_bytes(int groups) { return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 256); }
 
 }  // namespace nvfp4

@@ -25,6 +25,7 @@
 #include <cuda_runtime.h>
 #include <cfloat>
 #include <cstdint>
+#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -459,4 +460,63 @@ extern "C" nvfp4_status_t nvfp4_probe_cvt(const float* in, uint8_t* out_e2m1, ui
     const int grid = clamp_grid((n + 255) / 256, (int64_t)num_sms() * 16);
     probe_cvt_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(in, out_e2m1, out_e4m3, n);
     return cuda_status(cudaGetLastError());
+}
+
+// ---- quantization without a caller-provided workspace --------------------------------
+//
+// Some callers cannot allocate device memory at the point where they quantize:
+// a plugin whose host engine owns every byte of device memory and hands out no
+// allocator, or a latency-critical path where cudaMalloc (which may
+// synchronize the device) is not allowed.  For them the scratch lives in a
+// fixed array in this library's device image, sized for up to
+// kStaticMaxGroups row groups; every GPU that loads the library holds it
+// until the process exits.
+namespace nvfp4 {
+namespace {
+constexpr int kStaticMaxGroups = 1024;
+constexpr int64_t kStaticScratchBytes = quant_ws_bytes(kStaticMaxGroups);   // 8448 bytes
+std::mutex g_static_mu;
+void* g_static_ptr[64] = {};
+}  // namespace
+}  // namespace nvfp4
+
+static __device__ __align__(256) uint8_t g_static_quant_scratch[nvfp4::kStaticScratchBytes];
+
+namespace nvfp4 {
+namespace {
+// Device address of g_static_quant_scratch on the current device.  Host code
+// must not pass the symbol itself to a kernel: on the host it names a
+// host-side stand-in, not device memory.  Looked up once per device, with
+// that device current.
+void* static_scratch() {
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_static_mu);
+    if (!g_static_ptr[d]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_quant_scratch) != cudaSuccess || !p) return nullptr;
+        g_static_ptr[d] = p;
+    }
+    return g_static_ptr[d];
+}
+}  // namespace
+}  // namespace nvfp4
+
+extern "C" nvfp4_status_t nvfp4_quantize_act_static(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                                    const int32_t* group_offsets, int num_groups, uint8_t* codes,
+                                                    uint8_t* scales, float* global_scale, void* stream) {
+    if (rows < 0 || k <= 0 || ld < k || !x || !codes || !scales || !global_scale) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (group_offsets && num_groups < 1) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (!group_offsets && num_groups > 1) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (group_offsets && num_groups > kStaticMaxGroups) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
+    void* ws = static_scratch();
+    if (!ws) return NVFP4_ERR_CUDA;
+    const int groups = group_offsets ? num_groups : 1;
+    // The CTA counter and the amax slots must start at zero; the array keeps
+    // whatever the previous call on this device left in it.
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(ws, 0, (size_t)quant_ws_pad_off(groups), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    return nvfp4_quantize_act(x, rows, k, ld, group_offsets, num_groups, codes, scales, global_scale, ws, stream);
 }
