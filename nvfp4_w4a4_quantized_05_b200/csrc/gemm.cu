@@ -13,16 +13,26 @@
 // "Impact on the Open-Source Community and LLM Deployment Industry"; "W4A8 vs
 // NVFP4 quantization on GPUs", "Dequantization can erase a four-bit win").
 //
-// Kernel structure (one CTA per SM, persistent over output tiles):
+// Kernel structure (one CTA per SM, persistent over output tiles, 10 warps):
 //   warp 0     TMA producer: codes tiles by tensor-map copies (128-byte
 //              swizzle), scale tiles by bulk copies, into a STAGES-deep ring
 //              guarded by mbarriers.  No cluster multicast.
-//   warp 1     allocates tensor memory; one thread moves each stage's scale
-//              tiles to tensor memory (tcgen05.cp) and issues the MMAs
-//              (128 x BN x 64 each), then commits to the stage's "empty"
-//              barrier and, per tile, to the accumulator-full barrier.
+//   warp 1     allocates tensor memory; one thread issues the MMAs (128 x BN
+//              x 64 each) and commits to the stage's "empty" barrier, the
+//              scale buffer's "free" barrier and, per tile, the accumulator
+//              buffer's "full" barrier.
 //   warps 2-5  epilogue: tcgen05.ld of the FP32 accumulator, x (ga * gb),
-//              round to BF16, store.
+//              round to BF16, store.  Two accumulator buffers in tensor
+//              memory, so the epilogue of one tile overlaps the next tile's
+//              mainloop (when 2 x BN columns and the scale buffers fit).
+//   warps 6-9  scale staging: each warp owns one 32-lane quarter of tensor
+//              memory and writes the stage's scale tiles there with
+//              tcgen05.st, in the replicated layout the block-scaled MMA
+//              reads (lane i, column c of a 128-row block's k-step holds the
+//              four scales of row i + 32c).  Moving scales with tcgen05.cp
+//              would put ~100 cycles per copy on the tensor pipe, in series
+//              with the MMAs (12 copies per 128x256x256 k-tile); tcgen05.st
+//              from the otherwise idle warps keeps the tensor pipe for MMAs.
 // Every mbarrier wait is bounded (globaltimer); a wait that runs out sets the
 // library's device error word and the CTA winds down instead of hanging.
 //
@@ -46,9 +56,8 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 320;         // 10 warps, roles above
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kSfCol = 256;      // first tensor-memory column of the scale buffers
 constexpr int kMaxStages = 8;
 constexpr int kMaxGroups = 256;
 
@@ -78,8 +87,10 @@ struct GemmArgs {
 struct alignas(8) SmemTail {
     uint64_t full[kMaxStages];
     uint64_t empty[kMaxStages];
-    uint64_t tmem_full;
-    uint64_t tmem_empty;
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t sf_full[2];
+    uint64_t sf_empty[2];
     uint32_t tmem_base;
     volatile int abort_flag;
     int total_tiles;
@@ -142,27 +153,42 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int BN, int STAGES, bool SWAP, bool GROUPED>
-__global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
-    constexpr int NRB = BN >= 128 ? BN / 128 : 1;          // 128-row scale blocks on the B side
-    constexpr uint32_t A_BYTES = 128 * 128;                  // 128 rows x 256 FP4
-    constexpr uint32_t B_BYTES = BN * 128;
-    constexpr uint32_t SFA_BYTES = 4 * 512;                  // 4 k-steps x (128 rows x 4 scales)
-    constexpr uint32_t SFB_BYTES = NRB * 4 * 512;
-    constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
-    constexpr uint32_t SF_COLS = 16 + 16 * NRB;              // tensor-memory columns per k-tile of scales
-    constexpr int CW = BN >= 32 ? 32 : 16;                   // epilogue column chunk
-    constexpr uint32_t IDESC = idesc_mxf4nvf4(128, BN);
+// Compile-time shape of one kernel configuration.
+template <int BN_, int STAGES_, int ACC_>
+struct Cfg {
+    static constexpr int BN = BN_;
+    static constexpr int STAGES = STAGES_;
+    static constexpr int ACC = ACC_;                          // accumulator buffers in tensor memory
+    // 128-row scale blocks a B tile can touch: tiles start at multiples of BN,
+    // i.e. at a row offset 0 or 64 inside a block for BN = 192.
+    static constexpr int NSFB = BN == 192 ? 2 : (BN + 127) / 128;
+    static constexpr uint32_t A_BYTES = 128 * 128;            // 128 rows x 256 FP4
+    static constexpr uint32_t B_BYTES = BN * 128;
+    static constexpr uint32_t SFA_BYTES = 4 * 512;            // 4 k-steps x (128 rows x 4 scales)
+    static constexpr uint32_t SFB_BYTES = NSFB * 4 * 512;
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr uint32_t SF_COLS = 16 + 16 * NSFB;       // tensor-memory columns per k-tile of scales
+    static constexpr uint32_t SF_BASE = ACC * BN;             // first scale column
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(STAGES <= kMaxStages, "stages");
-    static_assert(kSfCol + 2 * SF_COLS <= kTmemCols, "tensor memory budget");
+    static_assert(ACC == 1 || ACC == 2, "accumulator buffers");
+    static_assert(SF_BASE + 2 * SF_COLS <= kTmemCols, "tensor memory budget");
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static_assert(SMEM <= 232448, "shared memory");
+};
+
+template <class C, bool SWAP, bool GROUPED>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+    constexpr int BN = C::BN, STAGES = C::STAGES, ACC = C::ACC, NSFB = C::NSFB;
+    constexpr int CW = BN >= 32 ? 32 : 16;                   // epilogue column chunk
+    constexpr uint32_t IDESC = idesc_mxf4nvf4(128, BN);
     static_assert(!(SWAP && GROUPED), "swap form is for the plain GEMM");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + STAGES * STAGE_BYTES);
+    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + STAGES * C::STAGE_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t limit = p.wait_limit_ns;
 
@@ -171,8 +197,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tail->full[s], 1);
             mbar_init(&tail->empty[s], 1);
         }
-        mbar_init(&tail->tmem_full, 1);
-        mbar_init(&tail->tmem_empty, 4);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tail->acc_full[b], 1);
+            mbar_init(&tail->acc_empty[b], 4);
+            mbar_init(&tail->sf_full[b], 4);
+            mbar_init(&tail->sf_empty[b], 1);
+        }
         tail->abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -242,19 +272,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint8_t* sfa_src = p.sfa + (int64_t)ti.sfa_rb * p.sfa_rb_stride;
                 const uint8_t* sfb_src = p.sfb + (int64_t)ti.group * p.sfb_group_stride +
                                          (int64_t)(ti.b_col0 / 128) * p.sfb_rb_stride;
-                const int nsfb = min(NRB, p.sfb_rb_per_group - ti.b_col0 / 128);
+                const int nsfb = min(NSFB, p.sfb_rb_per_group - ti.b_col0 / 128);
                 for (int kt = 0; kt < p.num_kt; ++kt) {
                     if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
                         ok = false;
                         break;
                     }
                     const int nat = min(4, p.num_ks - kt * 4);
-                    uint8_t* sA = smem + stage * STAGE_BYTES;
-                    uint8_t* sB = sA + A_BYTES;
-                    uint8_t* sSFA = sB + B_BYTES;
-                    uint8_t* sSFB = sSFA + SFA_BYTES;
+                    uint8_t* sA = smem + stage * C::STAGE_BYTES;
+                    uint8_t* sB = sA + C::A_BYTES;
+                    uint8_t* sSFA = sB + C::B_BYTES;
+                    uint8_t* sSFB = sSFA + C::SFA_BYTES;
                     uint64_t* bar = &tail->full[stage];
-                    mbar_arrive_expect_tx(bar, A_BYTES + B_BYTES + (uint32_t)nat * 512u * (1u + (uint32_t)nsfb));
+                    mbar_arrive_expect_tx(bar, C::A_BYTES + C::B_BYTES + (uint32_t)nat * 512u * (1u + (uint32_t)nsfb));
                     tma_load_2d(sA, &tmA, bar, kt * 128, ti.a_row0);
                     tma_load_2d(sB, &tmB, bar, kt * 128, ti.b_row0);
                     bulk_load(sSFA, sfa_src + (int64_t)kt * 2048, (uint32_t)nat * 512u, bar);
@@ -276,54 +306,94 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++it) {
-                if (!mbar_wait(&tail->tmem_empty, (uint32_t)(it & 1) ^ 1u, limit) || tail->abort_flag) {
+                const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
+                const uint32_t ab = ACC == 2 ? (uint32_t)(it & 1) : 0u;
+                const uint32_t au = ACC == 2 ? (uint32_t)(it >> 1) : (uint32_t)it;
+                if (!mbar_wait(&tail->acc_empty[ab], (au & 1u) ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
+                const uint32_t d_tmem = tmem + ab * BN;
+                const uint32_t sfb_off = 16 + (uint32_t)((ti.b_col0 % 128) / 32);
                 for (int kt = 0; kt < p.num_kt; ++kt, ++ktg) {
-                    if (!mbar_wait(&tail->full[stage], phase, limit) || tail->abort_flag) {
+                    const uint32_t sb = ktg & 1u, su = ktg >> 1;
+                    if (!mbar_wait(&tail->full[stage], phase, limit) ||
+                        !mbar_wait(&tail->sf_full[sb], su & 1u, limit) || tail->abort_flag) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     const int nat = min(4, p.num_ks - kt * 4);
-                    const uint32_t sA = smem_u32(smem + stage * STAGE_BYTES);
-                    const uint32_t sB = sA + A_BYTES;
-                    const uint32_t sSFA = sB + B_BYTES;
-                    const uint32_t sSFB = sSFA + SFA_BYTES;
-                    const uint32_t sf = tmem + kSfCol + (ktg & 1u) * SF_COLS;
-                    for (int j = 0; j < nat; ++j) tmem_cp_32x128b_x4(sf + j * 4, sdesc_sf_block(sSFA + j * 512));
-                    for (int rb = 0; rb < NRB; ++rb)
-                        for (int j = 0; j < nat; ++j)
-                            tmem_cp_32x128b_x4(sf + 16 + j * 4 * NRB + rb * 4,
-                                               sdesc_sf_block(sSFB + rb * 2048 + j * 512));
+                    const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
+                    const uint32_t sB = sA + C::A_BYTES;
+                    const uint32_t sf = tmem + C::SF_BASE + sb * C::SF_COLS;
                     for (int j = 0; j < nat; ++j)
-                        mma_mxf4nvf4(tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32), IDESC,
-                                     sf + j * 4, sf + 16 + j * 4 * NRB, (kt > 0 || j > 0) ? 1u : 0u);
+                        mma_mxf4nvf4(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32), IDESC,
+                                     sf + j * 4, sf + sfb_off + j * 4 * NSFB, (kt > 0 || j > 0) ? 1u : 0u);
                     tc_commit(&tail->empty[stage]);
+                    tc_commit(&tail->sf_empty[sb]);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (ok) tc_commit(&tail->tmem_full);
+                if (ok) tc_commit(&tail->acc_full[ab]);
             }
             if (!ok) raise_abort(tail, p.err);
         }
+    } else if (warp >= 6) {
+        // ---------------- scale staging (warps 6..9, one lane quarter each) ----------------
+        const int q = warp & 3;
+        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + C::SF_BASE;
+        uint32_t stage = 0, phase = 0, ktg = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+            for (int kt = 0; kt < p.num_kt; ++kt, ++ktg) {
+                const uint32_t sb = ktg & 1u, su = ktg >> 1;
+                if (!mbar_wait(&tail->full[stage], phase, limit) ||
+                    !mbar_wait(&tail->sf_empty[sb], (su & 1u) ^ 1u, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sSFA = smem_u32(smem + stage * C::STAGE_BYTES) + C::A_BYTES + C::B_BYTES;
+                const uint32_t sSFB = sSFA + C::SFA_BYTES;
+                const uint32_t dst = tq + sb * C::SF_COLS;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tmem_st_32x32b_x4(dst + j * 4, ld_shared_v4(sSFA + j * 512 + lane * 16));
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int rb = 0; rb < NSFB; ++rb)
+                        tmem_st_32x32b_x4(dst + 16 + j * 4 * NSFB + rb * 4,
+                                          ld_shared_v4(sSFB + rb * 2048 + j * 512 + lane * 16));
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tail->sf_full[sb]);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) raise_abort(tail, p.err);
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const int rloc = q * 32 + lane;               // A-side row inside the tile
-        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
         int it = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
             const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
-            if (!mbar_wait(&tail->tmem_full, (uint32_t)(it & 1), limit) || tail->abort_flag) {
+            const uint32_t ab = ACC == 2 ? (uint32_t)(it & 1) : 0u;
+            const uint32_t au = ACC == 2 ? (uint32_t)(it >> 1) : (uint32_t)it;
+            if (!mbar_wait(&tail->acc_full[ab], au & 1u, limit) || tail->abort_flag) {
                 if (lane == 0) raise_abort(tail, p.err);
                 break;
             }
             tc_fence_after();
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
             const float alpha = __fmul_rn(p.ga[ti.group], p.gb[ti.group]);
             const bool a_ok = rloc < ti.a_rows;
 #pragma unroll 1
@@ -369,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&tail->tmem_empty);
+            if (lane == 0) mbar_arrive(&tail->acc_empty[ab]);
         }
     }
 
@@ -411,23 +481,19 @@ bool make_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES, bool SWAP, bool GROUPED>
+template <class C, bool SWAP, bool GROUPED>
 nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid, cudaStream_t s) {
-    constexpr int NRB = BN >= 128 ? BN / 128 : 1;
-    constexpr size_t stage = 128 * 128 + BN * 128 + 2048 + NRB * 2048;
-    constexpr size_t smem = 1024 + STAGES * stage + sizeof(SmemTail);
-    static_assert(smem <= 232448, "shared memory");
-    auto kern = gemm_kernel<BN, STAGES, SWAP, GROUPED>;
+    auto kern = gemm_kernel<C, SWAP, GROUPED>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
     });
     if (attr_err != cudaSuccess) return NVFP4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = C::SMEM;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -436,6 +502,14 @@ nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
     cfg.numAttrs = 1;
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
 }
+
+// Kernel configurations: prefill / grouped use 128 x 192 tiles with two
+// accumulator buffers (2 x 192 + 2 x 48 scale columns of tensor memory);
+// decode uses the swapped form with a narrow token side.
+using CfgWide = Cfg<192, 4, 2>;
+using CfgDec16 = Cfg<16, 8, 2>;
+using CfgDec32 = Cfg<32, 8, 2>;
+using CfgDec64 = Cfg<64, 7, 2>;
 
 bool ptr_ok(const void* p) { return p && aligned16(p); }
 
@@ -490,11 +564,11 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         p.tiles_m = (int)((n + 127) / 128);
         p.tiles_n = 1;
         const int grid = (int)std::min<int64_t>(p.tiles_m, sms);
-        if (bn == 16) return launch<16, 7, true, false>(ta, tb, p, grid, s);
-        if (bn == 32) return launch<32, 7, true, false>(ta, tb, p, grid, s);
-        return launch<64, 7, true, false>(ta, tb, p, grid, s);
+        if (bn == 16) return launch<CfgDec16, true, false>(ta, tb, p, grid, s);
+        if (bn == 32) return launch<CfgDec32, true, false>(ta, tb, p, grid, s);
+        return launch<CfgDec64, true, false>(ta, tb, p, grid, s);
     }
-    constexpr int BN = 256;
+    constexpr int BN = CfgWide::BN;
     if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN))
         return NVFP4_ERR_CUDA;
     p.sfa = a_scales;
@@ -509,7 +583,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int grid = (int)std::min<int64_t>(tiles, sms);
-    return launch<BN, 4, false, false>(ta, tb, p, grid, s);
+    return launch<CfgWide, false, false>(ta, tb, p, grid, s);
 }
 
 extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
@@ -531,7 +605,7 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     const int sms = num_sms();
     if (sms <= 0) return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    constexpr int BN = 256;
+    constexpr int BN = CfgWide::BN;
     const int64_t sf_rb_stride = 128 * (k / 16);
     GemmArgs p = {};
     p.num_ks = (int)(k / 64);
@@ -562,5 +636,5 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     // upper bound of the tile count: sum_e ceil(n_e / 128) <= total_rows / 128 + num_experts
     const int64_t max_tiles = (total_rows / 128 + num_experts) * (int64_t)p.tiles_n;
     const int grid = (int)std::min<int64_t>(max_tiles, sms);
-    return launch<BN, 4, false, true>(ta, tb, p, grid, s);
+    return launch<CfgWide, false, true>(ta, tb, p, grid, s);
 }
