@@ -169,7 +169,9 @@ struct Cfg {
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t SF_COLS = 16 + 16 * NSFB;       // tensor-memory columns per k-tile of scales
     static constexpr uint32_t SF_BASE = ACC * BN;             // first scale column
-    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + sizeof(SmemTail);
+    // epilogue staging: per epilogue warp two 32-row x 64-byte BF16 boxes
+    static constexpr uint32_t EPI_BYTES = 4 * 2 * 2048;
+    static constexpr size_t SMEM = 1024 + (size_t)STAGES * STAGE_BYTES + EPI_BYTES + sizeof(SmemTail);
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(STAGES <= kMaxStages, "stages");
     static_assert(ACC == 1 || ACC == 2, "accumulator buffers");
@@ -180,7 +182,8 @@ struct Cfg {
 
 template <class C, bool SWAP, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const GemmArgs p) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
     constexpr int BN = C::BN, STAGES = C::STAGES, ACC = C::ACC, NSFB = C::NSFB;
     constexpr int CW = BN >= 32 ? 32 : 16;                   // epilogue column chunk
     constexpr uint32_t IDESC = idesc_mxf4nvf4(128, BN);
@@ -188,7 +191,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    SmemTail* tail = reinterpret_cast<SmemTail*>(smem + STAGES * C::STAGE_BYTES);
+    uint8_t* epi_smem = smem + STAGES * C::STAGE_BYTES;
+    SmemTail* tail = reinterpret_cast<SmemTail*>(epi_smem + C::EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t limit = p.wait_limit_ns;
 
@@ -207,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
+        if (!SWAP) prefetch_tmap(&tmC);
     }
     if (warp == 1) {
         tmem_alloc(&tail->tmem_base, kTmemCols);
@@ -381,8 +386,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok && lane == 0) raise_abort(tail, p.err);
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
+        // Non-swapped tiles: each warp converts its 32 rows x 32 columns of
+        // FP32 accumulator to BF16 in a swizzled 2 KB shared-memory box (two
+        // boxes per warp, alternating) and writes it with a TMA tensor store;
+        // the tensor bounds clip ragged tiles.  The last slab of an expert's
+        // rows in the grouped form (rows past the group belong to the next
+        // expert) and the swapped (transposed) decode form use direct stores.
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const int rloc = q * 32 + lane;               // A-side row inside the tile
+        const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * 4096u;
         int it = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
             const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
@@ -396,6 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
             const float alpha = __fmul_rn(p.ga[ti.group], p.gb[ti.group]);
             const bool a_ok = rloc < ti.a_rows;
+            const bool use_tma = !SWAP && (!GROUPED || q * 32 + 32 <= ti.a_rows);
 #pragma unroll 1
             for (int ch = 0; ch < BN / CW; ++ch) {
                 uint32_t v[CW];
@@ -406,24 +419,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 tmem_ld_wait();
                 if constexpr (!SWAP) {
-                    if (a_ok) {
+                    if (ch * CW >= ti.b_rows) continue;      // uniform: whole chunk past n
+                    if (use_tma) {
+                        const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
+                        if (lane == 0) bulk_wait_group_read<1>();   // the box's previous store has read it
+                        __syncwarp();
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            uint4 w;
+                            w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * alpha, __uint_as_float(v[8 * j + 1]) * alpha);
+                            w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * alpha, __uint_as_float(v[8 * j + 3]) * alpha);
+                            w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * alpha, __uint_as_float(v[8 * j + 5]) * alpha);
+                            w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * alpha, __uint_as_float(v[8 * j + 7]) * alpha);
+                            // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
+                            st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
+                        }
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_2d(&tmC, box, ti.b_col0 + ch * CW, ti.a_row0 + q * 32);
+                            bulk_commit_group();
+                        }
+                    } else if (a_ok) {
                         __nv_bfloat16* crow = p.c + (int64_t)(ti.a_row0 + rloc) * p.ldc + ti.b_col0 + ch * CW;
                         const int ncols = ti.b_rows - ch * CW;
-                        if (ncols >= CW) {
 #pragma unroll
-                            for (int i = 0; i < CW; i += 8) {
-                                uint4 w;
-                                w.x = pack_bf16x2(__uint_as_float(v[i + 0]) * alpha, __uint_as_float(v[i + 1]) * alpha);
-                                w.y = pack_bf16x2(__uint_as_float(v[i + 2]) * alpha, __uint_as_float(v[i + 3]) * alpha);
-                                w.z = pack_bf16x2(__uint_as_float(v[i + 4]) * alpha, __uint_as_float(v[i + 5]) * alpha);
-                                w.w = pack_bf16x2(__uint_as_float(v[i + 6]) * alpha, __uint_as_float(v[i + 7]) * alpha);
-                                *reinterpret_cast<uint4*>(crow + i) = w;
-                            }
-                        } else {
-#pragma unroll
-                            for (int i = 0; i < CW; ++i)
-                                if (i < ncols) crow[i] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
-                        }
+                        for (int i = 0; i < CW; ++i)
+                            if (i < ncols) crow[i] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
                     }
                 } else {
                     if (a_ok) {
@@ -441,6 +463,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tail->acc_empty[ab]);
         }
+        if (lane == 0) bulk_wait_group_all();   // stores done before the CTA's shared memory goes away
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -482,7 +506,8 @@ bool make_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ro
 }
 
 template <class C, bool SWAP, bool GROUPED>
-nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmArgs& args, int grid, cudaStream_t s) {
+nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+                      int grid, cudaStream_t s) {
     auto kern = gemm_kernel<C, SWAP, GROUPED>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
@@ -500,7 +525,7 @@ nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const GemmAr
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, args));
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args));
 }
 
 // Kernel configurations: prefill / grouped use 128 x 192 tiles with two
@@ -510,6 +535,21 @@ using CfgWide = Cfg<192, 4, 2>;
 using CfgDec16 = Cfg<16, 8, 2>;
 using CfgDec32 = Cfg<32, 8, 2>;
 using CfgDec64 = Cfg<64, 7, 2>;
+
+// BF16 [rows, cols] output with row stride ldc elements, 32 x 32 boxes,
+// 64-byte swizzle (matches the epilogue's staging layout).
+bool make_out_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t ldc) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)(ldc * 2)};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 bool ptr_ok(const void* p) { return p && aligned16(p); }
 
@@ -548,7 +588,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     p.wait_limit_ns = wait_limit_ns();
     p.err = device_error_word();
     if (!p.err) return NVFP4_ERR_CUDA;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     if (m <= 64) {
         // decode: weights on the 128-row side, tokens on the narrow side
         const int bn = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
@@ -564,12 +604,14 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         p.tiles_m = (int)((n + 127) / 128);
         p.tiles_n = 1;
         const int grid = (int)std::min<int64_t>(p.tiles_m, sms);
-        if (bn == 16) return launch<CfgDec16, true, false>(ta, tb, p, grid, s);
-        if (bn == 32) return launch<CfgDec32, true, false>(ta, tb, p, grid, s);
-        return launch<CfgDec64, true, false>(ta, tb, p, grid, s);
+        tc = tb;   // unused by the swapped form
+        if (bn == 16) return launch<CfgDec16, true, false>(ta, tb, tc, p, grid, s);
+        if (bn == 32) return launch<CfgDec32, true, false>(ta, tb, tc, p, grid, s);
+        return launch<CfgDec64, true, false>(ta, tb, tc, p, grid, s);
     }
     constexpr int BN = CfgWide::BN;
-    if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN))
+    if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN) ||
+        !make_out_map(&tc, c, m, n, ldc))
         return NVFP4_ERR_CUDA;
     p.sfa = a_scales;
     p.sfb = b_scales;
@@ -583,7 +625,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int grid = (int)std::min<int64_t>(tiles, sms);
-    return launch<CfgWide, false, false>(ta, tb, p, grid, s);
+    return launch<CfgWide, false, false>(ta, tb, tc, p, grid, s);
 }
 
 extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
@@ -629,12 +671,12 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     p.wait_limit_ns = wait_limit_ns();
     p.err = device_error_word();
     if (!p.err) return NVFP4_ERR_CUDA;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tc;
     if (!make_codes_map(&ta, a_codes, total_rows, k / 2, 128) ||
-        !make_codes_map(&tb, b_codes, n * num_experts, k / 2, BN))
+        !make_codes_map(&tb, b_codes, n * num_experts, k / 2, BN) || !make_out_map(&tc, c, total_rows, n, n))
         return NVFP4_ERR_CUDA;
     // upper bound of the tile count: sum_e ceil(n_e / 128) <= total_rows / 128 + num_experts
     const int64_t max_tiles = (total_rows / 128 + num_experts) * (int64_t)p.tiles_n;
     const int grid = (int)std::min<int64_t>(max_tiles, sms);
-    return launch<CfgWide, false, true>(ta, tb, p, grid, s);
+    return launch<CfgWide, false, true>(ta, tb, tc, p, grid, s);
 }

@@ -15,13 +15,18 @@
 // roundings to E4M3 / E2M1 are the hardware cvt.rn.satfinite instructions, so
 // the codes and scale bytes are bit-identical to the CPU definition.
 //
-// Memory-bound design: 16-byte coalesced loads, warp-task = 256 consecutive
-// elements of one row (lane = 8 elements, lane pair = one 16-element block),
-// 4 tasks in flight per warp; packed codes stored as coalesced 4-byte words;
-// 4 scale bytes gathered by shuffles into one word of the 512-byte tile.  The
-// amax pass ends with a "last CTA" step that publishes g, writes the group scale
-// offsets and re-zeroes the workspace; the quantizer is launched with
-// programmatic dependent launch so its CTAs are resident when g is ready.
+// Memory-bound design.  Kernel 1 (amax) runs as one wave of CTAs that stream
+// the tensor with 16-byte loads, 8 in flight per thread, tagged L2::evict_last
+// so the tensor stays in the 126 MB L2 for the second pass; it ends with a
+// "last CTA" step that publishes g, writes the group scale offsets and
+// re-zeroes the workspace.  Kernel 2 (quantize) is launched with programmatic
+// dependent launch: its CTAs issue their first loads (tagged evict_first)
+// before waiting for kernel 1, since only g depends on it.  A warp task is
+// 512 consecutive elements of one row; lane l owns 16-element block l (two
+// 16-byte loads), so the block amax, the E4M3 scale and the reciprocal are
+// computed once per block; the 16 codes leave as one 8-byte store (the warp
+// writes 256 contiguous bytes) and 4 scale bytes are gathered by shuffles
+// into one word of the 512-byte scale tile.  Task stepping is division-free.
 #include <cuda_runtime.h>
 #include <cfloat>
 #include <cstdint>
@@ -35,7 +40,6 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kUnroll = 4;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr float kGlobalDen = 2688.0f;   // 6 (largest E2M1) * 448 (largest E4M3)
 
@@ -138,34 +142,38 @@ struct AmaxArgs {
     float* gscale;
 };
 
-__global__ void __launch_bounds__(kThreads) amax_kernel(AmaxArgs a) {
+constexpr int kAmaxUnroll = 8;
+
+__global__ void __launch_bounds__(kThreads, 4) amax_kernel(AmaxArgs a) {
     const int e = blockIdx.y;
     int r0, r1;
     a.groups.range(e, r0, r1);
-    const int kc = a.k / 8;
+    const int kc = a.k / 8;                            // 16-byte chunks per row
     const int64_t items = (int64_t)(r1 - r0) * kc;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     const bool dense = (a.ld == (int64_t)a.k);
+    const uint16_t* base = a.x + (int64_t)r0 * a.ld;
+    const uint64_t pol = l2_policy_evict_last();
     uint32_t m = 0;
-    for (int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; i0 < items; i0 += stride * kUnroll) {
-        uint4 v[kUnroll];
+    for (int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; i0 < items; i0 += stride * kAmaxUnroll) {
+        uint4 v[kAmaxUnroll];
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
+        for (int u = 0; u < kAmaxUnroll; ++u) {
             const int64_t i = i0 + u * stride;
             v[u] = make_uint4(0, 0, 0, 0);
             if (i < items) {
                 const uint16_t* p;
                 if (dense) {
-                    p = a.x + (int64_t)r0 * a.k + i * 8;
+                    p = base + i * 8;
                 } else {
                     const int64_t r = i / kc;
-                    p = a.x + (r0 + r) * a.ld + (i - r * kc) * 8;
+                    p = base + r * a.ld + (i - r * kc) * 8;
                 }
-                v[u] = ld_nc_v4(p);
+                v[u] = ld_nc_v4_hint(p, pol);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) m = max(m, absmax8_bits(v[u]));
+        for (int u = 0; u < kAmaxUnroll; ++u) m = max(m, absmax8_bits(v[u]));
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
@@ -199,7 +207,7 @@ struct Quant1dArgs {
     const uint16_t* x;
     int64_t ld;
     int k;
-    int nseg;         // ceil(k / 256)
+    int nseg;         // ceil(k / 512): 512-element warp tasks per row
     int scale_cols;   // ceil(k / 64) * 4
     Groups groups;
     const int32_t* pad_rows;   // nullptr: one tensor, scale rows from 0
@@ -208,53 +216,96 @@ struct Quant1dArgs {
     uint8_t* scales;
 };
 
-__global__ void __launch_bounds__(kThreads) quant1d_kernel(Quant1dArgs a) {
-    pdl_wait();   // g (and the group scale offsets) come from amax_kernel
+constexpr int kQuantUnroll = 2;
+
+// Position (row, segment) of a warp task, advanced without divisions.
+struct TaskPos {
+    int row, seg;
+    __device__ __forceinline__ void advance(int drow, int dseg, int nseg) {
+        row += drow;
+        seg += dseg;
+        if (seg >= nseg) {
+            seg -= nseg;
+            ++row;
+        }
+    }
+};
+
+__device__ __forceinline__ void load_block16(const Quant1dArgs& a, int r0, int nrows, const TaskPos& t, int lane,
+                                             uint64_t pol, uint4& v0, uint4& v1) {
+    const int col = t.seg * 512 + lane * 16;
+    v0 = make_uint4(0, 0, 0, 0);
+    v1 = make_uint4(0, 0, 0, 0);
+    if (t.row < nrows && col < a.k) {
+        const uint16_t* p = a.x + (int64_t)(r0 + t.row) * a.ld + col;
+        v0 = ld_nc_v4_hint(p, pol);
+        v1 = ld_nc_v4_hint(p + 8, pol);
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
     const int e = blockIdx.y;
     int r0, r1;
     a.groups.range(e, r0, r1);
     const int nrows = r1 - r0;
+    const int lane = threadIdx.x & 31;
+    const int prows = round128(nrows);
+    const int w0 = blockIdx.x * kWarps + (threadIdx.x >> 5);
+    const int wstride = gridDim.x * kWarps;
+    const int nseg = a.nseg;
+    // task t -> (t / nseg, t % nseg); step kQuantUnroll * wstride tasks per iteration
+    TaskPos t0{w0 / nseg, w0 % nseg};
+    const int step = kQuantUnroll * wstride;
+    const int drow = step / nseg, dseg = step - (step / nseg) * nseg;
+    const int d1row = wstride / nseg, d1seg = wstride - d1row * nseg;
+    const uint64_t pol = l2_policy_evict_first();
+    const int64_t kbytes = a.k / 2;
+
+    // The input does not depend on kernel 1: start the first loads before waiting.
+    uint4 v[kQuantUnroll][2];
+    TaskPos tp[kQuantUnroll];
+    tp[0] = t0;
+#pragma unroll
+    for (int u = 1; u < kQuantUnroll; ++u) {
+        tp[u] = tp[u - 1];
+        tp[u].advance(d1row, d1seg, nseg);
+    }
+#pragma unroll
+    for (int u = 0; u < kQuantUnroll; ++u) load_block16(a, r0, nrows, tp[u], lane, pol, v[u][0], v[u][1]);
+
+    pdl_wait();   // g (and the group scale offsets) come from amax_kernel
     const int srow0 = a.pad_rows ? a.pad_rows[e] : 0;
     const float g = a.gscale[e];
     const float k6 = __fmul_rn(6.0f, g);
-    const int ntasks = round128(nrows) * a.nseg;
-    const int lane = threadIdx.x & 31;
-    const int wstride = gridDim.x * kWarps;
-    const int64_t kbytes = a.k / 2;
-    for (int t0 = blockIdx.x * kWarps + (threadIdx.x >> 5); t0 < ntasks; t0 += wstride * kUnroll) {
-        uint4 v[kUnroll];
+
+    while (tp[0].row < prows) {
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int t = t0 + u * wstride;
-            v[u] = make_uint4(0, 0, 0, 0);
-            if (t < ntasks) {
-                const int rr = t / a.nseg;
-                const int col = (t - rr * a.nseg) * 256 + lane * 8;
-                if (rr < nrows && col < a.k) v[u] = ld_nc_v4(a.x + (int64_t)(r0 + rr) * a.ld + col);
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const TaskPos t = tp[u];
+            if (t.row >= prows) break;   // uniform across the warp
+            const int col = t.seg * 512 + lane * 16;
+            uint32_t am = max(absmax8_bits(v[u][0]), absmax8_bits(v[u][1]));
+            float r;
+            const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, r);
+            if (t.row < nrows && col < a.k) {
+                uint2 q;
+                q.x = quant8(v[u][0], r);
+                q.y = quant8(v[u][1], r);
+                *reinterpret_cast<uint2*>(a.codes + (int64_t)(r0 + t.row) * kbytes + col / 2) = q;
+            }
+            const uint32_t s1 = __shfl_down_sync(kFull, sf, 1);
+            const uint32_t s2 = __shfl_down_sync(kFull, sf, 2);
+            const uint32_t s3 = __shfl_down_sync(kFull, sf, 3);
+            const int scol = t.seg * 32 + lane;
+            if ((lane & 3) == 0 && scol < a.scale_cols) {
+                const uint32_t word = (t.row < nrows) ? (sf | (s1 << 8) | (s2 << 16) | (s3 << 24)) : 0u;
+                *reinterpret_cast<uint32_t*>(a.scales + sf_tile_offset(srow0 + t.row, scol, a.scale_cols)) = word;
             }
         }
 #pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            const int t = t0 + u * wstride;
-            if (t >= ntasks) break;   // uniform across the warp
-            const int rr = t / a.nseg;
-            const int seg = t - rr * a.nseg;
-            const int col = seg * 256 + lane * 8;
-            uint32_t am = absmax8_bits(v[u]);
-            am = max(am, __shfl_xor_sync(kFull, am, 1));
-            float r;
-            const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, r);
-            const uint32_t q = quant8(v[u], r);
-            if (rr < nrows && col < a.k)
-                *reinterpret_cast<uint32_t*>(a.codes + (int64_t)(r0 + rr) * kbytes + col / 2) = q;
-            const uint32_t s1 = __shfl_down_sync(kFull, sf, 2);
-            const uint32_t s2 = __shfl_down_sync(kFull, sf, 4);
-            const uint32_t s3 = __shfl_down_sync(kFull, sf, 6);
-            const int scol = seg * 16 + (lane >> 1);
-            if ((lane & 7) == 0 && scol < a.scale_cols) {
-                const uint32_t word = (rr < nrows) ? (sf | (s1 << 8) | (s2 << 16) | (s3 << 24)) : 0u;
-                *reinterpret_cast<uint32_t*>(a.scales + sf_tile_offset(srow0 + rr, scol, a.scale_cols)) = word;
-            }
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            tp[u].advance(drow, dseg, nseg);
+            load_block16(a, r0, nrows, tp[u], lane, pol, v[u][0], v[u][1]);
         }
     }
     pdl_launch_dependents();
@@ -360,8 +411,8 @@ nvfp4_status_t run_amax(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, 
     a.gscale = gscale;
     const int64_t chunks = rows * (k / 8);
     const int64_t per_group = (chunks + groups - 1) / groups;
-    const int gx = clamp_grid((per_group + kThreads * kUnroll - 1) / (kThreads * kUnroll),
-                              (int64_t)num_sms() * 8 / groups);
+    const int gx = clamp_grid((per_group + kThreads * kAmaxUnroll - 1) / (kThreads * kAmaxUnroll),
+                              (int64_t)num_sms() * 4 / groups);
     amax_kernel<<<dim3(gx, groups), kThreads, 0, s>>>(a);
     return cuda_status(cudaGetLastError());
 }
@@ -400,7 +451,7 @@ extern "C" nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_
     q.x = xb;
     q.ld = ld;
     q.k = (int)k;
-    q.nseg = (int)nseg;
+    q.nseg = (int)((k + 511) / 512);
     q.scale_cols = (int)(round_up(k / 16, 4));
     q.groups.offsets = group_offsets;
     q.groups.rows = (int)rows;
@@ -410,9 +461,10 @@ extern "C" nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_
     q.gscale = global_scale;
     q.codes = codes;
     q.scales = scales;
-    const int64_t tasks = (round_up(rows, 128) + (group_offsets ? 127 * (int64_t)groups : 0)) * nseg;
+    const int64_t tasks = (round_up(rows, 128) + (group_offsets ? 127 * (int64_t)groups : 0)) * q.nseg;
     const int64_t per_group = (tasks + groups - 1) / groups;
-    const int qx = clamp_grid((per_group + kWarps * kUnroll - 1) / (kWarps * kUnroll), (int64_t)num_sms() * 8 / groups);
+    const int qx = clamp_grid((per_group + kWarps * kQuantUnroll - 1) / (kWarps * kQuantUnroll),
+                              (int64_t)num_sms() * 4 / groups);
     void* args[] = {&q};
     return cuda_status(launch_pdl(reinterpret_cast<const void*>(&quant1d_kernel), dim3(qx, groups), dim3(kThreads),
                                   args, s));
