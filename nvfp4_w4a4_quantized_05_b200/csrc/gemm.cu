@@ -356,23 +356,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
             for (int kt = 0; kt < p.num_kt; ++kt, ++ktg) {
                 const uint32_t sb = ktg & 1u, su = ktg >> 1;
-                if (!mbar_wait(&tail->full[stage], phase, limit) ||
-                    !mbar_wait(&tail->sf_empty[sb], (su & 1u) ^ 1u, limit) || tail->abort_flag) {
+                // read the stage's scale words first, then wait for the buffer
+                if (!mbar_wait(&tail->full[stage], phase, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sSFA = smem_u32(smem + stage * C::STAGE_BYTES) + C::A_BYTES + C::B_BYTES;
+                const uint32_t sSFB = sSFA + C::SFA_BYTES;
+                uint4 wa[4], wb[4][NSFB];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) wa[j] = ld_shared_v4(sSFA + j * 512 + lane * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int rb = 0; rb < NSFB; ++rb) wb[j][rb] = ld_shared_v4(sSFB + rb * 2048 + j * 512 + lane * 16);
+                if (!mbar_wait(&tail->sf_empty[sb], (su & 1u) ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t sSFA = smem_u32(smem + stage * C::STAGE_BYTES) + C::A_BYTES + C::B_BYTES;
-                const uint32_t sSFB = sSFA + C::SFA_BYTES;
                 const uint32_t dst = tq + sb * C::SF_COLS;
 #pragma unroll
-                for (int j = 0; j < 4; ++j) tmem_st_32x32b_x4(dst + j * 4, ld_shared_v4(sSFA + j * 512 + lane * 16));
+                for (int j = 0; j < 4; ++j) tmem_st_32x32b_x4(dst + j * 4, wa[j]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
-                    for (int rb = 0; rb < NSFB; ++rb)
-                        tmem_st_32x32b_x4(dst + 16 + j * 4 * NSFB + rb * 4,
-                                          ld_shared_v4(sSFB + rb * 2048 + j * 512 + lane * 16));
+                    for (int rb = 0; rb < NSFB; ++rb) tmem_st_32x32b_x4(dst + 16 + j * 4 * NSFB + rb * 4, wb[j][rb]);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -475,6 +484,327 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// ---- pair kernel: 2-SM tcgen05 MMA (M = 256 over a CTA pair) ------------------------
+//
+// A cluster of two CTAs on two SMs computes a 256 x BN output tile: CTA r loads
+// A rows [128r, 128r + 128) and B rows [r * BN/2, (r + 1) * BN/2) of the tile
+// (so per SM the operand traffic per MMA is a third lower than the single-CTA
+// 128 x BN tile), the leader (rank 0) issues tcgen05.mma.cta_group::2, and
+// each CTA ends up with its 128 rows x BN columns of FP32 accumulator in its
+// own tensor memory.  Both CTAs' operand loads complete on the leader's "full"
+// barrier; the leader's MMA commits arrive on both CTAs' barriers.  Each CTA
+// stages, at the same tensor-memory address as its peer, the scale factors of
+// its own 128 A rows and of all BN columns of B (the B codes are split over
+// the pair, but each SM's MMA datapath reads every column's B scales from its
+// own tensor memory).  Tensor memory per CTA: two 192-column accumulators and
+// three 40-column scale buffers (16 for A, 6 per k-step for B).
+struct PairCfg {
+    static constexpr int BN = 192;                    // pair tile width
+    static constexpr int BH = BN / 2;                 // B rows loaded per CTA
+    static constexpr int STAGES = 6;
+    static constexpr int NSB = 3;                     // scale buffers in tensor memory
+    static constexpr int NBC = BN / 32;               // B scale columns per k-step (all BN columns)
+    static constexpr uint32_t A_BYTES = 128 * 128;
+    static constexpr uint32_t B_BYTES = BH * 128;
+    static constexpr uint32_t SFA_BYTES = 4 * 512;
+    static constexpr uint32_t SFB_BYTES = 2 * 4 * 512;    // BN rows starting at 0 or 64 in a block: <= 2 blocks
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr uint32_t SF_COLS = 16 + 4 * NBC;
+    static constexpr uint32_t SF_BASE = 2 * BN;        // two accumulator buffers first
+    static constexpr uint32_t EPI_BYTES = 4 * 2 * 2048;
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static_assert(SF_BASE + NSB * SF_COLS <= kTmemCols, "tensor memory budget");
+    static_assert(BN % 64 == 0 && BN <= 192, "B tile starts at row 0 or 64 of a scale block and spans <= 2");
+    static_assert(NBC == 6, "scale staging writes 4 + 2 columns per k-step");
+};
+
+struct alignas(8) PairTail {
+    uint64_t full[PairCfg::STAGES];      // leader: both CTAs' A/B bytes
+    uint64_t empty[PairCfg::STAGES];     // each CTA: released by the leader's MMA commit
+    uint64_t sfl[PairCfg::STAGES];       // each CTA: its own scale bytes landed
+    uint64_t acc_full[2];                // each CTA: accumulator buffer ready
+    uint64_t acc_empty[2];               // leader: 8 epilogue warps released it
+    uint64_t sf_ready[PairCfg::NSB];     // leader: 8 scale warps staged a buffer
+    uint64_t sf_free[PairCfg::NSB];      // each CTA: MMAs reading a scale buffer done
+    uint32_t tmem_base;
+    volatile int abort_flag;
+};
+
+template <class P>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
+    constexpr int BN = P::BN, BH = P::BH, STAGES = P::STAGES, NBC = P::NBC;
+    constexpr uint32_t IDESC = idesc_mxf4nvf4(256, BN);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* epi_smem = smem + STAGES * P::STAGE_BYTES;
+    PairTail* tail = reinterpret_cast<PairTail*>(epi_smem + P::EPI_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&tail->full[s], 1);
+            mbar_init(&tail->empty[s], 1);
+            mbar_init(&tail->sfl[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tail->acc_full[b], 1);
+            mbar_init(&tail->acc_empty[b], 8);
+        }
+        for (int b = 0; b < P::NSB; ++b) {
+            mbar_init(&tail->sf_ready[b], 8);
+            mbar_init(&tail->sf_free[b], 1);
+        }
+        tail->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tail->tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    pdl_wait();
+    tc_fence_before();
+    cluster_sync();          // both CTAs' barriers initialized, tensor memory allocated
+    tc_fence_after();
+    const uint32_t tmem = tail->tmem_base;
+    const int tiles_m2 = (p.rows_a + 255) / 256;
+    const int total = tiles_m2 * p.tiles_n;
+    const int sfa_blocks = (p.rows_a + 127) / 128;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int t = cluster; t < total && ok; t += nclusters) {
+                const int tm = t % tiles_m2, tn = t / tiles_m2;
+                const int a_row = tm * 256 + 128 * (int)rank;
+                const int g0 = tn * BN + BH * (int)rank;          // first B row of this CTA's half
+                const bool sfa_ok = a_row / 128 < sfa_blocks;
+                const int a0 = (tn * BN) / 128;                   // B scales: all BN rows of the tile
+                const int nsfb = max(0, min(((tn * BN) % 128 + BN + 127) / 128, p.sfb_rb_per_group - a0));
+                const uint8_t* sfa_src = p.sfa + (int64_t)(a_row / 128) * p.sfa_rb_stride;
+                const uint8_t* sfb_src = p.sfb + (int64_t)a0 * p.sfb_rb_stride;
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    const int nat = min(4, p.num_ks - kt * 4);
+                    uint8_t* sA = smem + stage * P::STAGE_BYTES;
+                    uint8_t* sB = sA + P::A_BYTES;
+                    uint8_t* sSFA = sB + P::B_BYTES;
+                    uint8_t* sSFB = sSFA + P::SFA_BYTES;
+                    const uint32_t full0 = mapa_shared(smem_u32(&tail->full[stage]), 0);
+                    if (leader) mbar_arrive_expect_tx(&tail->full[stage], 2u * (P::A_BYTES + P::B_BYTES));
+                    tma_load_2d_pair(sA, &tmA, full0, kt * 128, a_row);
+                    tma_load_2d_pair(sB, &tmB, full0, kt * 128, g0);
+                    uint64_t* sbar = &tail->sfl[stage];
+                    const uint32_t sbytes = (uint32_t)nat * 512u * ((sfa_ok ? 1u : 0u) + (uint32_t)nsfb);
+                    mbar_arrive_expect_tx(sbar, sbytes);
+                    if (sfa_ok) bulk_load(sSFA, sfa_src + (int64_t)kt * 2048, (uint32_t)nat * 512u, sbar);
+                    for (int rb = 0; rb < nsfb; ++rb)
+                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * 2048,
+                                  (uint32_t)nat * 512u, sbar);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                tail->abort_flag = 1;
+                if (p.err) atomicOr(p.err, 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            // ---------------- MMA issuer (pair leader) ----------------
+            uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = cluster; t < total && ok; t += nclusters, ++it) {
+                const uint32_t ab = (uint32_t)(it & 1), au = (uint32_t)(it >> 1);
+                if (!mbar_wait(&tail->acc_empty[ab], (au & 1u) ^ 1u, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem + ab * BN;
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait(&tail->full[stage], phase, limit) ||
+                        !mbar_wait(&tail->sf_ready[sb], sph, limit) || tail->abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nat = min(4, p.num_ks - kt * 4);
+                    const uint32_t sA = smem_u32(smem + stage * P::STAGE_BYTES);
+                    const uint32_t sB = sA + P::A_BYTES;
+                    const uint32_t sf = tmem + P::SF_BASE + sb * P::SF_COLS;
+                    for (int j = 0; j < nat; ++j)
+                        mma_mxf4nvf4_pair(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
+                                          IDESC, sf + j * 4, sf + 16 + j * NBC, (kt > 0 || j > 0) ? 1u : 0u);
+                    tc_commit_pair(&tail->empty[stage], 0x3);
+                    tc_commit_pair(&tail->sf_free[sb], 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++sb == (uint32_t)P::NSB) {
+                        sb = 0;
+                        sph ^= 1u;
+                    }
+                }
+                if (ok) tc_commit_pair(&tail->acc_full[ab], 0x3);
+            }
+            if (!ok) {
+                tail->abort_flag = 1;
+                if (p.err) atomicOr(p.err, 1u);
+            }
+        }
+    } else if (warp >= 6) {
+        // ---------------- scale staging (both CTAs; warps 6..9, one lane quarter each) ----------------
+        const int q = warp & 3;
+        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + P::SF_BASE;
+        const uint32_t ready0 = mapa_shared(smem_u32(&tail->sf_ready[0]), 0);
+        const uint32_t ready_step = (uint32_t)(smem_u32(&tail->sf_ready[1]) - smem_u32(&tail->sf_ready[0]));
+        uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
+        bool ok = true;
+        for (int t = cluster; t < total && ok; t += nclusters) {
+            const int tn = t / tiles_m2;
+            const int off = (tn * BN) % 128;                  // first tile row inside the first scale block
+            for (int kt = 0; kt < p.num_kt; ++kt) {
+                // read this k-tile's scale words as soon as they land, then wait
+                // for the tensor-memory buffer: only the stores stay on the
+                // MMA's critical path
+                if (!mbar_wait(&tail->sfl[stage], phase, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sSFA = smem_u32(smem + stage * P::STAGE_BYTES) + P::A_BYTES + P::B_BYTES;
+                const uint32_t sSFB = sSFA + P::SFA_BYTES;
+                uint4 wa[4];
+                uint32_t wb[4][NBC];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) wa[j] = ld_shared_v4(sSFA + j * 512 + lane * 16);
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int c = 0; c < NBC; ++c) {
+                        // tile row 32c + lane of B: its 4 scales of k-step j
+                        const int rr = off + 32 * c + lane;           // row relative to the first loaded block
+                        const uint32_t addr = sSFB + (uint32_t)((rr >> 7) * 2048 + j * 512 + (rr & 31) * 16 +
+                                                                ((rr >> 5) & 3) * 4);
+                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(wb[j][c]) : "r"(addr));
+                    }
+                if (!mbar_wait(&tail->sf_free[sb], sph ^ 1u, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dst = tq + sb * P::SF_COLS;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tmem_st_32x32b_x4(dst + j * 4, wa[j]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    tmem_st_32x32b_x4(dst + 16 + j * NBC, make_uint4(wb[j][0], wb[j][1], wb[j][2], wb[j][3]));
+                    tmem_st_32x32b_x2(dst + 16 + j * NBC + 4, wb[j][4], wb[j][5]);
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(ready0 + sb * ready_step);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++sb == (uint32_t)P::NSB) {
+                    sb = 0;
+                    sph ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            tail->abort_flag = 1;
+            if (p.err) atomicOr(p.err, 1u);
+        }
+    } else if (warp >= 2) {
+        // ---------------- epilogue (both CTAs; warps 2..5) ----------------
+        const int q = warp & 3;
+        const int rloc = q * 32 + lane;
+        const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * 4096u;
+        const uint32_t empty0 = mapa_shared(smem_u32(&tail->acc_empty[0]), 0);
+        const uint32_t empty_step = (uint32_t)(smem_u32(&tail->acc_empty[1]) - smem_u32(&tail->acc_empty[0]));
+        int it = 0;
+        for (int t = cluster; t < total; t += nclusters, ++it) {
+            const int tm = t % tiles_m2, tn = t / tiles_m2;
+            const uint32_t ab = (uint32_t)(it & 1), au = (uint32_t)(it >> 1);
+            if (!mbar_wait(&tail->acc_full[ab], au & 1u, limit) || tail->abort_flag) {
+                if (lane == 0) {
+                    tail->abort_flag = 1;
+                    if (p.err) atomicOr(p.err, 1u);
+                }
+                break;
+            }
+            tc_fence_after();
+            const int a_row0 = tm * 256 + 128 * (int)rank;
+            const int n0 = tn * BN;
+            const int a_rows = p.rows_a - a_row0;
+            const int b_cols = min(BN, p.rows_b - n0);
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
+            const float alpha = __fmul_rn(p.ga[0], p.gb[0]);
+#pragma unroll 1
+            for (int ch = 0; ch < BN / 32; ++ch) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tq + ch * 32, v);
+                tmem_ld_wait();
+                if (ch * 32 >= b_cols || q * 32 >= a_rows) continue;   // uniform per warp
+                const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint4 w;
+                    w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * alpha, __uint_as_float(v[8 * j + 1]) * alpha);
+                    w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * alpha, __uint_as_float(v[8 * j + 3]) * alpha);
+                    w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * alpha, __uint_as_float(v[8 * j + 5]) * alpha);
+                    w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * alpha, __uint_as_float(v[8 * j + 7]) * alpha);
+                    st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmC, box, n0 + ch * 32, a_row0 + q * 32);
+                    bulk_commit_group();
+                }
+            }
+            (void)rloc;
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
+        }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();          // no CTA leaves while its peer may still touch its shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
 // ---- host side -----------------------------------------------------------------
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -526,6 +856,53 @@ nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args));
+}
+
+constexpr size_t kPairSmem = 1024 + (size_t)PairCfg::STAGES * PairCfg::STAGE_BYTES + PairCfg::EPI_BYTES + sizeof(PairTail);
+static_assert(kPairSmem <= 232448, "shared memory");
+
+cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kPairSmem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cfg;
+}
+
+// Number of CTA pairs that can be resident at once (one CTA per SM), per device.
+int pair_clusters_resident() {
+    static std::mutex mu;
+    static int cached[64] = {};
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[d] == 0) {
+        auto kern = gemm_pair_kernel<PairCfg>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
+            return 0;
+        cudaLaunchAttribute attr[2];
+        cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return 0;
+        cached[d] = n;
+    }
+    return cached[d];
+}
+
+nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
+                           int clusters, cudaStream_t s) {
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = pair_config(clusters, s, attr);
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairCfg>, ta, tb, tc, args));
 }
 
 // Kernel configurations: prefill / grouped use 128 x 192 tiles with two
@@ -608,6 +985,28 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         if (bn == 16) return launch<CfgDec16, true, false>(ta, tb, tc, p, grid, s);
         if (bn == 32) return launch<CfgDec32, true, false>(ta, tb, tc, p, grid, s);
         return launch<CfgDec64, true, false>(ta, tb, tc, p, grid, s);
+    }
+    if (m > 128) {
+        // prefill-class: 2-SM pair tiles of 256 x 224
+        const int clusters_max = pair_clusters_resident();
+        if (clusters_max > 0) {
+            if (!make_codes_map(&ta, a_codes, m, k / 2, 128) ||
+                !make_codes_map(&tb, b_codes, n, k / 2, PairCfg::BH) || !make_out_map(&tc, c, m, n, ldc))
+                return NVFP4_ERR_CUDA;
+            p.sfa = a_scales;
+            p.sfb = b_scales;
+            p.sfb_rb_per_group = (int)((n + 127) / 128);
+            p.ga = a_global;
+            p.gb = b_global;
+            p.rows_a = (int)m;
+            p.rows_b = (int)n;
+            p.tiles_m = (int)((m + 255) / 256);
+            p.tiles_n = (int)((n + PairCfg::BN - 1) / PairCfg::BN);
+            const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
+            if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+            const int clusters = (int)std::min<int64_t>(tiles, std::min(clusters_max, sms / 2));
+            return launch_pair(ta, tb, tc, p, clusters, s);
+        }
     }
     constexpr int BN = CfgWide::BN;
     if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN) ||
