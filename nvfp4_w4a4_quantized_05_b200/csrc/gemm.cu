@@ -168,6 +168,7 @@ struct Cfg {
     static constexpr uint32_t SFB_BYTES = NSFB * 4 * 512;
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t SF_COLS = 16 + 16 * NSFB;       // tensor-memory columns per k-tile of scales
+    static constexpr uint32_t SF_STRIDE = (SF_COLS + 31) / 32 * 32;   // buffers start 32-column aligned
     static constexpr uint32_t SF_BASE = ACC * BN;             // first scale column
     // epilogue staging: per epilogue warp two 32-row x 64-byte BF16 boxes
     static constexpr uint32_t EPI_BYTES = 4 * 2 * 2048;
@@ -175,9 +176,11 @@ struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(STAGES <= kMaxStages, "stages");
     static_assert(ACC == 1 || ACC == 2, "accumulator buffers");
-    static_assert(SF_BASE + 2 * SF_COLS <= kTmemCols, "tensor memory budget");
+    static_assert(SF_BASE + 2 * SF_STRIDE <= kTmemCols, "tensor memory budget");
+    static_assert(SF_BASE % 32 == 0, "wide tensor-memory stores start at a multiple of their width");
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 232448, "shared memory");
+    static_assert(SF_COLS == 32 || SF_COLS == 48, "scale staging writes 32 (+16) columns per k-tile");
 };
 
 template <class C, bool SWAP, bool GROUPED>
@@ -332,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int nat = min(4, p.num_ks - kt * 4);
                     const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
                     const uint32_t sB = sA + C::A_BYTES;
-                    const uint32_t sf = tmem + C::SF_BASE + sb * C::SF_COLS;
+                    const uint32_t sf = tmem + C::SF_BASE + sb * C::SF_STRIDE;
                     for (int j = 0; j < nat; ++j)
                         mma_mxf4nvf4(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32), IDESC,
                                      sf + j * 4, sf + sfb_off + j * 4 * NSFB, (kt > 0 || j > 0) ? 1u : 0u);
@@ -363,25 +366,35 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t sSFA = smem_u32(smem + stage * C::STAGE_BYTES) + C::A_BYTES + C::B_BYTES;
                 const uint32_t sSFB = sSFA + C::SFA_BYTES;
-                uint4 wa[4], wb[4][NSFB];
+                // one k-tile of scales in tensor-memory column order: A k-step j at 4j,
+                // B k-step j, 128-row block rb at 16 + 4 * NSFB * j + 4 * rb
+                uint32_t w[C::SF_COLS];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) wa[j] = ld_shared_v4(sSFA + j * 512 + lane * 16);
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = ld_shared_v4(sSFA + j * 512 + lane * 16);
+                    w[4 * j + 0] = v.x;
+                    w[4 * j + 1] = v.y;
+                    w[4 * j + 2] = v.z;
+                    w[4 * j + 3] = v.w;
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
-                    for (int rb = 0; rb < NSFB; ++rb) wb[j][rb] = ld_shared_v4(sSFB + rb * 2048 + j * 512 + lane * 16);
+                    for (int rb = 0; rb < NSFB; ++rb) {
+                        const uint4 v = ld_shared_v4(sSFB + rb * 2048 + j * 512 + lane * 16);
+                        w[16 + 4 * NSFB * j + 4 * rb + 0] = v.x;
+                        w[16 + 4 * NSFB * j + 4 * rb + 1] = v.y;
+                        w[16 + 4 * NSFB * j + 4 * rb + 2] = v.z;
+                        w[16 + 4 * NSFB * j + 4 * rb + 3] = v.w;
+                    }
                 if (!mbar_wait(&tail->sf_empty[sb], (su & 1u) ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t dst = tq + sb * C::SF_COLS;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tmem_st_32x32b_x4(dst + j * 4, wa[j]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-#pragma unroll
-                    for (int rb = 0; rb < NSFB; ++rb) tmem_st_32x32b_x4(dst + 16 + j * 4 * NSFB + rb * 4, wb[j][rb]);
+                const uint32_t dst = tq + sb * C::SF_STRIDE;
+                tmem_st_32x32b_x32(dst, w);
+                if constexpr (C::SF_COLS == 48) tmem_st_32x32b_x16(dst + 32, w + 32);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -497,12 +510,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // its own 128 A rows and of all BN columns of B (the B codes are split over
 // the pair, but each SM's MMA datapath reads every column's B scales from its
 // own tensor memory).  Tensor memory per CTA: two 192-column accumulators and
-// three 40-column scale buffers (16 for A, 6 per k-step for B).
+// two scale buffers of 40 columns (16 for A, 6 per k-step for B) at a
+// 64-column stride.
 struct PairCfg {
     static constexpr int BN = 192;                    // pair tile width
     static constexpr int BH = BN / 2;                 // B rows loaded per CTA
     static constexpr int STAGES = 6;
-    static constexpr int NSB = 3;                     // scale buffers in tensor memory
+    static constexpr int NSB = 2;                     // scale buffers in tensor memory
     static constexpr int NBC = BN / 32;               // B scale columns per k-step (all BN columns)
     static constexpr uint32_t A_BYTES = 128 * 128;
     static constexpr uint32_t B_BYTES = BH * 128;
@@ -510,12 +524,14 @@ struct PairCfg {
     static constexpr uint32_t SFB_BYTES = 2 * 4 * 512;    // BN rows starting at 0 or 64 in a block: <= 2 blocks
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t SF_COLS = 16 + 4 * NBC;
+    static constexpr uint32_t SF_STRIDE = 64;          // buffers start 32-column aligned
     static constexpr uint32_t SF_BASE = 2 * BN;        // two accumulator buffers first
     static constexpr uint32_t EPI_BYTES = 4 * 2 * 2048;
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-    static_assert(SF_BASE + NSB * SF_COLS <= kTmemCols, "tensor memory budget");
+    static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols && SF_COLS <= SF_STRIDE, "tensor memory budget");
+    static_assert(SF_BASE % 32 == 0, "wide tensor-memory stores start at a multiple of their width");
     static_assert(BN % 64 == 0 && BN <= 192, "B tile starts at row 0 or 64 of a scale block and spans <= 2");
-    static_assert(NBC == 6, "scale staging writes 4 + 2 columns per k-step");
+    static_assert(SF_COLS == 40, "scale staging writes 32 + 8 columns per k-tile");
 };
 
 struct alignas(8) PairTail {
@@ -649,7 +665,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int nat = min(4, p.num_ks - kt * 4);
                     const uint32_t sA = smem_u32(smem + stage * P::STAGE_BYTES);
                     const uint32_t sB = sA + P::A_BYTES;
-                    const uint32_t sf = tmem + P::SF_BASE + sb * P::SF_COLS;
+                    const uint32_t sf = tmem + P::SF_BASE + sb * P::SF_STRIDE;
                     for (int j = 0; j < nat; ++j)
                         mma_mxf4nvf4_pair(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
                                           IDESC, sf + j * 4, sf + 16 + j * NBC, (kt > 0 || j > 0) ? 1u : 0u);
@@ -692,10 +708,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 const uint32_t sSFA = smem_u32(smem + stage * P::STAGE_BYTES) + P::A_BYTES + P::B_BYTES;
                 const uint32_t sSFB = sSFA + P::SFA_BYTES;
-                uint4 wa[4];
-                uint32_t wb[4][NBC];
+                // one k-tile of scales, in tensor-memory column order: A k-step j at
+                // 4j, B k-step j at 16 + NBC * j (column c = tile rows 32c..32c+31)
+                uint32_t w[P::SF_COLS];
 #pragma unroll
-                for (int j = 0; j < 4; ++j) wa[j] = ld_shared_v4(sSFA + j * 512 + lane * 16);
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = ld_shared_v4(sSFA + j * 512 + lane * 16);
+                    w[4 * j + 0] = v.x;
+                    w[4 * j + 1] = v.y;
+                    w[4 * j + 2] = v.z;
+                    w[4 * j + 3] = v.w;
+                }
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
 #pragma unroll
@@ -704,21 +727,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const int rr = off + 32 * c + lane;           // row relative to the first loaded block
                         const uint32_t addr = sSFB + (uint32_t)((rr >> 7) * 2048 + j * 512 + (rr & 31) * 16 +
                                                                 ((rr >> 5) & 3) * 4);
-                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(wb[j][c]) : "r"(addr));
+                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w[16 + NBC * j + c]) : "r"(addr));
                     }
                 if (!mbar_wait(&tail->sf_free[sb], sph ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t dst = tq + sb * P::SF_COLS;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) tmem_st_32x32b_x4(dst + j * 4, wa[j]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    tmem_st_32x32b_x4(dst + 16 + j * NBC, make_uint4(wb[j][0], wb[j][1], wb[j][2], wb[j][3]));
-                    tmem_st_32x32b_x2(dst + 16 + j * NBC + 4, wb[j][4], wb[j][5]);
-                }
+                // two wide stores: each tcgen05.st costs about the same regardless of width
+                const uint32_t dst = tq + sb * P::SF_STRIDE;
+                tmem_st_32x32b_x32(dst, w);
+                tmem_st_32x32b_x8(dst + 32, w + 32);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();

@@ -16,8 +16,9 @@
 // the codes and scale bytes are bit-identical to the CPU definition.
 //
 // Memory-bound design.  Kernel 1 (amax) runs as one wave of CTAs that stream
-// the tensor with 16-byte loads, 8 in flight per thread, tagged L2::evict_last
-// so the tensor stays in the 126 MB L2 for the second pass; it ends with a
+// the tensor with 16-byte loads, 8 in flight per thread, keeping a packed
+// BF16 running max (max.xorsign.abs.bf16x2: one instruction per 2 x 2 values);
+// the tensor normally stays in the 126 MB L2 for the second pass.  It ends with a
 // "last CTA" step that publishes g, writes the group scale offsets and
 // re-zeroes the workspace.  Kernel 2 (quantize) is launched with programmatic
 // dependent launch: its CTAs issue their first loads (tagged evict_first)
@@ -60,23 +61,45 @@ struct Groups {
 
 __device__ __forceinline__ int round128(int v) { return (v + 127) & ~127; }
 
-// |x| of two packed BF16 values as two 16-bit patterns; for non-negative
-// BF16 the bit patterns order like the values, so max is an unsigned max.
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4& v) {
-    const uint32_t m = 0x7FFF7FFFu;
-    uint32_t a = __vmaxu2(v.x & m, v.y & m);
-    a = __vmaxu2(a, __vmaxu2(v.z & m, v.w & m));
-    return max(a & 0xFFFFu, a >> 16);
+// max(|a|, |b|) lane-wise on packed BF16 pairs (exact; the sign bit of the
+// result is the xor of the input signs and is cleared by absmax_bits).
+__device__ __forceinline__ uint32_t bmax_abs(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t absmax8_packed(const uint4& v) {
+    return bmax_abs(bmax_abs(v.x, v.y), bmax_abs(v.z, v.w));
+}
+// Packed BF16 magnitudes -> the larger one as a 16-bit pattern (for
+// non-negative BF16 the bit patterns order like the values).
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t packed) {
+    const uint32_t m = packed & 0x7FFF7FFFu;
+    return max(m & 0xFFFFu, m >> 16);
+}
+__device__ __forceinline__ uint32_t absmax8_bits(const uint4& v) { return absmax_bits(absmax8_packed(v)); }
+
+// (lo, hi) BF16 pair times (r, r): two IEEE round-to-nearest products.
+__device__ __forceinline__ void mul_bf16x2(uint32_t w, uint64_t rr, float& lo, float& hi) {
+    uint64_t x, y;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(rr));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(y));
+}
+__device__ __forceinline__ uint64_t pack_rr(float r) {
+    uint64_t rr;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(rr) : "f"(r));
+    return rr;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-
 // Eight BF16 values times r -> eight packed E2M1 codes.
-__device__ __forceinline__ uint32_t quant8(const uint4& v, float r) {
-    return cvt_e2m1x8(__fmul_rn(bf16_lo(v.x), r), __fmul_rn(bf16_hi(v.x), r), __fmul_rn(bf16_lo(v.y), r),
-                      __fmul_rn(bf16_hi(v.y), r), __fmul_rn(bf16_lo(v.z), r), __fmul_rn(bf16_hi(v.z), r),
-                      __fmul_rn(bf16_lo(v.w), r), __fmul_rn(bf16_hi(v.w), r));
+__device__ __forceinline__ uint32_t quant8(const uint4& v, uint64_t rr) {
+    float x[8];
+    mul_bf16x2(v.x, rr, x[0], x[1]);
+    mul_bf16x2(v.y, rr, x[2], x[3]);
+    mul_bf16x2(v.z, rr, x[4], x[5]);
+    mul_bf16x2(v.w, rr, x[6], x[7]);
+    return cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
 }
 
 // Block scale byte and element multiplier from the block amax.
@@ -153,8 +176,7 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(AmaxArgs a) {
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     const bool dense = (a.ld == (int64_t)a.k);
     const uint16_t* base = a.x + (int64_t)r0 * a.ld;
-    const uint64_t pol = l2_policy_evict_last();
-    uint32_t m = 0;
+    uint32_t acc = 0;   // packed BF16 running max of |x|
     for (int64_t i0 = (int64_t)blockIdx.x * kThreads + threadIdx.x; i0 < items; i0 += stride * kAmaxUnroll) {
         uint4 v[kAmaxUnroll];
 #pragma unroll
@@ -169,12 +191,13 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(AmaxArgs a) {
                     const int64_t r = i / kc;
                     p = base + r * a.ld + (i - r * kc) * 8;
                 }
-                v[u] = ld_nc_v4_hint(p, pol);
+                v[u] = ld_nc_v4(p);
             }
         }
 #pragma unroll
-        for (int u = 0; u < kAmaxUnroll; ++u) m = max(m, absmax8_bits(v[u]));
+        for (int u = 0; u < kAmaxUnroll; ++u) acc = bmax_abs(acc, absmax8_packed(v[u]));
     }
+    uint32_t m = absmax_bits(acc);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
     __shared__ uint32_t red[kWarps];
@@ -284,13 +307,14 @@ __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
             const TaskPos t = tp[u];
             if (t.row >= prows) break;   // uniform across the warp
             const int col = t.seg * 512 + lane * 16;
-            uint32_t am = max(absmax8_bits(v[u][0]), absmax8_bits(v[u][1]));
+            const uint32_t am = absmax_bits(bmax_abs(absmax8_packed(v[u][0]), absmax8_packed(v[u][1])));
             float r;
             const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, r);
             if (t.row < nrows && col < a.k) {
+                const uint64_t rr = pack_rr(r);
                 uint2 q;
-                q.x = quant8(v[u][0], r);
-                q.y = quant8(v[u][1], r);
+                q.x = quant8(v[u][0], rr);
+                q.y = quant8(v[u][1], rr);
                 *reinterpret_cast<uint2*>(a.codes + (int64_t)(r0 + t.row) * kbytes + col / 2) = q;
             }
             const uint32_t s1 = __shfl_down_sync(kFull, sf, 1);
@@ -339,17 +363,19 @@ __global__ void __launch_bounds__(kThreads) quant2d_kernel(Quant2dArgs a) {
 #pragma unroll
         for (int i = 0; i < 16; ++i)
             v[i] = valid ? ld_nc_v4(a.x + (int64_t)(tr * 16 + i) * a.ld + col) : make_uint4(0, 0, 0, 0);
-        uint32_t am = 0;
+        uint32_t pm = 0;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) am = max(am, absmax8_bits(v[i]));
+        for (int i = 0; i < 16; ++i) pm = bmax_abs(pm, absmax8_packed(v[i]));
+        uint32_t am = absmax_bits(pm);
         am = max(am, __shfl_xor_sync(kFull, am, 1));
         float r;
         const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, r);
+        const uint64_t rr = pack_rr(r);
         if (valid) {
 #pragma unroll
             for (int i = 0; i < 16; ++i)
                 *reinterpret_cast<uint32_t*>(a.codes + (int64_t)(tr * 16 + i) * kbytes + col / 2) =
-                    quant8(v[i], r);
+                    quant8(v[i], rr);
             if (a.compact && (lane & 1) == 0) a.compact[(int64_t)tr * (a.k / 16) + col / 16] = (uint8_t)sf;
         }
         const uint32_t s1 = __shfl_down_sync(kFull, sf, 2);
