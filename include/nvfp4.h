@@ -42,10 +42,12 @@
  *     that ran out) are reported by nvfp4_get_last_device_error.
  *   - Global scales and group offsets stay on the device: no call waits on
  *     the host for them.
- *   - workspace: device scratch of nvfp4_workspace_bytes(...) bytes.  It must
- *     be zero before its first use (nvfp4_workspace_init); every call that
- *     returns NVFP4_OK leaves it zero again.  Calls sharing one workspace
- *     must be ordered on one stream.
+ *   - workspace: device scratch of nvfp4_workspace_bytes(...) bytes, for one
+ *     device.  It must be zero before its first use (nvfp4_workspace_init);
+ *     after that, leave it untouched between calls: every call that returns
+ *     NVFP4_OK leaves it ready for the next (the one-tensor quantizer keeps a
+ *     per-CTA generation count in it).  Calls sharing one workspace must be
+ *     ordered on one stream.
  */
 #ifndef NVFP4_H
 #define NVFP4_H
@@ -118,8 +120,13 @@ nvfp4_status_t nvfp4_workspace_init(void* workspace, size_t bytes, void* stream)
  *                every byte of each group's padded scale block is written.
  *   global_scale device, FP32 [max(1, num_groups)].
  *   workspace    nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_ACT, rows, 0, k, num_groups).
- * Two kernels: a tensor-amax reduction, then the quantizer (launched with
- * programmatic dependent launch so its start overlaps the reduction's end).
+ * One tensor (group_offsets NULL): one cooperative launch, one CTA per SM
+ * (amax pass, a grid barrier through the workspace, quantize pass); the
+ * launch waits until every SM can take its CTA.  Row groups: two kernels, a
+ * per-group amax reduction, then the quantizer (launched with programmatic
+ * dependent launch so its start overlaps the reduction's end).
+ * After nvfp4_get_last_device_error reports NVFP4_ERR_TIMEOUT, initialize the
+ * workspace again before reusing it.
  */
 nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_t ld,
                                   const int32_t* group_offsets, int num_groups,
@@ -133,7 +140,7 @@ nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_
  * owns every byte of device memory and hands out no allocator, or a
  * latency-critical path that may not call cudaMalloc (it can synchronize the
  * whole device).
- *   Scratch: a fixed 8448-byte array in the library's device image (each GPU
+ *   Scratch: a fixed 41216-byte array in the library's device image (each GPU
  *   that loads the library holds it until the process exits), enough for at
  *   most 1024 row groups; num_groups > 1024 returns
  *   NVFP4_ERR_UNSUPPORTED_SHAPE.

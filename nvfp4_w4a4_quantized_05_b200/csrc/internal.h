@@ -1,6 +1,8 @@
 // internal.h -- host-side helpers shared by the translation units of libnvfp4.
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <cstdint>
 
@@ -15,6 +17,9 @@ unsigned int* device_error_word();
 // Number of SMs of the current device (cached per device).
 int num_sms();
 
+// The driver's cuTensorMapEncodeTiled (looked up once), or nullptr.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
 // Current limit of the bounded waits, in ns.
 uint64_t wait_limit_ns();
 
@@ -25,11 +30,21 @@ constexpr int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 inline nvfp4_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
 // Workspace layout of the quantizers (bytes):
-//   [0, 4)         CTA completion counter (uint32)
+//   [0, 4)         CTA completion counter (two-kernel path) or grid-barrier
+//                  arrivals (one-launch path), uint32
+//   [4, 8)         grid-barrier departures (one-launch path), uint32
 //   [16, 16+4G)    per-group amax as FP32 bit patterns (uint32)
 //   [pad_off, +4(G+1))  per-group first scale row (int32), written each call
+//   [part_off, +128*kMaxFusedCtas)  one-launch path: the word of CTA c at
+//                  part_off + 128 c (one per 128-byte line, so that pollers
+//                  spread over the L2 slices)
+constexpr int kMaxFusedCtas = 256;
+constexpr int kPartStrideWords = 32;
 constexpr int64_t quant_ws_amax_off() { return 16; }
 constexpr int64_t quant_ws_pad_off(int groups) { return round_up(16 + 4 * (int64_t)groups, 16); }
-constexpr int64_t quant_ws_bytes(int groups) { return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 256); }
+constexpr int64_t quant_ws_part_off(int groups) { return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 128); }
+constexpr int64_t quant_ws_bytes(int groups) {
+    return round_up(quant_ws_part_off(groups) + 4 * (int64_t)kPartStrideWords * kMaxFusedCtas, 256);
+}
 
 }  // namespace nvfp4

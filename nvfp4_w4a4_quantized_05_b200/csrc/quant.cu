@@ -10,24 +10,30 @@
 //     sf   = e4m3_rn_satfinite(block_amax / (6 g))
 //     d    = float(sf) * g ;  r = d == 0 ? 0 : min(1 / d, FLT_MAX)
 //     code = e2m1_rn_satfinite(x * r)
-// Every step is one IEEE binary32 operation rounded to nearest even
-// (__fdiv_rn / __fmul_rn / __frcp_rn, compiled with -fmad=false), and the
-// roundings to E4M3 / E2M1 are the hardware cvt.rn.satfinite instructions, so
-// the codes and scale bytes are bit-identical to the CPU definition.
+// Every step rounds as one IEEE binary32 operation to nearest even would
+// (compiled with -fmad=false), and the roundings to E4M3 / E2M1 are the
+// hardware cvt.rn.satfinite instructions, so the codes and scale bytes are
+// bit-identical to the CPU definition.  Two steps take an exact shortcut:
+// the block-scale quotient is bracketed between two products with the
+// reciprocal (the division runs only when the bracket straddles an E4M3
+// rounding boundary), and r comes from a 128-entry table per global scale.
 //
-// Memory-bound design.  Kernel 1 (amax) runs as one wave of CTAs that stream
-// the tensor with 16-byte loads, 8 in flight per thread, keeping a packed
-// BF16 running max (max.xorsign.abs.bf16x2: one instruction per 2 x 2 values);
-// the tensor normally stays in the 126 MB L2 for the second pass.  It ends with a
-// "last CTA" step that publishes g, writes the group scale offsets and
-// re-zeroes the workspace.  Kernel 2 (quantize) is launched with programmatic
-// dependent launch: its CTAs issue their first loads (tagged evict_first)
-// before waiting for kernel 1, since only g depends on it.  A warp task is
-// 512 consecutive elements of one row; lane l owns 16-element block l (two
-// 16-byte loads), so the block amax, the E4M3 scale and the reciprocal are
-// computed once per block; the 16 codes leave as one 8-byte store (the warp
-// writes 256 contiguous bytes) and 4 scale bytes are gathered by shuffles
-// into one word of the 512-byte scale tile.  Task stepping is division-free.
+// One tensor (the activation path): one cooperative launch, one CTA per SM.
+// Pass 1 streams the tensor from HBM through per-warp shared-memory slots for
+// the amax and keeps ~45% of it on chip; a grid barrier in the workspace
+// (one generation-tagged word per CTA) hands every CTA the same g; pass 2
+// quantizes the on-chip part, then the rest re-read from L2 by TMA.  A warp
+// task is 1024 values of one row; lane l owns blocks 2 l and 2 l + 1, so its
+// 16 code bytes leave in one store and two lanes make one 4-byte word of the
+// 512-byte scale tile.
+//
+// Row groups (MoE activations) and shapes outside the one-launch layout
+// (k % 64 != 0, very large tensors): kernel 1 reduces per-group amaxes with
+// 16-byte loads, 8 in flight per thread, and a "last CTA" step publishes the
+// global scales and group scale offsets; kernel 2 (programmatic dependent
+// launch) issues its first loads before waiting for kernel 1, then quantizes
+// with one 16-value block per lane.  Weights: 16 x 16 blocks, one scale per
+// tile written to each of its 16 rows.
 #include <cuda_runtime.h>
 #include <cfloat>
 #include <cstdint>
@@ -77,7 +83,6 @@ __device__ __forceinline__ uint32_t absmax_bits(uint32_t packed) {
     const uint32_t m = packed & 0x7FFF7FFFu;
     return max(m & 0xFFFFu, m >> 16);
 }
-__device__ __forceinline__ uint32_t absmax8_bits(const uint4& v) { return absmax_bits(absmax8_packed(v)); }
 
 // (lo, hi) BF16 pair times (r, r): two IEEE round-to-nearest products.
 __device__ __forceinline__ void mul_bf16x2(uint32_t w, uint64_t rr, float& lo, float& hi) {
@@ -102,7 +107,8 @@ __device__ __forceinline__ uint32_t quant8(const uint4& v, uint64_t rr) {
     return cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
 }
 
-// Block scale byte and element multiplier from the block amax.
+// Block scale byte and element multiplier from the block amax (exact IEEE steps;
+// used by the 16 x 16 weight quantizer, where it runs once per 256 values).
 __device__ __forceinline__ uint32_t block_scale(float bamax, float g, float k6, float& r) {
     const uint32_t sf = cvt_e4m3(__fdiv_rn(bamax, k6));
     const float d = __fmul_rn(e4m3_to_f32(sf), g);
@@ -110,9 +116,94 @@ __device__ __forceinline__ uint32_t block_scale(float bamax, float g, float k6, 
     return sf;
 }
 
+// Per-CTA constants of the 1D block quantizer for one global scale g.
+struct BlockQ {
+    float k6;           // 6 g
+    uint64_t inv_lo2;   // (il, il): il = RN(RN(1 / (6 g)) * (1 - 2^-20)); 0 when 6 g is subnormal
+    uint64_t inv_hi2;   // (ih, ih): ih = RN(RN(1 / (6 g)) * (1 + 2^-20)); +inf when 6 g is subnormal
+};
+__device__ __forceinline__ BlockQ make_blockq(float g) {
+    BlockQ c;
+    c.k6 = __fmul_rn(6.0f, g);
+    float il = 0.0f, ih = __int_as_float(0x7F800000);
+    if (c.k6 >= FLT_MIN) {   // else RN(1 / (6 g)) may overflow: every block takes the division
+        const float inv = __frcp_rn(c.k6);
+        il = __fmul_rn(inv, 1.0f - 0x1p-20f);
+        ih = __fmul_rn(inv, 1.0f + 0x1p-20f);
+    }
+    c.inv_lo2 = pack_rr(il);
+    c.inv_hi2 = pack_rr(ih);
+    return c;
+}
+
+// sf = e4m3_rn_satfinite(RN(bamax / (6 g))), bit-exact, mostly without a
+// division.  lo = RN(bamax * il) and hi = RN(bamax * ih) bracket the correctly
+// rounded quotient strictly (il and ih are within 2^-21 relative of 1 / (6 g)
+// on either side, far more than the 2^-24 error of each rounding), and
+// rounding to E4M3 is monotone: when lo and hi round to the same byte, so does
+// the quotient.  Otherwise (an E4M3 rounding boundary within ~2^-20 relative,
+// or 6 g subnormal) the exact IEEE quotient is rounded.
+__device__ __forceinline__ uint32_t block_sf(float bamax, const BlockQ& c) {
+    const uint32_t lo = cvt_e4m3(__fmul_rn(bamax, __uint_as_float((uint32_t)c.inv_lo2)));
+    const uint32_t hi = cvt_e4m3(__fmul_rn(bamax, __uint_as_float((uint32_t)c.inv_hi2)));
+    return lo == hi ? lo : cvt_e4m3(__fdiv_rn(bamax, c.k6));
+}
+// The scale bytes of two blocks, sf0 | sf1 << 8: both brackets with two paired
+// multiplies and two paired conversions, one branch for both.
+__device__ __forceinline__ uint32_t block_sf2(float b0, float b1, const BlockQ& c) {
+    uint64_t bb, lo, hi;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(bb) : "f"(b0), "f"(b1));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(lo) : "l"(bb), "l"(c.inv_lo2));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(hi) : "l"(bb), "l"(c.inv_hi2));
+    float lo0, lo1, hi0, hi1;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo0), "=f"(lo1) : "l"(lo));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(hi0), "=f"(hi1) : "l"(hi));
+    const uint32_t plo = cvt_e4m3x2(lo1, lo0);
+    if (plo == cvt_e4m3x2(hi1, hi0)) return plo;
+    return cvt_e4m3x2(__fdiv_rn(b1, c.k6), __fdiv_rn(b0, c.k6));
+}
+
+// rtab[sf] = (r, r) for a block with scale byte sf: d = float(sf) * g,
+// r = d == 0 ? 0 : min(1 / d, FLT_MAX), stored as the FP32 pair that the paired
+// multiplies take.  128 entries (bytes 0..127; 127 is never produced by the
+// saturating conversion).  Threads 0..127 fill it.
+__device__ __forceinline__ void fill_rtab(uint64_t* rtab, float g, int tid) {
+    if (tid < 128) {
+        const float d = __fmul_rn(e4m3_to_f32((uint32_t)tid), g);
+        rtab[tid] = pack_rr((d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX));
+    }
+}
+
 __device__ __forceinline__ int64_t sf_tile_offset(int srow, int scol, int scale_cols) {
     return ((int64_t)(srow >> 7) * (scale_cols >> 2) + (scol >> 2)) * 512 + (srow & 31) * 16 +
            ((srow >> 5) & 3) * 4 + (scol & 3);
+}
+
+// One warp task: 512 consecutive values of one row, segment seg.  Lane l holds
+// block l (values v0, v1) and quantizes it; its 8 code bytes leave in one store
+// (the warp writes 256 contiguous bytes) and lanes 4i store the scale word of
+// blocks 4i..4i+3.  Rows past the tensor (row_ok false) and columns past k hold
+// zeros, so they produce zero scale bytes for the padded scale tile.  valid
+// false (warp-uniform) stores nothing: callers run a fixed number of tasks
+// side by side without branches between them.
+__device__ __forceinline__ void quantize_task(const uint4& v0, const uint4& v1, bool row_ok, int seg, int lane,
+                                              int k, int scale_cols, uint8_t* code_row, uint8_t* scales, int srow,
+                                              const BlockQ& c, const uint64_t* rtab, bool valid = true) {
+    const uint32_t am = absmax_bits(bmax_abs(absmax8_packed(v0), absmax8_packed(v1)));
+    const uint32_t sf = block_sf(__uint_as_float(am << 16), c);
+    const int col = seg * 512 + lane * 16;
+    if (valid && row_ok && col < k) {
+        const uint64_t rr = rtab[sf];
+        uint2 q;
+        q.x = quant8(v0, rr);
+        q.y = quant8(v1, rr);
+        *reinterpret_cast<uint2*>(code_row + col / 2) = q;
+    }
+    const uint32_t p = sf | (__shfl_down_sync(kFull, sf, 1) << 8);
+    const uint32_t word = p | (__shfl_down_sync(kFull, p, 2) << 16);
+    const int scol = seg * 32 + lane;
+    if (valid && (lane & 3) == 0 && scol < scale_cols)
+        *reinterpret_cast<uint32_t*>(scales + sf_tile_offset(srow, scol, scale_cols)) = word;
 }
 
 // Exclusive prefix over groups of round128(group rows), by one CTA.
@@ -299,38 +390,381 @@ __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
     pdl_wait();   // g (and the group scale offsets) come from amax_kernel
     const int srow0 = a.pad_rows ? a.pad_rows[e] : 0;
     const float g = a.gscale[e];
-    const float k6 = __fmul_rn(6.0f, g);
+    __shared__ uint64_t rtab[128];
+    fill_rtab(rtab, g, threadIdx.x);
+    const BlockQ c = make_blockq(g);
+    __syncthreads();
 
     while (tp[0].row < prows) {
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
             const TaskPos t = tp[u];
             if (t.row >= prows) break;   // uniform across the warp
-            const int col = t.seg * 512 + lane * 16;
-            const uint32_t am = absmax_bits(bmax_abs(absmax8_packed(v[u][0]), absmax8_packed(v[u][1])));
-            float r;
-            const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, r);
-            if (t.row < nrows && col < a.k) {
-                const uint64_t rr = pack_rr(r);
-                uint2 q;
-                q.x = quant8(v[u][0], rr);
-                q.y = quant8(v[u][1], rr);
-                *reinterpret_cast<uint2*>(a.codes + (int64_t)(r0 + t.row) * kbytes + col / 2) = q;
-            }
-            const uint32_t s1 = __shfl_down_sync(kFull, sf, 1);
-            const uint32_t s2 = __shfl_down_sync(kFull, sf, 2);
-            const uint32_t s3 = __shfl_down_sync(kFull, sf, 3);
-            const int scol = t.seg * 32 + lane;
-            if ((lane & 3) == 0 && scol < a.scale_cols) {
-                const uint32_t word = (t.row < nrows) ? (sf | (s1 << 8) | (s2 << 16) | (s3 << 24)) : 0u;
-                *reinterpret_cast<uint32_t*>(a.scales + sf_tile_offset(srow0 + t.row, scol, a.scale_cols)) = word;
-            }
+            quantize_task(v[u][0], v[u][1], t.row < nrows, t.seg, lane, a.k, a.scale_cols,
+                          a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row, c, rtab);
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
             tp[u].advance(drow, dseg, nseg);
             load_block16(a, r0, nrows, tp[u], lane, pol, v[u][0], v[u][1]);
         }
+    }
+    pdl_launch_dependents();
+}
+
+// ---- one launch for one tensor: amax, grid barrier, quantize ---------------------
+//
+// One CTA of 1024 threads per SM (the grid is launched cooperatively, so all CTAs
+// are resident together).  A warp task is 1024 consecutive values of one row;
+// lane l owns values 32 l .. 32 l + 31 of it, i.e. blocks 2 l and 2 l + 1, so its
+// 16 code bytes leave in one store and two lanes make one scale word.  CTA c
+// owns a contiguous range of tasks and warp w of it a contiguous run of those.
+// Each warp owns kStage task slots of shared memory (2 KB each; 192 KB per SM)
+// and streams its tasks through them, kStage tasks in flight.  Pass 1 copies
+// with cp.async (each lane moves 16-byte units lane, 32 + lane, ...; zero fill
+// past the tensor) and reduces each landed task to the amax; the warp's last
+// kStage tasks stay in their slots (~28 MB of the tensor on chip across the
+// GPU).  A grid barrier in the
+// workspace publishes the per-CTA amaxes; every CTA reduces them in the same
+// order, so all hold the same g.  Pass 2 quantizes the tasks still on chip
+// first, refilling each freed slot with one of the warp's other tasks by TMA
+// (one 3-D box per task, 128-byte swizzle, zero fill past the tensor; L2 hits:
+// the tensor was just read), then works through those as they land.
+constexpr int kFThreads = 1024;
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kTaskVals = 1024;                  // values per warp task
+constexpr int kTaskBytes = kTaskVals * 2;
+constexpr int kStage = 3;                        // task slots per warp
+
+struct FusedArgs {
+    const uint16_t* x;
+    int64_t ld;
+    int rows, k, nseg, scale_cols;
+    int tasks;        // round128(rows) * nseg
+    int full_segs;    // segments that need no guards: k / 1024
+    uint32_t sc4x512; // (scale_cols / 4) * 512: bytes of one 128-row band of scale tiles
+    float* gscale;
+    uint8_t* codes;
+    uint8_t* scales;
+    uint32_t* part;   // per-CTA generation | amax words, 32 words apart
+    uint64_t limit;
+    unsigned* err;
+};
+
+// A task sits in its slot as 16 rows of 128 bytes (64 values each) in the TMA
+// 128-byte swizzle: 16-byte unit u (values 8 u .. 8 u + 7) at unit
+// (u & ~7) | ((u & 7) ^ ((u >> 3) & 7)).  Lane l reads units 4 l .. 4 l + 3 and
+// copies units 32 i + l; either way every 8-lane phase touches 8 distinct
+// 16-byte bank groups.
+__device__ __forceinline__ int slot_unit(int u) { return (u & ~7) | ((u & 7) ^ ((u >> 3) & 7)); }
+
+// Per-lane constants of the one-launch path.
+struct LaneC {
+    int lane;
+    uint32_t ld_off[4];   // byte offsets of units 4 lane + i in a slot
+    uint32_t st_off[4];   // byte offsets of units 32 i + lane in a slot
+    uint32_t s_off;       // (lane / 2) * 512: the lane pair's scale tile within the segment
+};
+__device__ __forceinline__ LaneC make_lanec(int lane) {
+    LaneC lc;
+    lc.lane = lane;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        lc.ld_off[i] = (uint32_t)slot_unit(4 * lane + i) * 16u;
+        lc.st_off[i] = (uint32_t)slot_unit(32 * i + lane) * 16u;
+    }
+    lc.s_off = (uint32_t)(lane >> 1) * 512u;
+    return lc;
+}
+
+// Task positions walk one task at a time, row-major over (row, segment).
+struct SrcCursor {   // which box a task's values come from
+    int row, seg;
+    __device__ __forceinline__ void init(const FusedArgs& a, int t) {
+        row = t / a.nseg;
+        seg = t - row * a.nseg;
+    }
+    __device__ __forceinline__ void next(const FusedArgs& a) {
+        if (++seg == a.nseg) {
+            seg = 0;
+            ++row;
+        }
+    }
+};
+struct DstCursor {   // where a task's codes and scale words go (32-bit byte offsets)
+    int row, seg;
+    uint32_t co;     // row * k / 2 + seg * 512
+    uint32_t so;     // scale word of the segment's first four blocks
+    __device__ __forceinline__ void set_row(const FusedArgs& a) {
+        const uint32_t r = (uint32_t)row;
+        co = r * (uint32_t)(a.k >> 1) + ((uint32_t)seg << 9);
+        so = (r >> 7) * a.sc4x512 + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + ((uint32_t)seg << 13);
+    }
+    __device__ __forceinline__ void init(const FusedArgs& a, int t) {
+        row = t / a.nseg;
+        seg = t - row * a.nseg;
+        set_row(a);
+    }
+    __device__ __forceinline__ void next(const FusedArgs& a) {
+        if (++seg == a.nseg) {
+            seg = 0;
+            ++row;
+            set_row(a);
+        } else {
+            co += kTaskVals / 2;
+            so += 8192u;   // 16 scale tiles of 512 bytes per segment
+        }
+    }
+};
+
+// Quantize the task held in slot sb.  FULL: the whole task is inside the tensor.
+template <bool FULL>
+__device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb, const DstCursor& t,
+                                              const LaneC& lc, const BlockQ& c, const uint64_t* rtab) {
+    uint4 u[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4*>(sb + lc.ld_off[i]);
+    // Packed maxima of |x| per block, then both blocks' halves against each other:
+    // m = (amax of block 2 lane + 1 in the high half, of block 2 lane in the low).
+    const uint32_t m0 = bmax_abs(absmax8_packed(u[0]), absmax8_packed(u[1]));
+    const uint32_t m1 = bmax_abs(absmax8_packed(u[2]), absmax8_packed(u[3]));
+    const uint32_t m = bmax_abs(__byte_perm(m0, m1, 0x5410), __byte_perm(m0, m1, 0x7632));
+    const float b0 = __uint_as_float((m << 16) & 0x7FFF0000u);
+    const float b1 = __uint_as_float(m & 0x7FFF0000u);
+    const uint32_t pair = block_sf2(b0, b1, c);   // scale bytes of blocks 2 lane, 2 lane + 1
+    const uint64_t rr0 = rtab[pair & 0xFFu], rr1 = rtab[pair >> 8];
+    uint4 q;
+    q.x = quant8(u[0], rr0);
+    q.y = quant8(u[1], rr0);
+    q.z = quant8(u[2], rr1);
+    q.w = quant8(u[3], rr1);
+    const uint32_t word = __byte_perm(pair, __shfl_down_sync(kFull, pair, 1), 0x5410);
+    const bool even = (lc.lane & 1) == 0;
+    uint8_t* dst = a.codes + t.co + 16 * lc.lane;
+    uint32_t* sw = reinterpret_cast<uint32_t*>(a.scales + t.so + lc.s_off);
+    if (FULL) {
+        *reinterpret_cast<uint4*>(dst) = q;
+        if (even) *sw = word;
+    } else {
+        // Rows past the tensor and values past k arrived as zeros: their scale
+        // bytes are 0, as the padded scale tile wants; no codes are stored there.
+        if (t.row < a.rows && t.seg * kTaskVals + 32 * lc.lane < a.k) *reinterpret_cast<uint4*>(dst) = q;
+        if (even && t.seg * (kTaskVals / 16) + 2 * lc.lane < a.scale_cols) *sw = word;
+    }
+}
+__device__ __forceinline__ void quantize_any(const FusedArgs& a, const char* sb, const DstCursor& t,
+                                             const LaneC& lc, const BlockQ& c, const uint64_t* rtab) {
+    if (t.row < a.rows && t.seg < a.full_segs)
+        quantize_slot<true>(a, sb, t, lc, c, rtab);
+    else
+        quantize_slot<false>(a, sb, t, lc, c, rtab);
+}
+
+// Grid barrier and amax reduction in one: CTA c publishes its word (part
+// + 32 c, one per 128-byte line) = gen << 16 | (its BF16 amax bits), so a reader that sees this call's
+// generation also sees the amax.  gen is one more (mod 2^16) than the
+// generation of the CTA's own word from the previous call (0 in a fresh
+// workspace), the same for every CTA.  Warp 0 of each CTA polls all G words
+// until every one carries gen; false if that wait ran out (error word set).
+__device__ __forceinline__ bool grid_amax(uint32_t* part, int G, uint32_t gen, uint64_t limit, unsigned* err,
+                                          int lane, uint32_t& amax_bits) {
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        bool mine = true;
+        uint32_t mx = 0;
+        for (int i = lane; i < G; i += 32) {
+            const uint32_t w = ld_relaxed_gpu_u32(part + kPartStrideWords * i);
+            mine = mine && (w >> 16) == gen;
+            mx = max(mx, w & 0xFFFFu);
+        }
+        if (__all_sync(kFull, mine)) {
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o));
+            amax_bits = mx;
+            return true;
+        }
+        if (globaltimer_ns() - t0 > limit) {
+            if (lane == 0) atomicOr(err, 1u);
+            return false;
+        }
+    }
+}
+
+// A warp's slot ring: slot s is kTaskBytes at base + (warp + 32 s) * kTaskBytes,
+// filled by one TMA box and completed on bar[s].
+struct Ring {
+    char* base;
+    uint64_t* bar;     // this warp's kStage barriers
+    int warp;
+    uint32_t phase;    // bit s: parity of the next completion of slot s
+    uint32_t box_bytes;
+    __device__ __forceinline__ char* slot(int s) const { return base + (warp + 32 * s) * kTaskBytes; }
+};
+// Lane 0 starts the copy of task t into slot s; the warp's reads of the slot's
+// previous task are done (the caller's __syncwarp).
+__device__ __forceinline__ void stage(const CUtensorMap* tmap, Ring& r, int s, const SrcCursor& t, uint64_t pol,
+                                      int lane) {
+    if (lane == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&r.bar[s], r.box_bytes);
+        tma_load_3d(r.slot(s), tmap, &r.bar[s], 0, t.seg * (kTaskVals / 64), t.row, pol);
+    }
+}
+// Wait (bounded) until the copy into slot s has landed.
+__device__ __forceinline__ void land(Ring& r, int s, const FusedArgs& a) {
+    if (!mbar_wait(&r.bar[s], (r.phase >> s) & 1u, a.limit)) atomicOr(a.err, 1u);
+    r.phase ^= 1u << s;
+}
+
+// Pass 1 copy: the warp starts the cp.async copy of task t into slot s.
+__device__ __forceinline__ void stage_cp(const FusedArgs& a, const Ring& r, int s, const SrcCursor& t,
+                                         const LaneC& lc, uint64_t pol) {
+    const uint16_t* p = a.x + (int64_t)t.row * a.ld + t.seg * kTaskVals + 8 * lc.lane;
+    const uint32_t d = smem_u32(r.slot(s));
+    const bool row_in = t.row < a.rows;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool in = row_in && t.seg * kTaskVals + 256 * i + 8 * lc.lane < a.k;
+        cp_async16(d + lc.st_off[i], in ? p + 256 * i : a.x, in ? 16u : 0u, pol);
+    }
+}
+
+// Pass 2 of one warp with tasks tw .. tw + n - 1, the last nres = min(kStage, n)
+// of them still on chip: task n - nres + k is in slot (n - nres + k) % kStage.
+// Quantizing it frees the slot for task k of the n - nres others, and then
+// task q of the others follows task q - kStage through the same slot.
+__device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const FusedArgs& a, Ring& r,
+                                            const uint64_t* rtab, const BlockQ& c, int tw, int n, const LaneC& lc) {
+    const uint64_t pol = l2_policy_evict_first();   // last use
+    const int nres = n < kStage ? n : kStage;
+    const int nl = n - nres;
+    DstCursor rp, lq;
+    SrcCursor lp;
+    rp.init(a, tw + n - nres);
+    lq.init(a, tw);
+    lp.init(a, tw);
+    int s = (n - nres) % kStage;
+    for (int k = 0; k < nres; ++k) {
+        quantize_any(a, r.slot(s), rp, lc, c, rtab);
+        rp.next(a);
+        __syncwarp();   // every lane is done reading the slot
+        if (k < nl) {
+            stage(tmap, r, s, lp, pol, lc.lane);
+            lp.next(a);
+        }
+        s = (s + 1 == kStage) ? 0 : s + 1;
+    }
+    // s is back at the slot of the first on-chip task, where task 0 lands.
+    for (int q = 0; q < nl; ++q) {
+        land(r, s, a);
+        quantize_any(a, r.slot(s), lq, lc, c, rtab);
+        lq.next(a);
+        __syncwarp();
+        if (q + kStage < nl) {
+            stage(tmap, r, s, lp, pol, lc.lane);
+            lp.next(a);
+        }
+        s = (s + 1 == kStage) ? 0 : s + 1;
+    }
+}
+
+__global__ void __launch_bounds__(kFThreads, 1)
+    quant1d_fused_kernel(const __grid_constant__ CUtensorMap tmap, FusedArgs a, uint32_t box_bytes) {
+    extern __shared__ __align__(1024) uint8_t dsm[];   // kStage task slots per warp (+ alignment pad)
+    __shared__ __align__(8) uint64_t sbar[kStage * kFWarps];
+    __shared__ uint64_t rtab[128];
+    __shared__ uint32_t red[kFWarps];
+    __shared__ uint32_t s_amax, s_gen;
+    __shared__ int s_ok;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int G = gridDim.x;
+    const int t0 = (int)((int64_t)a.tasks * blockIdx.x / G);
+    const int cnt = (int)((int64_t)a.tasks * (blockIdx.x + 1) / G) - t0;
+    // Warp w takes a contiguous run of the CTA's tasks.
+    const int tw = t0 + cnt * warp / kFWarps;
+    const int n = t0 + cnt * (warp + 1) / kFWarps - tw;
+    uint32_t gen = 0;
+    if (tid == 0) gen = ((ld_relaxed_gpu_u32(a.part + kPartStrideWords * blockIdx.x) >> 16) + 1u) & 0xFFFFu;
+    if (tid < kStage * kFWarps) mbar_init(&sbar[tid], 1);
+    fence_mbar_init();
+    __syncthreads();
+    Ring r;
+    r.base = reinterpret_cast<char*>(dsm) + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u);   // 128-byte swizzle: 1 KB aligned
+    r.bar = &sbar[warp * kStage];
+    r.warp = warp;
+    r.phase = 0;
+    r.box_bytes = box_bytes;
+    if (lane == 0) prefetch_tmap(&tmap);
+
+    // ---- pass 1: amax through the slot ring; the last kStage tasks stay on chip
+    const LaneC lc = make_lanec(lane);
+    uint32_t acc = 0;
+    {
+        const uint64_t pol_keep = l2_policy_evict_normal();   // read again in pass 2
+        const uint64_t pol_last = l2_policy_evict_first();    // stays on chip: not read again
+        SrcCursor sp;                                         // next task to copy
+        sp.init(a, tw);
+#pragma unroll
+        for (int i = 0; i < kStage; ++i) {
+            if (i < n) {
+                stage_cp(a, r, i, sp, lc, i >= n - kStage ? pol_last : pol_keep);
+                sp.next(a);
+            }
+            cp_async_commit();
+        }
+        // One commit group per step (empty once nothing is left): with at most
+        // kStage - 1 groups pending, the oldest copy has landed.
+        int s = 0;
+        for (int i = 0; i < n; ++i) {
+            cp_async_wait<kStage - 1>();
+            __syncwarp();   // every lane's copies into the slot have landed
+            const char* sb = r.slot(s);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                acc = bmax_abs(acc, absmax8_packed(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q])));
+            if (i + kStage < n) {
+                __syncwarp();   // every lane is done reading the slot
+                stage_cp(a, r, s, sp, lc, i + kStage >= n - kStage ? pol_last : pol_keep);
+                sp.next(a);
+            }
+            cp_async_commit();
+            s = (s + 1 == kStage) ? 0 : s + 1;
+        }
+        cp_async_wait<0>();
+        __syncwarp();
+    }
+    uint32_t m = absmax_bits(acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+
+    // ---- grid barrier: publish this CTA's amax, gather everyone's
+    if (tid == 0) {
+        uint32_t b = red[0];
+        for (int w = 1; w < kFWarps; ++w) b = max(b, red[w]);
+        st_relaxed_gpu_u32(a.part + kPartStrideWords * blockIdx.x, (gen << 16) | b);
+        s_gen = gen;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint32_t amax_bits = 0;
+        const bool got = grid_amax(a.part, G, s_gen, a.limit, a.err, lane, amax_bits);
+        if (lane == 0) {
+            s_ok = got ? 1 : 0;
+            s_amax = amax_bits;
+        }
+    }
+    __syncthreads();
+    const bool ok = s_ok != 0;
+    if (ok) {
+        const float amax = __uint_as_float(s_amax << 16);
+        const float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kGlobalDen);
+        if (blockIdx.x == 0 && tid == 0) a.gscale[0] = g;
+        fill_rtab(rtab, g, tid);
+        const BlockQ c = make_blockq(g);
+        __syncthreads();
+        fused_pass2(&tmap, a, r, rtab, c, tw, n, lc);
     }
     pdl_launch_dependents();
 }
@@ -422,6 +856,86 @@ cudaError_t launch_pdl(const void* func, dim3 grid, dim3 block, void** args, cud
     return cudaLaunchKernelExC(&cfg, func, args);
 }
 
+// One-launch quantization of one tensor.  Returns NVFP4_ERR_UNSUPPORTED_SHAPE
+// (nothing launched) when the tensor does not fit its layout -- k % 64 != 0, or
+// codes / scales too large for 32-bit offsets -- or the device cannot hold one
+// such CTA per SM; the caller then takes the two-kernel path.
+nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes, uint8_t* scales,
+                         float* gscale, void* workspace, cudaStream_t s) {
+    constexpr int kSmemMax = kStage * kFWarps * kTaskBytes + 1024;
+    if (k % 64 != 0 || round_up(rows, 128) * k >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    static std::mutex mu;
+    static int ready[64] = {};   // per device: 0 unknown, 1 usable, -1 not usable
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return NVFP4_ERR_CUDA;
+    {
+        std::lock_guard<std::mutex> lk(mu);
+        if (ready[dev] == 0) {
+            int occ = 0;
+            const bool ok =
+                tensor_map_encoder() != nullptr &&
+                cudaFuncSetAttribute(quant1d_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) ==
+                    cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quant1d_fused_kernel, kFThreads, kSmemMax) ==
+                    cudaSuccess &&
+                occ >= 1;
+            ready[dev] = ok ? 1 : -1;
+        }
+        if (ready[dev] < 0) {
+            cudaGetLastError();
+            return NVFP4_ERR_UNSUPPORTED_SHAPE;
+        }
+    }
+    // x as a 3-D tensor [rows][k / 64][64]: one box = one task (16 x 64 values of a
+    // row; narrower when k < 1024), 128-byte swizzle, zero fill past the tensor.
+    const cuuint32_t box1 = (cuuint32_t)(k / 64 < kTaskVals / 64 ? k / 64 : kTaskVals / 64);
+    CUtensorMap tmap;
+    {
+        const cuuint64_t dims[3] = {64, (cuuint64_t)(k / 64), (cuuint64_t)(rows > 0 ? rows : 1)};
+        const cuuint64_t strides[2] = {128, (cuuint64_t)ld * 2};
+        const cuuint32_t box[3] = {64, box1, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (tensor_map_encoder()(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<uint16_t*>(x), dims, strides,
+                                 box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    }
+    uint32_t box_bytes = box1 * 128u;
+    FusedArgs a;
+    a.x = x;
+    a.ld = ld;
+    a.rows = (int)rows;
+    a.k = (int)k;
+    a.nseg = (int)((k + kTaskVals - 1) / kTaskVals);
+    a.scale_cols = (int)(k / 16);
+    a.tasks = (int)(round_up(rows, 128) * a.nseg);
+    a.full_segs = (int)(k / kTaskVals);
+    a.sc4x512 = (uint32_t)(a.scale_cols / 4) * 512u;
+    const int G = num_sms() < kMaxFusedCtas ? num_sms() : kMaxFusedCtas;
+    const int64_t per = (a.tasks + G - 1) / G;
+    const int64_t per_warp = (per + kFWarps - 1) / kFWarps;
+    const int depth = (int)(per_warp < kStage ? per_warp : kStage);
+    a.gscale = gscale;
+    a.codes = codes;
+    a.scales = scales;
+    a.part = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_part_off(1));
+    a.limit = wait_limit_ns();
+    a.err = device_error_word();
+    if (!a.err) return NVFP4_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kFThreads);
+    cfg.dynamicSmemBytes = (size_t)depth * kFWarps * kTaskBytes + 1024;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs resident at once (grid barrier)
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {&tmap, &a, &box_bytes};
+    return cuda_status(cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&quant1d_fused_kernel), args));
+}
+
 nvfp4_status_t run_amax(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const int32_t* offsets, int groups,
                         void* workspace, float* gscale, cudaStream_t s) {
     AmaxArgs a;
@@ -470,6 +984,10 @@ extern "C" nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_
     if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
+    if (!group_offsets) {
+        const nvfp4_status_t fs = run_fused(xb, rows, k, ld, codes, scales, global_scale, workspace, s);
+        if (fs != NVFP4_ERR_UNSUPPORTED_SHAPE) return fs;
+    }
     nvfp4_status_t st = run_amax(xb, rows, k, ld, group_offsets, groups, workspace, global_scale, s);
     if (st != NVFP4_OK) return st;
 
@@ -552,7 +1070,7 @@ extern "C" nvfp4_status_t nvfp4_probe_cvt(const float* in, uint8_t* out_e2m1, ui
 namespace nvfp4 {
 namespace {
 constexpr int kStaticMaxGroups = 1024;
-constexpr int64_t kStaticScratchBytes = quant_ws_bytes(kStaticMaxGroups);   // 8448 bytes
+constexpr int64_t kStaticScratchBytes = quant_ws_bytes(kStaticMaxGroups);   // 41216 bytes
 std::mutex g_static_mu;
 void* g_static_ptr[64] = {};
 }  // namespace

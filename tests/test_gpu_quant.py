@@ -75,7 +75,9 @@ def test_cvt_e4m3_every_pattern_below_1024():
 
 # ---- 1D activations ------------------------------------------------------------------
 
-@pytest.mark.parametrize("shape", [(16, 256), (1, 16), (3, 48), (130, 320), (257, 4112), (64, 5120), (1, 5120)])
+@pytest.mark.parametrize("shape", [(16, 256), (1, 16), (3, 48), (130, 320), (257, 4112), (64, 5120), (1, 5120),
+                                   (300, 3072), (1000, 2080), (200, 1040), (5000, 3104), (5000, 3136), (700, 1088),
+                                   (129, 960)])
 def test_quantize_act_matches_oracle(shape):
     xb = W.gaussian_bf16(shape, 0, 100 + shape[0], 1.0, outlier_frac=0.01)
     _assert_same_1d(xb)
@@ -113,6 +115,29 @@ def test_quantize_act_edge_values(case):
     _assert_same_1d(xb)
 
 
+@pytest.mark.parametrize("amax_bits", [0x3F80, 0x4340, 0x3B4D, 0x0B00, 0x0080, 0x0001, 0x7F7F])
+def test_block_scale_every_bf16_block_amax(amax_bits):
+    """One block per positive BF16 value up to the tensor amax: each block's
+    amax is that value (at a random position, random sign), so the block
+    scale rounding meets every E4M3 rounding boundary the quotient can hit,
+    exact midpoints included.  Amax 0x0080 / 0x0001 make 6 g subnormal."""
+    rng = np.random.default_rng(amax_bits)
+    pats = np.arange(1, amax_bits + 1, dtype=np.uint32)
+    nb = pats.size
+    bpr = 64                                            # blocks per row: k = 1024
+    rows = -(-nb // bpr)
+    blocks = np.zeros((rows * bpr, 16), np.uint16)
+    peak = (pats << 16).view(np.float32)
+    frac = rng.random((nb, 16), dtype=np.float32)
+    others = ((peak[:, None] * frac).view(np.uint32) >> 16).astype(np.uint16)   # truncation: |v| <= peak
+    others |= (rng.integers(0, 2, size=(nb, 16)) << 15).astype(np.uint16)
+    pos = rng.integers(0, 16, size=nb)
+    others[np.arange(nb), pos] = pats.astype(np.uint16) | (rng.integers(0, 2, size=nb) << 15).astype(np.uint16)
+    blocks[:nb] = others
+    xb = blocks.reshape(rows, bpr * 16)
+    _assert_same_1d(xb)
+
+
 def test_quantize_act_strided_rows():
     import torch
     wide = W.gaussian_bf16((70, 384), 0, 41, 1.0, outlier_frac=0.01)
@@ -125,7 +150,24 @@ def test_quantize_act_strided_rows():
     assert q.global_scale.cpu().numpy()[0] == np.float32(og)
 
 
-def test_workspace_left_zero_and_reusable():
+def test_quantize_act_strided_rows_large():
+    """Row stride > k on a tensor large enough that part of it is re-read from L2."""
+    import torch
+    wide = W.gaussian_bf16((10000, 2176), 0, 43, 1.0, outlier_frac=0.001)
+    x = bf16_to_device(wide)[:, :2048]
+    q = nv.quantize_act(x)
+    torch.cuda.synchronize()
+    nv.check_device_error()
+    oc, osf, og = O.quantize_1d(np.ascontiguousarray(wide[:, :2048]))
+    assert np.array_equal(q.codes.cpu().numpy(), oc)
+    assert np.array_equal(q.scales.cpu().numpy(), osf)
+    assert q.global_scale.cpu().numpy()[0] == np.float32(og)
+
+
+def test_workspace_reusable_across_calls():
+    """The workspace carries state between calls (grid-barrier generations):
+    repeated calls on one workspace, and a re-initialized one, give the
+    oracle's results; the counter words stay zero."""
     import torch
     xb = W.gaussian_bf16((300, 512), 0, 42, 1.0)
     x = bf16_to_device(xb)
@@ -134,14 +176,20 @@ def test_workspace_left_zero_and_reusable():
     codes = torch.empty((300, 256), dtype=torch.uint8, device=dev)
     scales = torch.empty(nv.nvfp4_scale_bytes(300, 512), dtype=torch.uint8, device=dev)
     g = torch.empty(1, dtype=torch.float32, device=dev)
-    for _ in range(3):
+    oc, osf, og = O.quantize_1d(xb)
+    stream = torch.cuda.current_stream().cuda_stream
+    for it in range(5):
+        if it == 3:
+            assert nv.nvfp4_workspace_init(ws.data_ptr(), ws.numel(), stream) == 0
+        codes.fill_(0xAA)
         st = nv.nvfp4_quantize_act(x.data_ptr(), 300, 512, 512, None, 0, codes.data_ptr(), scales.data_ptr(),
-                                   g.data_ptr(), ws.data_ptr(), torch.cuda.current_stream().cuda_stream)
+                                   g.data_ptr(), ws.data_ptr(), stream)
         assert st == 0
         torch.cuda.synchronize()
-        assert int(ws[:16].abs().sum()) == 0 and int(ws.sum()) == 0
-    oc, osf, og = O.quantize_1d(xb)
-    assert np.array_equal(codes.cpu().numpy(), oc) and np.array_equal(scales.cpu().numpy(), osf)
+        nv.check_device_error()
+        assert int(ws[:16].abs().sum()) == 0
+        assert np.array_equal(codes.cpu().numpy(), oc) and np.array_equal(scales.cpu().numpy(), osf)
+        assert g.cpu().numpy()[0] == np.float32(og)
 
 
 # ---- grouped (MoE) ---------------------------------------------------------------------
