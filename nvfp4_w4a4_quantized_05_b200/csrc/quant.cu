@@ -911,6 +911,8 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     a.tasks = (int)(round_up(rows, 128) * a.nseg);
     a.full_segs = (int)(k / kTaskVals);
     a.sc4x512 = (uint32_t)(a.scale_cols / 4) * 512u;
+    // One CTA per SM, for every tensor: the grid-barrier generations live in
+    // the CTAs' own words, so the grid must not change from call to call.
     const int G = num_sms() < kMaxFusedCtas ? num_sms() : kMaxFusedCtas;
     const int64_t per = (a.tasks + G - 1) / G;
     const int64_t per_warp = (per + kFWarps - 1) / kFWarps;
@@ -923,7 +925,7 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     a.err = device_error_word();
     if (!a.err) return NVFP4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(G);
+    cfg.gridDim = dim3((unsigned)G);
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = (size_t)depth * kFWarps * kTaskBytes + 1024;
     cfg.stream = s;
