@@ -512,11 +512,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 // own tensor memory).  Tensor memory per CTA: two 192-column accumulators and
 // two scale buffers of 40 columns (16 for A, 6 per k-step for B) at a
 // 64-column stride.
+template <int BN_, int STAGES_, int NSB_, int ACC_>
 struct PairCfg {
-    static constexpr int BN = 192;                    // pair tile width
+    static constexpr int BN = BN_;                    // pair tile width
     static constexpr int BH = BN / 2;                 // B rows loaded per CTA
-    static constexpr int STAGES = 6;
-    static constexpr int NSB = 2;                     // scale buffers in tensor memory
+    static constexpr int STAGES = STAGES_;
+    static constexpr int NSB = NSB_;                  // scale buffers in tensor memory
+    static constexpr int ACC = ACC_;                  // accumulator buffers in tensor memory
     static constexpr int NBC = BN / 32;               // B scale columns per k-step (all BN columns)
     static constexpr uint32_t A_BYTES = 128 * 128;
     static constexpr uint32_t B_BYTES = BH * 128;
@@ -524,24 +526,32 @@ struct PairCfg {
     static constexpr uint32_t SFB_BYTES = 2 * 4 * 512;    // BN rows starting at 0 or 64 in a block: <= 2 blocks
     static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr uint32_t SF_COLS = 16 + 4 * NBC;
-    static constexpr uint32_t SF_STRIDE = 64;          // buffers start 32-column aligned
-    static constexpr uint32_t SF_BASE = 2 * BN;        // two accumulator buffers first
+    static constexpr uint32_t SF_STRIDE = SF_COLS;     // packed buffers, written with 8-column stores
+    static constexpr uint32_t SF_BASE = ACC * BN;      // accumulator buffers first
     static constexpr uint32_t EPI_BYTES = 4 * 2 * 2048;
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
-    static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols && SF_COLS <= SF_STRIDE, "tensor memory budget");
-    static_assert(SF_BASE % 32 == 0, "wide tensor-memory stores start at a multiple of their width");
-    static_assert(BN % 64 == 0 && BN <= 192, "B tile starts at row 0 or 64 of a scale block and spans <= 2");
-    static_assert(SF_COLS == 40, "scale staging writes 32 + 8 columns per k-tile");
+    static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols, "tensor memory budget");
+    static_assert(SF_BASE % 8 == 0 && SF_STRIDE % 8 == 0, "8-column stores start at a multiple of 8");
+    static_assert(BN % 64 == 0 && (BN <= 192 || BN == 256),
+                  "a B tile starts at row 0 or 64 of a scale block and spans <= 2 blocks");
+    static_assert(ACC == 1 || ACC == 2, "accumulator buffers");
 };
+// 256 x 256 tiles with one accumulator: the kernel is bound by the operand
+// bytes each SM pulls from L2, and a square tile needs 14% fewer of them per
+// flop than 256 x 192 with two accumulators (measured: 149.5 vs 161.8 us on
+// the 4096 x 14336 x 4096 prefill).  While the epilogue drains the
+// accumulator the producer keeps filling the 5 stages.
+using PairUse = PairCfg<256, 5, 4, 1>;
 
+template <class P>
 struct alignas(8) PairTail {
-    uint64_t full[PairCfg::STAGES];      // leader: both CTAs' A/B bytes
-    uint64_t empty[PairCfg::STAGES];     // each CTA: released by the leader's MMA commit
-    uint64_t sfl[PairCfg::STAGES];       // each CTA: its own scale bytes landed
-    uint64_t acc_full[2];                // each CTA: accumulator buffer ready
-    uint64_t acc_empty[2];               // leader: 8 epilogue warps released it
-    uint64_t sf_ready[PairCfg::NSB];     // leader: 8 scale warps staged a buffer
-    uint64_t sf_free[PairCfg::NSB];      // each CTA: MMAs reading a scale buffer done
+    uint64_t full[P::STAGES];        // leader: both CTAs' A/B bytes
+    uint64_t empty[P::STAGES];       // each CTA: released by the leader's MMA commit
+    uint64_t sfl[P::STAGES];         // each CTA: its own scale bytes landed
+    uint64_t acc_full[P::ACC];       // each CTA: accumulator buffer ready
+    uint64_t acc_empty[P::ACC];      // leader: 8 epilogue warps released it
+    uint64_t sf_ready[P::NSB];       // leader: 8 scale warps staged a buffer
+    uint64_t sf_free[P::NSB];        // each CTA: MMAs reading a scale buffer done
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -555,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_smem = smem + STAGES * P::STAGE_BYTES;
-    PairTail* tail = reinterpret_cast<PairTail*>(epi_smem + P::EPI_BYTES);
+    PairTail<P>* tail = reinterpret_cast<PairTail<P>*>(epi_smem + P::EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
@@ -568,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&tail->empty[s], 1);
             mbar_init(&tail->sfl[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < P::ACC; ++b) {
             mbar_init(&tail->acc_full[b], 1);
             mbar_init(&tail->acc_empty[b], 8);
         }
@@ -648,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             int it = 0;
             bool ok = true;
             for (int t = cluster; t < total && ok; t += nclusters, ++it) {
-                const uint32_t ab = (uint32_t)(it & 1), au = (uint32_t)(it >> 1);
+                const uint32_t ab = (uint32_t)(it % P::ACC), au = (uint32_t)(it / P::ACC);
                 if (!mbar_wait(&tail->acc_empty[ab], (au & 1u) ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
                     break;
@@ -734,10 +744,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     break;
                 }
                 tc_fence_after();
-                // two wide stores: each tcgen05.st costs about the same regardless of width
+                // 8-column stores (the buffers are packed SF_COLS columns apart)
                 const uint32_t dst = tq + sb * P::SF_STRIDE;
-                tmem_st_32x32b_x32(dst, w);
-                tmem_st_32x32b_x8(dst + 32, w + 32);
+#pragma unroll
+                for (int i = 0; i < (int)P::SF_COLS / 8; ++i) tmem_st_32x32b_x8(dst + 8 * i, w + 8 * i);
                 tmem_st_wait();
                 tc_fence_before();
                 __syncwarp();
@@ -766,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int it = 0;
         for (int t = cluster; t < total; t += nclusters, ++it) {
             const int tm = t % tiles_m2, tn = t / tiles_m2;
-            const uint32_t ab = (uint32_t)(it & 1), au = (uint32_t)(it >> 1);
+            const uint32_t ab = (uint32_t)(it % P::ACC), au = (uint32_t)(it / P::ACC);
             if (!mbar_wait(&tail->acc_full[ab], au & 1u, limit) || tail->abort_flag) {
                 if (lane == 0) {
                     tail->abort_flag = 1;
@@ -864,7 +874,8 @@ nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args));
 }
 
-constexpr size_t kPairSmem = 1024 + (size_t)PairCfg::STAGES * PairCfg::STAGE_BYTES + PairCfg::EPI_BYTES + sizeof(PairTail);
+constexpr size_t kPairSmem =
+    1024 + (size_t)PairUse::STAGES * PairUse::STAGE_BYTES + PairUse::EPI_BYTES + sizeof(PairTail<PairUse>);
 static_assert(kPairSmem <= 232448, "shared memory");
 
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
@@ -892,7 +903,7 @@ int pair_clusters_resident() {
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return 0;
     std::lock_guard<std::mutex> lk(mu);
     if (cached[d] == 0) {
-        auto kern = gemm_pair_kernel<PairCfg>;
+        auto kern = gemm_pair_kernel<PairUse>;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
             return 0;
         cudaLaunchAttribute attr[2];
@@ -908,7 +919,7 @@ nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const C
                            int clusters, cudaStream_t s) {
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pair_config(clusters, s, attr);
-    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairCfg>, ta, tb, tc, args));
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairUse>, ta, tb, tc, args));
 }
 
 // Kernel configurations: prefill / grouped use 128 x 192 tiles with two
@@ -997,7 +1008,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         const int clusters_max = pair_clusters_resident();
         if (clusters_max > 0) {
             if (!make_codes_map(&ta, a_codes, m, k / 2, 128) ||
-                !make_codes_map(&tb, b_codes, n, k / 2, PairCfg::BH) || !make_out_map(&tc, c, m, n, ldc))
+                !make_codes_map(&tb, b_codes, n, k / 2, PairUse::BH) || !make_out_map(&tc, c, m, n, ldc))
                 return NVFP4_ERR_CUDA;
             p.sfa = a_scales;
             p.sfb = b_scales;
@@ -1007,7 +1018,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
             p.rows_a = (int)m;
             p.rows_b = (int)n;
             p.tiles_m = (int)((m + 255) / 256);
-            p.tiles_n = (int)((n + PairCfg::BN - 1) / PairCfg::BN);
+            p.tiles_n = (int)((n + PairUse::BN - 1) / PairUse::BN);
             const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
             if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
             const int clusters = (int)std::min<int64_t>(tiles, std::min(clusters_max, sms / 2));

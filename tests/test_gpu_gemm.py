@@ -56,6 +56,9 @@ def test_tiny_workload_end_to_end():
     (16, 64, 256),       # swap path, BN 16
     (1, 64, 320),        # single token
     (300, 16, 448),      # narrow n
+    (129, 264, 128),     # 2-SM pair tile with one valid row in its second half
+    (520, 776, 512),     # pair tiles: ragged m (3 row tiles) and n (4th column tile 8 wide)
+    (1000, 2072, 576),   # many pair tiles, both edges ragged, partial last k-tile
 ])
 def test_gemm_matches_oracle(m, n, k):
     (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 0)
