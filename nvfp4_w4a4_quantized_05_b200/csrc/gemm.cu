@@ -36,12 +36,10 @@
 // Every mbarrier wait is bounded (globaltimer); a wait that runs out sets the
 // library's device error word and the CTA winds down instead of hanging.
 //
-// Operand roles: the "A side" fills the 128-row MMA dimension, the "B side" the
-// BN-wide dimension.  Normally A side = activations, B side = weights; for
-// m <= 64 (decode) they swap so the weights stream through the 128-row side
-// and the few tokens sit in a narrow BN, and the epilogue stores transposed.
-// The grouped form walks (expert, m-tile, n-tile) triples built from the
-// device offsets array.
+// Operand roles: the "A side" (activations) fills the 128-row MMA dimension,
+// the "B side" (weights) the BN-wide dimension.  For m > 128 the 2-SM pair
+// kernel below takes over (256-row tiles).  The grouped form walks (expert,
+// m-tile, n-tile) triples built from the device offsets array.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -60,6 +58,7 @@ constexpr int kThreads = 320;         // 10 warps, roles above
 constexpr int kPairThreads = 448;     // pair kernel: 14 warps (8 epilogue warps, scale warps 10-13)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 8;
+constexpr int kMaxScaleBufs = 8;
 constexpr int kMaxGroups = 256;
 
 struct GemmArgs {
@@ -90,8 +89,8 @@ struct alignas(8) SmemTail {
     uint64_t empty[kMaxStages];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
-    uint64_t sf_full[2];
-    uint64_t sf_empty[2];
+    uint64_t sf_full[kMaxScaleBufs];
+    uint64_t sf_empty[kMaxScaleBufs];
     uint32_t tmem_base;
     volatile int abort_flag;
     int total_tiles;
@@ -155,15 +154,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 
 // Compile-time shape of one kernel configuration.
-template <int BN_, int STAGES_, int ACC_>
+template <int BN_, int STAGES_, int ACC_, int NSB_ = 2, int AROWS_ = 128>
 struct Cfg {
+    static constexpr int AROWS = AROWS_;                      // A rows loaded per stage (the MMA reads 128)
     static constexpr int BN = BN_;
     static constexpr int STAGES = STAGES_;
     static constexpr int ACC = ACC_;                          // accumulator buffers in tensor memory
+    static constexpr int NSB = NSB_;                          // scale buffers in tensor memory
     // 128-row scale blocks a B tile can touch: tiles start at multiples of BN,
     // i.e. at a row offset 0 or 64 inside a block for BN = 192.
     static constexpr int NSFB = BN == 192 ? 2 : (BN + 127) / 128;
-    static constexpr uint32_t A_BYTES = 128 * 128;            // 128 rows x 256 FP4
+    static constexpr uint32_t A_BYTES = AROWS * 128;          // AROWS rows x 256 FP4
     static constexpr uint32_t B_BYTES = BN * 128;
     static constexpr uint32_t SFA_BYTES = 4 * 512;            // 4 k-steps x (128 rows x 4 scales)
     static constexpr uint32_t SFB_BYTES = NSFB * 4 * 512;
@@ -177,21 +178,21 @@ struct Cfg {
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(STAGES <= kMaxStages, "stages");
     static_assert(ACC == 1 || ACC == 2, "accumulator buffers");
-    static_assert(SF_BASE + 2 * SF_STRIDE <= kTmemCols, "tensor memory budget");
+    static_assert(NSB >= 2 && NSB <= kMaxScaleBufs, "scale buffers");
+    static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols, "tensor memory budget");
     static_assert(SF_BASE % 32 == 0, "wide tensor-memory stores start at a multiple of their width");
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
     static_assert(SMEM <= 232448, "shared memory");
     static_assert(SF_COLS == 32 || SF_COLS == 48, "scale staging writes 32 (+16) columns per k-tile");
 };
 
-template <class C, bool SWAP, bool GROUPED>
+template <class C, bool GROUPED>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
     constexpr int BN = C::BN, STAGES = C::STAGES, ACC = C::ACC, NSFB = C::NSFB;
     constexpr int CW = BN >= 32 ? 32 : 16;                   // epilogue column chunk
     constexpr uint32_t IDESC = idesc_mxf4nvf4(128, BN);
-    static_assert(!(SWAP && GROUPED), "swap form is for the plain GEMM");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -208,6 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tail->acc_full[b], 1);
             mbar_init(&tail->acc_empty[b], 4);
+        }
+        for (int b = 0; b < C::NSB; ++b) {
             mbar_init(&tail->sf_full[b], 4);
             mbar_init(&tail->sf_empty[b], 1);
         }
@@ -215,7 +218,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_mbar_init();
         prefetch_tmap(&tmA);
         prefetch_tmap(&tmB);
-        if (!SWAP) prefetch_tmap(&tmC);
+        prefetch_tmap(&tmC);
     }
     if (warp == 1) {
         tmem_alloc(&tail->tmem_base, kTmemCols);
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t d_tmem = tmem + ab * BN;
                 const uint32_t sfb_off = 16 + (uint32_t)((ti.b_col0 % 128) / 32);
                 for (int kt = 0; kt < p.num_kt; ++kt, ++ktg) {
-                    const uint32_t sb = ktg & 1u, su = ktg >> 1;
+                    const uint32_t sb = ktg % C::NSB, su = ktg / C::NSB;
                     if (!mbar_wait(&tail->full[stage], phase, limit) ||
                         !mbar_wait(&tail->sf_full[sb], su & 1u, limit) || tail->abort_flag) {
                         ok = false;
@@ -359,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
             for (int kt = 0; kt < p.num_kt; ++kt, ++ktg) {
-                const uint32_t sb = ktg & 1u, su = ktg >> 1;
+                const uint32_t sb = ktg % C::NSB, su = ktg / C::NSB;
                 // read the stage's scale words first, then wait for the buffer
                 if (!mbar_wait(&tail->full[stage], phase, limit) || tail->abort_flag) {
                     ok = false;
@@ -409,12 +412,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok && lane == 0) raise_abort(tail, p.err);
     } else {
         // ---------------- epilogue (warps 2..5) ----------------
-        // Non-swapped tiles: each warp converts its 32 rows x 32 columns of
-        // FP32 accumulator to BF16 in a swizzled 2 KB shared-memory box (two
-        // boxes per warp, alternating) and writes it with a TMA tensor store;
-        // the tensor bounds clip ragged tiles.  The last slab of an expert's
-        // rows in the grouped form (rows past the group belong to the next
-        // expert) and the swapped (transposed) decode form use direct stores.
+        // Each warp converts its 32 rows x 32 columns of FP32 accumulator to
+        // BF16 in a swizzled 2 KB shared-memory box (two boxes per warp,
+        // alternating) and writes it with a TMA tensor store; the tensor bounds
+        // clip ragged tiles.  The last slab of an expert's rows in the grouped
+        // form (rows past the group belong to the next expert) uses direct
+        // stores.
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const int rloc = q * 32 + lane;               // A-side row inside the tile
         const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * 4096u;
@@ -431,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
             const float alpha = __fmul_rn(p.ga[ti.group], p.gb[ti.group]);
             const bool a_ok = rloc < ti.a_rows;
-            const bool use_tma = !SWAP && (!GROUPED || q * 32 + 32 <= ti.a_rows);
+            const bool use_tma = !GROUPED || q * 32 + 32 <= ti.a_rows;
 #pragma unroll 1
             for (int ch = 0; ch < BN / CW; ++ch) {
                 uint32_t v[CW];
@@ -441,45 +444,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tmem_ld_32x32b_x16(tq + ch * CW, v);
                 }
                 tmem_ld_wait();
-                if constexpr (!SWAP) {
-                    if (ch * CW >= ti.b_rows) continue;      // uniform: whole chunk past n
-                    if (use_tma) {
-                        const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
-                        if (lane == 0) bulk_wait_group_read<1>();   // the box's previous store has read it
-                        __syncwarp();
+                if (ch * CW >= ti.b_rows) continue;      // uniform: whole chunk past n
+                if (use_tma) {
+                    const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
+                    if (lane == 0) bulk_wait_group_read<1>();   // the box's previous store has read it
+                    __syncwarp();
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint4 w;
-                            w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * alpha, __uint_as_float(v[8 * j + 1]) * alpha);
-                            w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * alpha, __uint_as_float(v[8 * j + 3]) * alpha);
-                            w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * alpha, __uint_as_float(v[8 * j + 5]) * alpha);
-                            w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * alpha, __uint_as_float(v[8 * j + 7]) * alpha);
-                            // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
-                            st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
-                        }
-                        fence_proxy_async_smem();
-                        __syncwarp();
-                        if (lane == 0) {
-                            tma_store_2d(&tmC, box, ti.b_col0 + ch * CW, ti.a_row0 + q * 32);
-                            bulk_commit_group();
-                        }
-                    } else if (a_ok) {
-                        __nv_bfloat16* crow = p.c + (int64_t)(ti.a_row0 + rloc) * p.ldc + ti.b_col0 + ch * CW;
-                        const int ncols = ti.b_rows - ch * CW;
-#pragma unroll
-                        for (int i = 0; i < CW; ++i)
-                            if (i < ncols) crow[i] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
+                    for (int j = 0; j < 4; ++j) {
+                        uint4 w;
+                        w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * alpha, __uint_as_float(v[8 * j + 1]) * alpha);
+                        w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * alpha, __uint_as_float(v[8 * j + 3]) * alpha);
+                        w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * alpha, __uint_as_float(v[8 * j + 5]) * alpha);
+                        w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * alpha, __uint_as_float(v[8 * j + 7]) * alpha);
+                        // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
+                        st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
                     }
-                } else {
-                    if (a_ok) {
-                        const int n = ti.a_row0 + rloc;
-#pragma unroll
-                        for (int i = 0; i < CW; ++i) {
-                            const int m = ti.b_col0 + ch * CW + i;
-                            if (ch * CW + i < ti.b_rows)
-                                p.c[(int64_t)m * p.ldc + n] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
-                        }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmC, box, ti.b_col0 + ch * CW, ti.a_row0 + q * 32);
+                        bulk_commit_group();
                     }
+                } else if (a_ok) {
+                    __nv_bfloat16* crow = p.c + (int64_t)(ti.a_row0 + rloc) * p.ldc + ti.b_col0 + ch * CW;
+                    const int ncols = ti.b_rows - ch * CW;
+#pragma unroll
+                    for (int i = 0; i < CW; ++i)
+                        if (i < ncols) crow[i] = __float2bfloat16_rn(__uint_as_float(v[i]) * alpha);
                 }
             }
             tc_fence_before();
@@ -502,7 +493,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //
 // A cluster of two CTAs on two SMs computes a 256 x BN output tile: CTA r loads
 // A rows [128r, 128r + 128) and B rows [r * BN/2, (r + 1) * BN/2) of the tile
-// (so per SM the operand traffic per MMA is a third lower than the single-CTA
+// (so per SM the operand traffic per MMA is lower than for a single-CTA
 // 128 x BN tile), the leader (rank 0) issues tcgen05.mma.cta_group::2, and
 // each CTA ends up with its 128 rows x BN columns of FP32 accumulator in its
 // own tensor memory.  Both CTAs' operand loads complete on the leader's "full"
@@ -510,9 +501,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // stages, at the same tensor-memory address as its peer, the scale factors of
 // its own 128 A rows and of all BN columns of B (the B codes are split over
 // the pair, but each SM's MMA datapath reads every column's B scales from its
-// own tensor memory).  Tensor memory per CTA: two 192-column accumulators and
-// two scale buffers of 40 columns (16 for A, 6 per k-step for B) at a
-// 64-column stride.
+// own tensor memory).  Warps: 0 producer, 1 MMA (leader), 2-9 epilogue (two
+// per tensor-memory lane quarter), 10-13 scale staging.  Tensor memory per CTA
+// (256 x 256 tiles): one 256-column accumulator and four packed scale buffers
+// of 48 columns (16 for A, 8 per k-step for B).
 template <int BN_, int STAGES_, int NSB_, int ACC_>
 struct PairCfg {
     static constexpr int BN = BN_;                    // pair tile width
@@ -869,10 +861,10 @@ bool make_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <class C, bool SWAP, bool GROUPED>
+template <class C, bool GROUPED>
 nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                       int grid, cudaStream_t s) {
-    auto kern = gemm_kernel<C, SWAP, GROUPED>;
+    auto kern = gemm_kernel<C, GROUPED>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -940,13 +932,18 @@ nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const C
     return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairUse>, ta, tb, tc, args));
 }
 
-// Kernel configurations: prefill / grouped use 128 x 192 tiles with two
-// accumulator buffers (2 x 192 + 2 x 48 scale columns of tensor memory);
-// decode uses the swapped form with a narrow token side.
+// Kernel configurations: 64 < m <= 128 and the grouped form use 128 x 192
+// tiles with two accumulator buffers (2 x 192 + 2 x 48 scale columns of
+// tensor memory).
 using CfgWide = Cfg<192, 4, 2>;
-using CfgDec16 = Cfg<16, 8, 2>;
-using CfgDec32 = Cfg<32, 8, 2>;
-using CfgDec64 = Cfg<64, 7, 2>;
+// Decode (m <= 64): the tokens stay on the 128-row MMA side (the MMA work is
+// free in this weight-bound regime) but only 64 rows of them are loaded per
+// stage -- the MMA's rows 64..127 read the stage's other bytes and those
+// accumulator rows are never stored -- which leaves room for a fifth stage of
+// weights in flight.  Weights take the 192-wide side: 134 tiles for n = 25600,
+// one wave on 148 SMs (measured: 21-23 us for m = 1..64 against 29-36 us with
+// the weights on the 128-row side in 200 tiles).
+using CfgDecW = Cfg<192, 5, 2, 2, 64>;
 
 // BF16 [rows, cols] output with row stride ldc elements, 32 x 32 boxes,
 // 64-byte swizzle (matches the epilogue's staging layout).
@@ -1002,24 +999,20 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     if (!p.err) return NVFP4_ERR_CUDA;
     CUtensorMap ta, tb, tc;
     if (m <= 64) {
-        // decode: weights on the 128-row side, tokens on the narrow side
-        const int bn = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
-        if (!make_codes_map(&ta, b_codes, n, k / 2, 128) || !make_codes_map(&tb, a_codes, m, k / 2, bn))
+        if (!make_codes_map(&ta, a_codes, m, k / 2, CfgDecW::AROWS) ||
+            !make_codes_map(&tb, b_codes, n, k / 2, CfgDecW::BN) || !make_out_map(&tc, c, m, n, ldc))
             return NVFP4_ERR_CUDA;
-        p.sfa = b_scales;
-        p.sfb = a_scales;
-        p.sfb_rb_per_group = (int)((m + 127) / 128);
-        p.ga = b_global;
-        p.gb = a_global;
-        p.rows_a = (int)n;
-        p.rows_b = (int)m;
-        p.tiles_m = (int)((n + 127) / 128);
-        p.tiles_n = 1;
-        const int grid = (int)std::min<int64_t>(p.tiles_m, sms);
-        tc = tb;   // unused by the swapped form
-        if (bn == 16) return launch<CfgDec16, true, false>(ta, tb, tc, p, grid, s);
-        if (bn == 32) return launch<CfgDec32, true, false>(ta, tb, tc, p, grid, s);
-        return launch<CfgDec64, true, false>(ta, tb, tc, p, grid, s);
+        p.sfa = a_scales;
+        p.sfb = b_scales;
+        p.sfb_rb_per_group = (int)((n + 127) / 128);
+        p.ga = a_global;
+        p.gb = b_global;
+        p.rows_a = (int)m;
+        p.rows_b = (int)n;
+        p.tiles_m = 1;
+        p.tiles_n = (int)((n + CfgDecW::BN - 1) / CfgDecW::BN);
+        const int grid = (int)std::min<int64_t>((int64_t)p.tiles_n, sms);
+        return launch<CfgDecW, false>(ta, tb, tc, p, grid, s);
     }
     if (m > 128) {
         // prefill-class: 2-SM pair tiles of 256 x 224
@@ -1059,7 +1052,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int grid = (int)std::min<int64_t>(tiles, sms);
-    return launch<CfgWide, false, false>(ta, tb, tc, p, grid, s);
+    return launch<CfgWide, false>(ta, tb, tc, p, grid, s);
 }
 
 extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
@@ -1112,5 +1105,5 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     // upper bound of the tile count: sum_e ceil(n_e / 128) <= total_rows / 128 + num_experts
     const int64_t max_tiles = (total_rows / 128 + num_experts) * (int64_t)p.tiles_n;
     const int grid = (int)std::min<int64_t>(max_tiles, sms);
-    return launch<CfgWide, false, true>(ta, tb, tc, p, grid, s);
+    return launch<CfgWide, true>(ta, tb, tc, p, grid, s);
 }
