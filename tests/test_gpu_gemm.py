@@ -59,6 +59,8 @@ def test_tiny_workload_end_to_end():
     (129, 264, 128),     # 2-SM pair tile with one valid row in its second half
     (520, 776, 512),     # pair tiles: ragged m (3 row tiles) and n (4th column tile 8 wide)
     (1000, 2072, 576),   # many pair tiles, both edges ragged, partial last k-tile
+    (2304, 2336, 256),   # more pair tiles than resident pairs: a partial second wave
+    (2560, 4000, 128),   # ditto, with the last wave at the ragged n edge
 ])
 def test_gemm_matches_oracle(m, n, k):
     (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 0)
