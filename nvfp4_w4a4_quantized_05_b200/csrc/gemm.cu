@@ -525,7 +525,7 @@ struct PairCfg {
     static constexpr uint32_t EPI_BYTES = EPI_WARPS * 2 * 2048;
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
     static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols, "tensor memory budget");
-    static_assert(BN % 64 == 0, "each epilogue warp of a quarter drains BN / 2 columns");
+    static_assert(BN % 128 == 0, "each epilogue warp of a quarter drains BN / 2 columns, 64 at a time");
     static_assert(SF_BASE % 8 == 0 && SF_STRIDE % 8 == 0, "8-column stores start at a multiple of 8");
     static_assert(BN % 64 == 0 && (BN <= 192 || BN == 256),
                   "a B tile starts at row 0 or 64 of a scale block and spans <= 2 blocks");
@@ -765,10 +765,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // ---------------- epilogue (both CTAs; warps 2..9) ----------------
         // Two warps per tensor-memory lane quarter, each draining half of the
         // tile's columns; a warp releases the accumulator right after its last
-        // tensor-memory reads, before converting and storing those chunks, so
-        // the next tile's MMAs wait only for the reads (measured on the prefill
-        // shape: 4 warps 143 us, 8 warps 139 us, 8 warps reading 64 columns at
-        // a time 135 us; 16 warps were slower).
+        // tensor-memory reads, before staging and storing, so the next tile's
+        // MMAs wait only for the reads (measured on the prefill shape: 4 warps
+        // 143 us, 8 warps 139 us, 8 warps reading 64 columns at a time 135 us,
+        // converting all of them before the stores 133 us; 16 warps were slower).
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
         const int c0 = half * (BN / 64), c1 = c0 + BN / 64;
@@ -793,33 +793,40 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const int b_cols = min(BN, p.rows_b - n0);
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
             const float alpha = __fmul_rn(p.ga[0], p.gb[0]);
-            // two 32-column reads at a time; release after the last pair
-#pragma unroll 1
-            for (int cp = c0; cp < c1; cp += 2) {
+            // Read the warp's BN / 2 columns 64 at a time and convert them to
+            // BF16 in registers; release the accumulator after the last read,
+            // then stage and store.
+            uint32_t bf[BN / 4];
+#pragma unroll
+            for (int cp = 0; cp < BN / 128; ++cp) {
                 uint32_t va0[32], va1[32];
-                tmem_ld_32x32b_x32(tq + cp * 32, va0);
-                tmem_ld_32x32b_x32(tq + cp * 32 + 32, va1);
+                tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
+                tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
                 tmem_ld_wait();
-                if (cp + 2 == c1) {
+                if (cp == BN / 128 - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
                 }
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int ch = cp + h;
-                const uint32_t* v = h ? va1 : va0;
+                for (int i = 0; i < 16; ++i) {
+                    bf[cp * 32 + i] = pack_bf16x2(__uint_as_float(va0[2 * i]) * alpha,
+                                                  __uint_as_float(va0[2 * i + 1]) * alpha);
+                    bf[cp * 32 + 16 + i] = pack_bf16x2(__uint_as_float(va1[2 * i]) * alpha,
+                                                       __uint_as_float(va1[2 * i + 1]) * alpha);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < BN / 64; ++h) {
+                const int ch = c0 + h;
                 if (ch * 32 >= b_cols || q * 32 >= a_rows) continue;   // uniform per warp
                 const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
-                    uint4 w;
-                    w.x = pack_bf16x2(__uint_as_float(v[8 * j + 0]) * alpha, __uint_as_float(v[8 * j + 1]) * alpha);
-                    w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * alpha, __uint_as_float(v[8 * j + 3]) * alpha);
-                    w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * alpha, __uint_as_float(v[8 * j + 5]) * alpha);
-                    w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * alpha, __uint_as_float(v[8 * j + 7]) * alpha);
+                    const uint4 w = make_uint4(bf[h * 16 + 4 * j], bf[h * 16 + 4 * j + 1], bf[h * 16 + 4 * j + 2],
+                                               bf[h * 16 + 4 * j + 3]);
                     st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
                 }
                 fence_proxy_async_smem();
@@ -828,7 +835,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     tma_store_2d(&tmC, box, n0 + ch * 32, a_row0 + q * 32);
                     bulk_commit_group();
                 }
-            }
             }
         }
         if (lane == 0) bulk_wait_group_all();
