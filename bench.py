@@ -238,9 +238,17 @@ class Quant:
         self.qbytes = quant_bytes(self.rows, self.k)
         self.flops = 0.0
         self.launches_per_step = 1                    # one cooperative launch
+        # the weight variant (16 x 16 blocks), reported beside the step
+        self.wn = 14336
+        self.w = torch.from_numpy(W.quant_weight(0, self.wn, self.k).view(np.int16)).to(dev).view(torch.bfloat16)
+        self.qw = nv.quantize_weight_2d(self.w)
+        self.wqbytes = quant_bytes(self.wn, self.k)
 
     def quantize(self):
         self.nv.quantize_act(self.a, out=self.qa)
+
+    def quantize_weight(self):
+        self.nv.quantize_weight_2d(self.w, out=self.qw)
 
     step = quantize
 
@@ -527,6 +535,12 @@ def run_ours(args):
                             "peak_note": f"{peaks['source']} HBM copy bandwidth", "avg_launch_ms": q_avg * 1e3}
     line["quantize"] = {"gbs": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"], "avg_ms": q_avg * 1e3,
                         "algorithmic_bytes": wl.qbytes}
+    if hasattr(wl, "quantize_weight"):
+        w_avg = statistics.mean(timed_loop(torch, wl.quantize_weight, kiters, flush))
+        w_gbs = wl.wqbytes / w_avg / 1e9
+        line["weight_quantize"] = {"workload": f"bf16 [{wl.wn},{wl.k}] N(0,0.02) -> nvfp4, 16x16 blocks",
+                                   "gbs": w_gbs, "frac_hbm": w_gbs / peaks["hbm_gbs"], "avg_ms": w_avg * 1e3,
+                                   "algorithmic_bytes": wl.wqbytes, "kernels": "amax_kernel + quant2d_kernel"}
     if isinstance(wl, Decode):
         line["weight_stream"] = {"gbs": wl.wbytes / g_avg / 1e9, "frac_hbm": wl.wbytes / g_avg / 1e9 / peaks["hbm_gbs"],
                                  "bytes": wl.wbytes}

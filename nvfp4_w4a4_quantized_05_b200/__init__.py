@@ -247,23 +247,29 @@ def quantize_act(x, offsets=None, out: Optional[NVFP4Tensor] = None) -> NVFP4Ten
     return NVFP4Tensor(codes, scales, g, rows, k, offsets)
 
 
-def quantize_weight_2d(w, compact: bool = False):
+def quantize_weight_2d(w, compact: bool = False, out: Optional[NVFP4Tensor] = None):
     """16x16-block NVFP4 quantization of a BF16 [n, k] CUDA tensor.  Returns
-    the NVFP4Tensor (and the [n/16, k/16] compact scales when asked)."""
+    the NVFP4Tensor (and the [n/16, k/16] compact scales when asked); `out`
+    reuses the buffers of an earlier result of the same shape."""
     import torch
     if w.dtype != torch.bfloat16 or w.dim() != 2 or not w.is_cuda:
         raise TypeError("w must be a 2-D bfloat16 CUDA tensor")
     n, k = w.shape
     dev = w.device
-    codes = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty(nvfp4_scale_bytes(n, k), dtype=torch.uint8, device=dev)
+    if out is not None:
+        if out.rows != n or out.k != k or out.scales.numel() < nvfp4_scale_bytes(n, k) or out.offsets is not None:
+            raise ValueError("out does not match the input shape")
+        codes, scales, g = out.codes, out.scales, out.global_scale
+    else:
+        codes = torch.empty((n, k // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty(nvfp4_scale_bytes(n, k), dtype=torch.uint8, device=dev)
+        g = torch.empty(1, dtype=torch.float32, device=dev)
     sfc = torch.empty((n // 16, k // 16), dtype=torch.uint8, device=dev) if compact else None
-    g = torch.empty(1, dtype=torch.float32, device=dev)
     ws = _workspace(torch, dev, OP_QUANTIZE_WEIGHT_2D)
     st = nvfp4_quantize_weight_2d(_ptr(w), n, k, w.stride(0), _ptr(codes), _ptr(scales), _ptr(sfc), _ptr(g),
                                   _ptr(ws), _stream_ptr(torch, dev))
     _check(st, "nvfp4_quantize_weight_2d")
-    t = NVFP4Tensor(codes, scales, g, n, k)
+    t = out if out is not None else NVFP4Tensor(codes, scales, g, n, k)
     return (t, sfc) if compact else t
 
 

@@ -240,3 +240,28 @@ def test_quantize_weight_2d_full_weight_workload():
     assert t.global_scale.cpu().numpy()[0] == np.float32(og)
     assert np.array_equal(t.codes.cpu().numpy(), oc)
     assert np.array_equal(t.scales.cpu().numpy(), osf)
+
+
+def test_out_buffers_reused_across_inputs():
+    """`out=` writes a second input's result over the first one's buffers
+    (activations and 2D weights): the result is the oracle's for the second
+    input, with nothing left from the first."""
+    import torch
+    x1 = W.gaussian_bf16((200, 1024), 0, 301, 1.0)
+    x2 = W.laplace_outliers_bf16((200, 1024), 0, 302)
+    qa = nv.quantize_act(bf16_to_device(x1))
+    nv.quantize_act(bf16_to_device(x2), out=qa)
+    torch.cuda.synchronize()
+    oc, osf, og = O.quantize_1d(x2)
+    assert np.array_equal(qa.codes.cpu().numpy(), oc) and np.array_equal(qa.scales.cpu().numpy(), osf)
+    assert qa.global_scale.cpu().numpy()[0] == np.float32(og)
+    w1 = W.gaussian_bf16((96, 512), 0, 303, 0.02)
+    w2 = W.gaussian_bf16((96, 512), 0, 304, 3.0)
+    qw = nv.quantize_weight_2d(bf16_to_device(w1))
+    nv.quantize_weight_2d(bf16_to_device(w2), out=qw)
+    torch.cuda.synchronize()
+    oc, osf, og = O.quantize_2d(w2)
+    assert np.array_equal(qw.codes.cpu().numpy(), oc) and np.array_equal(qw.scales.cpu().numpy(), osf)
+    assert qw.global_scale.cpu().numpy()[0] == np.float32(og)
+    with pytest.raises(ValueError):
+        nv.quantize_weight_2d(bf16_to_device(W.gaussian_bf16((80, 512), 0, 305, 0.02)), out=qw)
