@@ -12,12 +12,12 @@ once, outside the timed region), C bf16 [4096, 14336].
                     [--workload prefill|quant|decode|moe] [--decode-m M]
 
 Prints one JSON line.  `value` is whole-job throughput (TFLOP/s of 2*M*N*K
-per step, summed over ranks, divided by the slowest rank's time).  L2 is
-flushed (a 256 MiB write) before every timed step and outside its events.
-Timing: CUDA events on the launching stream around each step; per-kernel
-durations come from separate event-timed loops of the GEMM and of the
-quantizer alone on the same inputs.  N > 1 runs N independent replicas (the
-path needs no exchange between GPUs), one process per GPU.
+per step, summed over ranks, divided by the slowest rank's time).  The steps
+rotate over enough independent buffer sets that no step finds its inputs in
+L2.  Timing: the K steps run as CUDA-graph replays on one stream between one
+pair of CUDA events; per-kernel durations come from a copy of the same graph
+with an event between consecutive kernels.  N > 1 runs N independent
+replicas (the path needs no exchange between GPUs), one process per GPU.
 
 --impl reference times the CPU oracle (plain C, binary64 GEMM) on a bounded
 sample of the same workload: rank 0 only.
@@ -37,7 +37,6 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-L2_FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 FP4_PER_BF16 = 4.0            # dense FP4 / dense BF16 nominal ratio (9 / 2.25 PFLOP/s)
@@ -163,6 +162,40 @@ def barrier(world: int):
 
 
 # ---- workloads ----------------------------------------------------------------------------
+#
+# Each workload holds R independent buffer sets (activations, their NVFP4
+# form, weights, output) and step i works on set i % R.  R is chosen so that
+# between two uses of one set the other sets move at least twice the L2 size:
+# every step finds its inputs in HBM, none left in L2 by an earlier step.
+
+L2_BYTES = 128 << 20          # upper bound of the 126 MB L2
+
+
+MAX_SETS = 16
+# Idle time before each timed loop, so that every loop starts from the same
+# power state: under a dense FP4 GEMM the board reaches its power cap after
+# about 0.1 s and the SM clock steps down from 1965 MHz to about 1800 MHz.
+REST_S = 0.5
+
+
+def rotation_count(*set_bytes: int) -> int:
+    """Sets needed so that, for each of the given per-set footprints (a whole
+    step, or one kernel timed alone), the other sets move twice the L2 size;
+    at most MAX_SETS (only a tiny decode activation would want more)."""
+    return min(MAX_SETS, max(max(2, 1 + -(-2 * L2_BYTES // max(1, b))) for b in set_bytes))
+
+
+def nbytes(*ts) -> int:
+    return sum(t.numel() * t.element_size() for t in ts)
+
+
+def to_device(torch, bits, dev):
+    return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def clone_q(nv, t):
+    return nv.NVFP4Tensor(t.codes.clone(), t.scales.clone(), t.global_scale.clone(), t.rows, t.k, t.offsets)
+
 
 class Prefill:
     name = "prefill"
@@ -170,28 +203,53 @@ class Prefill:
     def __init__(self, nv, torch, dev, m=4096, n=14336, k=4096):
         import workloads as W
         self.m, self.n, self.k = m, n, k
-        a, w = W.prefill(0, m, n, k)
-        self.a_host = a
-        self.a = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-        wdev = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16)
-        self.w = nv.quantize_weight_2d(wdev)          # offline: pre-quantized weights
-        del wdev
-        self.c = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        self._build(nv, torch, dev, *W.prefill(0, m, n, k))
+
+    def _build(self, nv, torch, dev, a, w):
+        m, n, k = self.m, self.n, self.k
         self.nv = nv
+        self.a_host = a
+        a0 = to_device(torch, a, dev)
+        wdev = to_device(torch, w, dev)
+        w0 = nv.quantize_weight_2d(wdev)              # offline: pre-quantized weights
+        del wdev
+        q0 = nv.quantize_act(a0)
+        c0 = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        self.set_bytes = nbytes(a0, q0.codes, q0.scales, w0.codes, w0.scales, c0)
+        self.kernel_bytes = (nbytes(a0, q0.codes, q0.scales), nbytes(q0.codes, q0.scales, w0.codes, w0.scales, c0))
+        self.R = R = rotation_count(self.set_bytes, *self.kernel_bytes)
+        self.a = [a0] + [a0.clone() for _ in range(R - 1)]
+        self.qa = [q0] + [clone_q(nv, q0) for _ in range(R - 1)]
+        self.w = [w0] + [clone_q(nv, w0) for _ in range(R - 1)]
+        self.c = [c0] + [torch.empty_like(c0) for _ in range(R - 1)]
         self.flops = 2.0 * m * n * k
-        self.qa = nv.quantize_act(self.a)
         self.qbytes = quant_bytes(m, k)
+        self.wbytes = nbytes(w0.codes, w0.scales)
         self.launches_per_step = 2                    # one-launch quantizer, GEMM
 
-    def quantize(self):
-        self.nv.quantize_act(self.a, out=self.qa)
+    def quantize(self, i):
+        j = i % self.R
+        self.nv.quantize_act(self.a[j], out=self.qa[j])
 
-    def gemm(self):
-        self.nv.gemm(self.qa, self.w, out=self.c)
+    def gemm(self, i):
+        j = i % self.R
+        self.nv.gemm(self.qa[j], self.w[j], out=self.c[j])
 
-    def step(self):
-        self.quantize()
-        self.gemm()
+    kernels = (quantize, gemm)
+
+    def step(self, i):
+        self.quantize(i)
+        self.gemm(i)
+
+    def result(self, i):
+        return self.c[i % self.R]
+
+    def gemm_label(self):
+        if self.m <= 64:
+            return "gemm_kernel (tcgen05 mxf4nvf4; 64 token rows x 192 weight rows per tile)"
+        if self.m > 128:
+            return "gemm_pair_kernel (tcgen05 mxf4nvf4, cta_group::2; 256 x 256 tiles)"
+        return "gemm_kernel (tcgen05 mxf4nvf4; 128 x 192 tiles)"
 
     def config(self):
         return {"workload": f"prefill W4A4: A bf16 [{self.m},{self.k}] dynamically quantized (1D blocks) x "
@@ -205,19 +263,7 @@ class Decode(Prefill):
     def __init__(self, nv, torch, dev, m=64):
         import workloads as W
         self.m, self.n, self.k = m, 25600, 5120
-        a, w = W.decode(m)
-        self.a_host = a
-        self.a = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
-        wdev = torch.from_numpy(w.view(np.int16)).to(dev).view(torch.bfloat16)
-        self.w = nv.quantize_weight_2d(wdev)
-        del wdev
-        self.c = torch.empty((m, self.n), dtype=torch.bfloat16, device=dev)
-        self.nv = nv
-        self.flops = 2.0 * m * self.n * self.k
-        self.qa = nv.quantize_act(self.a)
-        self.qbytes = quant_bytes(m, self.k)
-        self.wbytes = self.n * self.k // 2 + nv.nvfp4_scale_bytes(self.n, self.k)
-        self.launches_per_step = 2
+        self._build(nv, torch, dev, *W.decode(m))
 
     def config(self):
         return {"workload": f"decode W4A4: A bf16 [{self.m},{self.k}] quantized per call x W nvfp4 "
@@ -229,28 +275,42 @@ class Quant:
 
     def __init__(self, nv, torch, dev):
         import workloads as W
+        self.nv = nv
         self.rows, self.k = 8192, 4096
         x = W.quant_act(0)
         self.a_host = x
-        self.a = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
-        self.nv = nv
-        self.qa = nv.quantize_act(self.a)
+        a0 = to_device(torch, x, dev)
+        q0 = nv.quantize_act(a0)
+        self.set_bytes = nbytes(a0, q0.codes, q0.scales)
+        self.kernel_bytes = (self.set_bytes,)
+        self.R = R = rotation_count(self.set_bytes)
+        self.a = [a0] + [a0.clone() for _ in range(R - 1)]
+        self.qa = [q0] + [clone_q(nv, q0) for _ in range(R - 1)]
         self.qbytes = quant_bytes(self.rows, self.k)
         self.flops = 0.0
         self.launches_per_step = 1                    # one cooperative launch
         # the weight variant (16 x 16 blocks), reported beside the step
         self.wn = 14336
-        self.w = torch.from_numpy(W.quant_weight(0, self.wn, self.k).view(np.int16)).to(dev).view(torch.bfloat16)
-        self.qw = nv.quantize_weight_2d(self.w)
+        w0 = to_device(torch, W.quant_weight(0, self.wn, self.k), dev)
+        qw0 = nv.quantize_weight_2d(w0)
+        self.RW = RW = rotation_count(nbytes(w0, qw0.codes, qw0.scales))
+        self.w = [w0] + [w0.clone() for _ in range(RW - 1)]
+        self.qw = [qw0] + [clone_q(nv, qw0) for _ in range(RW - 1)]
         self.wqbytes = quant_bytes(self.wn, self.k)
 
-    def quantize(self):
-        self.nv.quantize_act(self.a, out=self.qa)
+    def quantize(self, i):
+        j = i % self.R
+        self.nv.quantize_act(self.a[j], out=self.qa[j])
 
-    def quantize_weight(self):
-        self.nv.quantize_weight_2d(self.w, out=self.qw)
-
+    kernels = (quantize,)
     step = quantize
+
+    def quantize_weight(self, i):
+        j = i % self.RW
+        self.nv.quantize_weight_2d(self.w[j], out=self.qw[j])
+
+    def result(self, i):
+        return self.qa[i % self.R].codes
 
     def config(self):
         return {"workload": "activation quantizer: bf16 [8192,4096] Laplace(0,1) + 0.1% +-U[50,200] -> nvfp4 "
@@ -262,35 +322,51 @@ class Moe:
 
     def __init__(self, nv, torch, dev):
         import workloads as W
+        self.nv = nv
         a, off, w = W.moe(0)
         E, N, K = w.shape
         self.E, self.n, self.k, self.rows = E, N, K, a.shape[0]
         self.a_host = a
-        self.a = torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        a0 = to_device(torch, a, dev)
         self.off = torch.from_numpy(off).to(dev)
-        wdev = torch.from_numpy(w.reshape(E * N, K).view(np.int16)).to(dev).view(torch.bfloat16)
+        wdev = to_device(torch, w.reshape(E * N, K), dev)
         tw = [nv.quantize_weight_2d(wdev[e * N:(e + 1) * N]) for e in range(E)]
         del wdev
-        self.b_codes = torch.stack([t.codes for t in tw])
-        self.b_scales = torch.cat([t.scales for t in tw])
-        self.b_global = torch.cat([t.global_scale for t in tw])
+        b0 = (torch.stack([t.codes for t in tw]), torch.cat([t.scales for t in tw]),
+              torch.cat([t.global_scale for t in tw]))
         del tw
-        self.c = torch.empty((self.rows, N), dtype=torch.bfloat16, device=dev)
-        self.nv = nv
+        q0 = nv.quantize_act(a0, self.off)
+        c0 = torch.empty((self.rows, N), dtype=torch.bfloat16, device=dev)
+        self.set_bytes = nbytes(a0, q0.codes, q0.scales, b0[0], b0[1], c0)
+        self.kernel_bytes = (nbytes(a0, q0.codes, q0.scales), nbytes(q0.codes, q0.scales, b0[0], b0[1], c0))
+        self.R = R = rotation_count(self.set_bytes, *self.kernel_bytes)
+        self.a = [a0] + [a0.clone() for _ in range(R - 1)]
+        self.qa = [q0] + [clone_q(nv, q0) for _ in range(R - 1)]
+        self.b = [b0] + [tuple(t.clone() for t in b0) for _ in range(R - 1)]
+        self.c = [c0] + [torch.empty_like(c0) for _ in range(R - 1)]
         self.flops = 2.0 * self.rows * N * K
-        self.qa = nv.quantize_act(self.a, self.off)
         self.qbytes = quant_bytes(self.rows, K, E)
         self.launches_per_step = 3                    # per-group amax, quantize, grouped GEMM
 
-    def quantize(self):
-        self.nv.quantize_act(self.a, self.off, out=self.qa)
+    def quantize(self, i):
+        j = i % self.R
+        self.nv.quantize_act(self.a[j], self.off, out=self.qa[j])
 
-    def gemm(self):
-        self.nv.grouped_gemm(self.qa, self.b_codes, self.b_scales, self.b_global, self.n, out=self.c)
+    def gemm(self, i):
+        j = i % self.R
+        self.nv.grouped_gemm(self.qa[j], *self.b[j], self.n, out=self.c[j])
 
-    def step(self):
-        self.quantize()
-        self.gemm()
+    kernels = (quantize, gemm)
+
+    def step(self, i):
+        self.quantize(i)
+        self.gemm(i)
+
+    def result(self, i):
+        return self.c[i % self.R]
+
+    def gemm_label(self):
+        return "gemm_kernel<grouped> (tcgen05 mxf4nvf4; 128 x 192 tiles per expert group)"
 
     def config(self):
         return {"workload": f"MoE grouped W4A4: {self.rows // 8} tokens top-8 of {self.E} experts, A bf16 "
@@ -300,18 +376,73 @@ class Moe:
 
 
 # ---- timing helpers -------------------------------------------------------------------------
+#
+# The timed work runs as CUDA graphs captured on one side stream: a graph of
+# R consecutive steps (one per buffer set) replayed, plus a graph of the
+# remaining K mod R steps, so exactly K steps run between one pair of events.
 
-def timed_loop(torch, fn, iters, flush):
-    """Per-iteration CUDA-event times (seconds) of fn, L2 flushed before each."""
-    s = torch.cuda.current_stream()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
-    for i in range(iters):
-        flush(i)
-        evs[i][0].record(s)
-        fn()
-        evs[i][1].record(s)
-    torch.cuda.synchronize()
-    return [a.elapsed_time(b) * 1e-3 for a, b in evs]
+def capture(torch, stream, calls):
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for f in calls:
+            f()
+    return g
+
+
+class StepGraphs:
+    """Exactly `n` calls fn(0), fn(1), ... (fn(i) works on buffer set i % R)
+    as replays of captured graphs on `stream`."""
+
+    def __init__(self, torch, stream, fn, R, n):
+        self.torch, self.stream, self.n = torch, stream, n
+        with torch.cuda.stream(stream):
+            for i in range(R):                        # first calls on this stream: workspaces, attributes
+                fn(i)
+        stream.synchronize()
+        self.full = capture(torch, stream, [lambda i=i: fn(i) for i in range(R)])
+        self.reps, rem = divmod(n, R)
+        self.part = capture(torch, stream, [lambda i=i: fn(i) for i in range(rem)]) if rem else None
+        self.R, self.rem = R, rem
+        self.setup_calls = R
+
+    def warm(self, at_least: int) -> int:
+        """Untimed replays (at least `at_least` calls, every graph once);
+        returns the calls run, the first eager ones included."""
+        done = self.setup_calls
+        with self.torch.cuda.stream(self.stream):
+            while True:
+                self.full.replay()
+                done += self.R
+                if done >= at_least:
+                    break
+            if self.part is not None:
+                self.part.replay()
+                done += self.rem
+        self.stream.synchronize()
+        return done
+
+    def run(self):
+        """The n calls between two events; returns (start, end) events."""
+        torch = self.torch
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(self.stream):
+            e0.record()
+            for _ in range(self.reps):
+                self.full.replay()
+            if self.part is not None:
+                self.part.replay()
+            e1.record()
+        return e0, e1
+
+
+def graph_seconds(torch, stream, fn, R, n):
+    """Average seconds per call of fn over n graph-replayed calls (after one
+    untimed pass over every graph)."""
+    g = StepGraphs(torch, stream, fn, R, n)
+    g.warm(0)
+    e0, e1 = g.run()
+    stream.synchronize()
+    return e0.elapsed_time(e1) * 1e-3 / n
 
 
 def cpu_baseline_prefill(wl, max_seconds=12.0):
@@ -437,69 +568,72 @@ def run_ours(args):
     peaks = load_peaks()
     wl = {"prefill": Prefill, "decode": Decode, "quant": Quant, "moe": Moe}[args.workload]
     wl = wl(nv, torch, dev, m=args.decode_m) if args.workload == "decode" else wl(nv, torch, dev)
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    cs = torch.cuda.Stream(dev)
+    sampler = ClockSampler(local)
+    sampler.start()
 
-    def flush(i):
-        # Write 256 MiB (twice L2), then read it back: the writes' dirty lines
-        # are written back during the flush, not during the next timed step.
-        flush_buf.fill_(i & 0xFF)
-        flush_buf.view(torch.float32).sum()       # one read, no widening copy
-
-    # warm-up
-    for i in range(max(3, args.warmup)):
-        flush(i)
-        wl.step()
-    torch.cuda.synchronize()
+    # capture, then warm-up (eager first calls + one replay of every graph)
+    steps = StepGraphs(torch, cs, wl.step, wl.R, args.steps)
+    warm = steps.warm(max(3, args.warmup))
     nv.check_device_error()
 
     # ---- timed region: exactly K steps ----
-    sampler = ClockSampler(local)
-    sampler.start()
+    time.sleep(REST_S)
     barrier(world)
     torch.cuda.synchronize()
     t0 = time.perf_counter()
-    step_times = timed_loop(torch, wl.step, args.steps, flush)
+    e0, e1 = steps.run()
     torch.cuda.synchronize()
     barrier(world)
     t1 = time.perf_counter()
-    sampler.stop()
     nv.check_device_error()
-    total = reduce_max(sum(step_times), world, dev)
+    total = reduce_max(e0.elapsed_time(e1) * 1e-3, world, dev)
     clocks = sampler.summary(t0, t1)
+    del steps
 
-    # ---- per-kernel times on the same inputs (separate event-timed loops) ----
+    # ---- per-kernel times: each kernel alone, back to back over the same buffer sets ----
     kiters = max(10, min(args.steps, 200))
-    q_times = timed_loop(torch, wl.quantize, kiters, flush)
-    q_avg = statistics.mean(q_times)
-    g_avg = None
-    if hasattr(wl, "gemm"):
-        g_times = timed_loop(torch, wl.gemm, kiters, flush)
-        g_avg = statistics.mean(g_times)
+    ktimes, kclocks = [], []
+    for f in wl.kernels:
+        time.sleep(REST_S)
+        ta = time.perf_counter()
+        ktimes.append(graph_seconds(torch, cs, lambda i, f=f: f(wl, i), wl.R, kiters))
+        kclocks.append(sampler.summary(ta, time.perf_counter()))
+    q_avg = ktimes[0]
+    g_avg = ktimes[1] if len(ktimes) > 1 else None
     nv.check_device_error()
 
     # ---- end to end through the public API from pinned host memory ----
     e2e = None
     if not args.no_e2e:
         a_pinned = torch.from_numpy(wl.a_host.view(np.int16)).pin_memory()
-        out_dev = wl.c if hasattr(wl, "c") else wl.qa.codes
-        out_pinned = torch.empty(out_dev.shape, dtype=out_dev.dtype).pin_memory()
+        out0 = wl.result(0)
+        out_pinned = torch.empty(out0.shape, dtype=out0.dtype).pin_memory()
 
-        def e2e_step():
-            wl.a.view(torch.int16).copy_(a_pinned, non_blocking=True)
-            wl.step()
-            src = wl.c if hasattr(wl, "c") else wl.qa.codes
-            out_pinned.copy_(src, non_blocking=True)
-        for i in range(2):
-            e2e_step()
-        e_times = timed_loop(torch, e2e_step, max(5, min(args.steps, 50)), flush)
-        e_avg = reduce_max(statistics.mean(e_times), world, dev)
+        def e2e_step(i):
+            wl.a[i % wl.R].view(torch.int16).copy_(a_pinned, non_blocking=True)
+            wl.step(i)
+            out_pinned.copy_(wl.result(i), non_blocking=True)
+        n_e2e = max(5, min(args.steps, 50))
+        with torch.cuda.stream(cs):
+            for i in range(2):
+                e2e_step(i)
+            cs.synchronize()
+            ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ea.record()
+            for i in range(n_e2e):
+                e2e_step(i)
+            eb.record()
+        cs.synchronize()
+        e_avg = reduce_max(ea.elapsed_time(eb) * 1e-3 / n_e2e, world, dev)
         h2d = a_pinned.numel() * a_pinned.element_size()
         d2h = out_pinned.numel() * out_pinned.element_size()
         if wl.flops:
             ev, eu = world * wl.flops / e_avg / 1e12, "TFLOP/s"
         else:
             ev, eu = world * wl.qbytes / e_avg / 1e9, "GB/s"
-        e2e = {"value": ev, "unit": eu, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+        e2e = {"value": ev, "unit": eu, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "path": "eager calls of the Python binding on one stream; pinned host buffers"}
 
     ms = total / args.steps * 1e3
     fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
@@ -511,32 +645,42 @@ def run_ours(args):
     else:
         value = world * wl.qbytes * args.steps / total / 1e9
         line.update({"value": value, "unit": "GB/s"})
-    line.update({"n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms,
+    line.update({"n_gpus": world, "steps": args.steps, "warmup": warm, "ms_per_step": ms,
                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                  "dtype": "fp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate)",
                  "data": "synthetic (seeded; see workloads/)"})
     cfg = wl.config()
-    cfg.update({"l2": "flushed before every timed step (256 MiB written, then read back; outside the step's events)",
+    l2 = (f"inputs larger than L2: steps rotate over {wl.R} buffer sets of {wl.set_bytes / 1e6:.1f} MB; "
+          f"between two uses of a set the others move {(wl.R - 1) * wl.set_bytes / 1e6:.0f} MB (L2 126 MB)")
+    small = min(wl.kernel_bytes)
+    if (wl.R - 1) * small < 2 * L2_BYTES:
+        l2 += (f"; the quantizer timed alone cycles through only {(wl.R - 1) * small / 1e6:.0f} MB, so its "
+               f"{small / 1e6:.2f} MB of activations may sit in L2, as a previous layer's output would")
+    cfg.update({"l2": l2,
+                "launch": f"CUDA graphs of {wl.R} steps replayed on one stream; per-kernel times from graphs "
+                          "of that kernel alone over the same buffer sets",
                 "parallelism": f"replicas x{world}" if world > 1 else "single GPU"})
     line["config"] = cfg
     if g_avg is not None:
         g_tflops = wl.flops / g_avg / 1e12
-        line["roofline"] = {"bound": "tensor", "kernel": "gemm_kernel (tcgen05 mxf4nvf4)",
+        line["roofline"] = {"bound": "tensor", "kernel": wl.gemm_label(),
                             "achieved": g_tflops, "peak": fp4_peak, "unit": "TFLOP/s",
                             "frac": g_tflops / fp4_peak, "traffic": load_traffic(f"gemm_{wl.name}"),
                             "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_PER_BF16} "
                                          "(dense FP4 / BF16 nominal ratio)",
-                            "avg_launch_ms": g_avg * 1e3}
+                            "avg_launch_ms": g_avg * 1e3, "launches_timed": kiters, "clocks": kclocks[1]}
     else:
         line["roofline"] = {"bound": "hbm", "kernel": "quant1d_fused_kernel (one cooperative launch)",
                             "achieved": q_gbs,
                             "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": q_gbs / peaks["hbm_gbs"],
                             "traffic": load_traffic(f"quant_{wl.name}"),
-                            "peak_note": f"{peaks['source']} HBM copy bandwidth", "avg_launch_ms": q_avg * 1e3}
+                            "peak_note": f"{peaks['source']} HBM copy bandwidth", "avg_launch_ms": q_avg * 1e3,
+                            "launches_timed": kiters, "clocks": kclocks[0]}
     line["quantize"] = {"gbs": q_gbs, "frac_hbm": q_gbs / peaks["hbm_gbs"], "avg_ms": q_avg * 1e3,
                         "algorithmic_bytes": wl.qbytes}
     if hasattr(wl, "quantize_weight"):
-        w_avg = statistics.mean(timed_loop(torch, wl.quantize_weight, kiters, flush))
+        time.sleep(REST_S)
+        w_avg = graph_seconds(torch, cs, wl.quantize_weight, wl.RW, kiters)
         w_gbs = wl.wqbytes / w_avg / 1e9
         line["weight_quantize"] = {"workload": f"bf16 [{wl.wn},{wl.k}] N(0,0.02) -> nvfp4, 16x16 blocks",
                                    "gbs": w_gbs, "frac_hbm": w_gbs / peaks["hbm_gbs"], "avg_ms": w_avg * 1e3,
@@ -547,6 +691,7 @@ def run_ours(args):
     line["e2e"] = e2e
     line["gpu_launches"] = wl.launches_per_step * args.steps
     line["clocks"] = clocks
+    sampler.stop()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = (cpu_baseline_quant(wl) if wl.name == "quant" else
                                 cpu_baseline_prefill(wl) if wl.name in ("prefill", "decode") else None)
@@ -561,7 +706,8 @@ def run_ours(args):
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default: enough for a >= 50 ms timed region on this workload)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["prefill", "quant", "decode", "moe"], default="prefill")
@@ -570,6 +716,11 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = (20 if args.impl == "reference" else
+                      {"prefill": 500, "quant": 2000, "decode": 2000, "moe": 300}[args.workload])
+    if args.steps < 1:
+        ap.error("--steps must be at least 1")
     if args.impl == "reference":
         return run_reference(args)
     return run_ours(args)
