@@ -46,8 +46,9 @@
  *     device.  It must be zero before its first use (nvfp4_workspace_init);
  *     after that, leave it untouched between calls: every call that returns
  *     NVFP4_OK leaves it ready for the next (the one-tensor quantizer keeps a
- *     per-CTA generation count in it).  Calls sharing one workspace must be
- *     ordered on one stream.
+ *     per-CTA generation count in it; the GEMM returns its hand-off counters
+ *     to zero).  Calls sharing one workspace must be ordered on one stream.
+ *     After NVFP4_ERR_TIMEOUT, zero it again.
  */
 #ifndef NVFP4_H
 #define NVFP4_H
@@ -184,12 +185,18 @@ nvfp4_status_t nvfp4_quantize_weight_2d(const void* w, int64_t n, int64_t k, int
  *   b_codes, b_scales, b_global: device; output of either quantizer on [n, k].
  *   c: device BF16 [m, n], row stride ldc elements (ldc >= n, ldc % 8 == 0).
  *   m >= 0, n > 0, k > 0, k % 64 == 0.
- *   workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, 0) bytes (may be
- *   NULL when that is 0).
- * For m <= 64 the kernel runs with the operands swapped (weights fill the
- * 128-row MMA side; tokens fill the narrow N side), as decode is bound by
- * streaming the weights ("W4A8 vs NVFP4 quantization on GPUs", "Batch size can
- * change the winner"). */
+ *   workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, 0) bytes, 16-byte
+ *   aligned, zeroed before first use (see above); NULL is allowed.  For m > 128
+ *   the kernel runs on pairs of SMs with 256 x 256 output tiles; when the tiles
+ *   do not fill whole waves of pairs, the k-range of the last tiles is shared
+ *   out between pairs (stream-K), and a pair hands its FP32 partial sums to the
+ *   pair that owns the tile through this workspace (about 19 MB on a B200).
+ *   With NULL, or when the size is 0, every tile is computed whole; the result
+ *   differs only in the FP32 summation order of those last tiles.
+ * For m <= 64 the 128-row MMA side loads only 64 token rows per stage and the
+ * weights take the 192-wide side, so that the whole weight matrix streams in
+ * one wave: decode is bound by reading the weights ("W4A8 vs NVFP4
+ * quantization on GPUs", "Batch size can change the winner"). */
 nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                           const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
                           void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,

@@ -212,6 +212,21 @@ def _workspace(torch, device, op: int, groups: int = 0):
     return ws
 
 
+def _gemm_workspace(torch, device, m: int, n: int, k: int):
+    """Scratch for the GEMM's stream-K tail (None when the shape needs none):
+    one zeroed buffer per device and stream, grown on demand; every call
+    leaves it zeroed for the next."""
+    nbytes = nvfp4_workspace_bytes(OP_GEMM, m, n, k, 0)
+    if nbytes == 0:
+        return None
+    key = (device.index, OP_GEMM, 0, torch.cuda.current_stream(device).cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
 def _ptr(t) -> int:
     return 0 if t is None else int(t.data_ptr())
 
@@ -280,8 +295,9 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out=None):
         raise ValueError("k mismatch")
     dev = a.codes.device
     c = out if out is not None else torch.empty((a.rows, b.rows), dtype=torch.bfloat16, device=dev)
+    ws = _gemm_workspace(torch, dev, a.rows, b.rows, a.k)
     st = nvfp4_gemm(_ptr(a.codes), _ptr(a.scales), _ptr(a.global_scale), _ptr(b.codes), _ptr(b.scales),
-                    _ptr(b.global_scale), _ptr(c), c.stride(0), a.rows, b.rows, a.k, None, _stream_ptr(torch, dev))
+                    _ptr(b.global_scale), _ptr(c), c.stride(0), a.rows, b.rows, a.k, _ptr(ws), _stream_ptr(torch, dev))
     _check(st, "nvfp4_gemm")
     return c
 

@@ -38,8 +38,10 @@
 //
 // Operand roles: the "A side" (activations) fills the 128-row MMA dimension,
 // the "B side" (weights) the BN-wide dimension.  For m > 128 the 2-SM pair
-// kernel below takes over (256-row tiles).  The grouped form walks (expert,
-// m-tile, n-tile) triples built from the device offsets array.
+// kernel below takes over (256 x 256 tiles, persistent over tiles, with a
+// stream-K share-out of the last waves' k-tiles so that all pairs finish
+// together).  The grouped form walks (expert, m-tile, n-tile) triples built
+// from the device offsets array.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
@@ -47,6 +49,7 @@
 
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -82,6 +85,12 @@ struct GemmArgs {
     int num_groups;
     uint64_t wait_limit_ns;
     unsigned int* err;
+    // pair kernel, stream-K tail (see PairWork): tiles [0, dp_tiles) are whole;
+    // the k-tiles of the rest are shared out evenly
+    int dp_tiles;
+    int64_t sk_units;
+    float* partial;            // per CTA of each pair: FP32 [BN / 4][128] x 4 partial sums
+    uint32_t* sk_flags;        // per CTA of each pair: a ready counter, kSkFlagStride words apart
 };
 
 struct alignas(8) SmemTail {
@@ -538,6 +547,71 @@ struct PairCfg {
 // accumulator the producer keeps filling the 5 stages.
 using PairUse = PairCfg<256, 5, 4, 1>;
 
+// ---- stream-K tail of the pair kernel ----------------------------------------------
+//
+// With T tiles on P resident pairs and T % P != 0, the last partial wave would
+// leave most pairs idle (prefill 4096 x 14336: 896 tiles on 74 pairs, so 8
+// pairs run a 13th tile while 66 wait).  Instead every pair first takes whole
+// tiles pair, pair + P, ... below dp_tiles = (T / P - 1) * P, then an equal
+// share of the k-tiles of the remaining T - dp_tiles tiles (between P and
+// 2P - 1 of them) in tile order.  A share holds at least one tile's k-tiles,
+// so a tile is split between at most two consecutive pairs: pair c computes
+// its first k-tiles [0, ke) last in its share (the "head", owner of the
+// output); pair c + 1 computes the rest [kb, num_kt) first in its own share
+// (the "continuation").  The continuation's epilogue stores its FP32
+// accumulator to a workspace slot and counts its 8 epilogue warps in a
+// per-CTA counter; once the head's MMAs are done, one thread of its epilogue
+// waits (bounded) for the count of 8, copies the slot into the now idle stage
+// buffers with bulk copies and returns the counter to zero for the next
+// launch; the epilogue adds the copy to its own accumulator before scaling
+// and storing as usual.
+constexpr int kSkFlagStride = 16;      // uint32 words: one 64-byte line per CTA
+constexpr uint32_t kSkWarps = 8;       // epilogue warps per CTA
+
+// Calls f(std::integral_constant<int, i>) for i = 0 .. N-1 (compile-time indices).
+template <int N, int I = 0, class F>
+__device__ __forceinline__ void static_for(F&& f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for<N, I + 1>(f);
+    }
+}
+
+struct PairWork {
+    int t = -1, kb = 0, ke = 0;        // current item: tile t, k-tiles [kb, ke)
+    int u = -1;                        // next stream-K unit (sk_units < 2^31, host), -1 in the whole-tile phase
+    __device__ bool next(const GemmArgs& p, int cluster) {
+        const int P = (int)(gridDim.x >> 1);
+        if (u < 0) {
+            t = t < 0 ? cluster : t + P;
+            if (t < p.dp_tiles) {
+                kb = 0;
+                ke = p.num_kt;
+                return true;
+            }
+            u = (int)(p.sk_units * cluster / P);
+        }
+        const int u1 = (int)(p.sk_units * (cluster + 1) / P);
+        if (u >= u1) return false;
+        const int j = u / p.num_kt;
+        t = p.dp_tiles + j;
+        kb = u - j * p.num_kt;
+        ke = min(p.num_kt, kb + (u1 - u));
+        u += ke - kb;
+        return true;
+    }
+};
+
+// Bounded wait until all epilogue warps of the continuation have counted in.
+__device__ __forceinline__ bool sk_wait_ready(const uint32_t* ready, uint64_t limit_ns, volatile int* abort_flag) {
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu_u32(ready) < kSkWarps) {
+        if (*abort_flag || globaltimer_ns() - t0 > limit_ns) return false;
+        __nanosleep(128);
+    }
+    return true;
+}
+
 template <class P>
 struct alignas(8) PairTail {
     uint64_t full[P::STAGES];        // leader: both CTAs' A/B bytes
@@ -547,6 +621,7 @@ struct alignas(8) PairTail {
     uint64_t acc_empty[P::ACC];      // leader: the epilogue warps of both CTAs released it
     uint64_t sf_ready[P::NSB];       // leader: 8 scale warps staged a buffer
     uint64_t sf_free[P::NSB];        // each CTA: MMAs reading a scale buffer done
+    uint64_t sk_bar;                 // each CTA: the next pair's partial sums landed (stream-K head)
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -564,7 +639,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
-    const int cluster = blockIdx.x >> 1, nclusters = gridDim.x >> 1;
+    const int cluster = blockIdx.x >> 1;
     const uint64_t limit = p.wait_limit_ns;
 
     if (threadIdx.x == 0) {
@@ -581,6 +656,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             mbar_init(&tail->sf_ready[b], 8);
             mbar_init(&tail->sf_free[b], 1);
         }
+        mbar_init(&tail->sk_bar, 1);
         tail->abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -597,7 +673,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
     const int tiles_m2 = (p.rows_a + 255) / 256;
-    const int total = tiles_m2 * p.tiles_n;
     const int sfa_blocks = (p.rows_a + 127) / 128;
 
     if (warp == 0) {
@@ -605,7 +680,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             // ---------------- TMA producer (both CTAs) ----------------
             uint32_t stage = 0, phase = 0;
             bool ok = true;
-            for (int t = cluster; t < total && ok; t += nclusters) {
+            PairWork w;
+            while (ok && w.next(p, cluster)) {
+                const int t = w.t;
                 const int tm = t % tiles_m2, tn = t / tiles_m2;
                 const int a_row = tm * 256 + 128 * (int)rank;
                 const int g0 = tn * BN + BH * (int)rank;          // first B row of this CTA's half
@@ -614,7 +691,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 const int nsfb = max(0, min(((tn * BN) % 128 + BN + 127) / 128, p.sfb_rb_per_group - a0));
                 const uint8_t* sfa_src = p.sfa + (int64_t)(a_row / 128) * p.sfa_rb_stride;
                 const uint8_t* sfb_src = p.sfb + (int64_t)a0 * p.sfb_rb_stride;
-                for (int kt = 0; kt < p.num_kt; ++kt) {
+                for (int kt = w.kb; kt < w.ke; ++kt) {
                     if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
                         ok = false;
                         break;
@@ -652,7 +729,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
             int it = 0;
             bool ok = true;
-            for (int t = cluster; t < total && ok; t += nclusters, ++it) {
+            PairWork w;
+            for (; ok && w.next(p, cluster); ++it) {
                 const uint32_t ab = (uint32_t)(it % P::ACC), au = (uint32_t)(it / P::ACC);
                 if (!mbar_wait(&tail->acc_empty[ab], (au & 1u) ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
@@ -660,7 +738,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + ab * BN;
-                for (int kt = 0; kt < p.num_kt; ++kt) {
+                for (int kt = w.kb; kt < w.ke; ++kt) {
                     if (!mbar_wait(&tail->full[stage], phase, limit) ||
                         !mbar_wait(&tail->sf_ready[sb], sph, limit) || tail->abort_flag) {
                         ok = false;
@@ -673,7 +751,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const uint32_t sf = tmem + P::SF_BASE + sb * P::SF_STRIDE;
                     for (int j = 0; j < nat; ++j)
                         mma_mxf4nvf4_pair(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
-                                          IDESC, sf + j * 4, sf + 16 + j * NBC, (kt > 0 || j > 0) ? 1u : 0u);
+                                          IDESC, sf + j * 4, sf + 16 + j * NBC, (kt > w.kb || j > 0) ? 1u : 0u);
                     tc_commit_pair(&tail->empty[stage], 0x3);
                     tc_commit_pair(&tail->sf_free[sb], 0x3);
                     if (++stage == STAGES) {
@@ -700,10 +778,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t ready_step = (uint32_t)(smem_u32(&tail->sf_ready[1]) - smem_u32(&tail->sf_ready[0]));
         uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
         bool ok = true;
-        for (int t = cluster; t < total && ok; t += nclusters) {
-            const int tn = t / tiles_m2;
+        PairWork w;
+        while (ok && w.next(p, cluster)) {
+            const int tn = w.t / tiles_m2;
             const int off = (tn * BN) % 128;                  // first tile row inside the first scale block
-            for (int kt = 0; kt < p.num_kt; ++kt) {
+            for (int kt = w.kb; kt < w.ke; ++kt) {
                 // read this k-tile's scale words as soon as they land, then wait
                 // for the tensor-memory buffer: only the stores stay on the
                 // MMA's critical path
@@ -771,15 +850,40 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // converting all of them before the stores 133 us; 16 warps were slower).
         const int q = warp & 3;
         const int half = (warp - 2) >> 2;
-        const int c0 = half * (BN / 64), c1 = c0 + BN / 64;
+        const int c0 = half * (BN / 64);
         const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * 4096u;
         const uint32_t empty0 = mapa_shared(smem_u32(&tail->acc_empty[0]), 0);
         const uint32_t empty_step = (uint32_t)sizeof(uint64_t);
         int it = 0;
-        for (int t = cluster; t < total; t += nclusters, ++it) {
-            const int tm = t % tiles_m2, tn = t / tiles_m2;
+        PairWork w;
+        for (; w.next(p, cluster); ++it) {
+            const int tm = w.t % tiles_m2, tn = w.t / tiles_m2;
             const uint32_t ab = (uint32_t)(it % P::ACC), au = (uint32_t)(it / P::ACC);
-            if (!mbar_wait(&tail->acc_full[ab], au & 1u, limit) || tail->abort_flag) {
+            // stream-K roles of this item: a continuation hands its partial sums
+            // to the previous pair; a head adds those of the next pair
+            const bool give = w.kb > 0, take = w.ke < p.num_kt;
+            const int slot_idx = (give ? cluster : cluster + 1) * 2 + (int)rank;
+            bool wait_ok = mbar_wait(&tail->acc_full[ab], au & 1u, limit) && !tail->abort_flag;
+            if (wait_ok && take) {
+                // The head is this pair's last item: with its MMAs done the stage
+                // buffers are free, so one bulk copy brings the next pair's partial
+                // sums (128 x BN FP32) on chip while the accumulator is read.
+                if (warp == 2 && lane == 0) {
+                    wait_ok = sk_wait_ready(p.sk_flags + slot_idx * kSkFlagStride, limit, &tail->abort_flag);
+                    if (wait_ok) {
+                        fence_proxy_async_global();
+                        constexpr uint32_t kPart = 128u * BN * 4u, kPiece = 16384u;
+                        mbar_arrive_expect_tx(&tail->sk_bar, kPart);
+                        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.partial) + (size_t)slot_idx * kPart;
+                        for (uint32_t o = 0; o < kPart; o += kPiece) bulk_load(smem + o, src + o, kPiece, &tail->sk_bar);
+                    }
+                }
+                wait_ok = __shfl_sync(0xffffffffu, wait_ok ? 1 : 0, 0) != 0;
+                if (wait_ok) wait_ok = mbar_wait(&tail->sk_bar, 0u, limit) && !tail->abort_flag;
+                // the copy has read the slot: clear the counter for the next launch
+                if (wait_ok && warp == 2 && lane == 0) st_relaxed_gpu_u32(p.sk_flags + slot_idx * kSkFlagStride, 0u);
+            }
+            if (!wait_ok) {
                 if (lane == 0) {
                     tail->abort_flag = 1;
                     if (p.err) atomicOr(p.err, 1u);
@@ -793,9 +897,99 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const int b_cols = min(BN, p.rows_b - n0);
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
             const float alpha = __fmul_rn(p.ga[0], p.gb[0]);
-            // Read the warp's BN / 2 columns 64 at a time and convert them to
-            // BF16 in registers; release the accumulator after the last read,
-            // then stage and store.
+            // One 32-column chunk (16 BF16 pairs per lane) through a staging box to C.
+            auto store_chunk = [&](int ch, const uint32_t* w16) {
+                if (ch * 32 >= b_cols || q * 32 >= a_rows) return;   // uniform per warp
+                const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
+                if (lane == 0) bulk_wait_group_read<1>();
+                __syncwarp();
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = make_uint4(w16[4 * j], w16[4 * j + 1], w16[4 * j + 2], w16[4 * j + 3]);
+                    st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), v);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmC, box, n0 + ch * 32, a_row0 + q * 32);
+                    bulk_commit_group();
+                }
+            };
+            if (give) {
+                // Continuation: FP32 partial sums to the workspace slot, 4-column
+                // group g of row r at slot[g * 128 + r] (lane-contiguous 16-byte
+                // pieces), then one count per warp.
+                float4* slot = reinterpret_cast<float4*>(p.partial + (size_t)slot_idx * (128 * BN)) + q * 32 + lane;
+#pragma unroll
+                for (int cp = 0; cp < BN / 128; ++cp) {
+                    uint32_t va0[32], va1[32];
+                    tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
+                    tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
+                    tmem_ld_wait();
+                    if (cp == BN / 128 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
+                    }
+                    float4* part = slot + (c0 + cp * 2) * 8 * 128;   // one base, immediate offsets
+                    static_for<8>([&](auto ic) {
+                        constexpr int i = decltype(ic)::value;
+                        st_global_v4_at<i * 2048>(part, va0[4 * i], va0[4 * i + 1], va0[4 * i + 2], va0[4 * i + 3]);
+                        st_global_v4_at<(8 + i) * 2048>(part, va1[4 * i], va1[4 * i + 1], va1[4 * i + 2],
+                                                        va1[4 * i + 3]);
+                    });
+                }
+                // the warp barrier orders every lane's stores before lane 0's
+                // release, which carries them to the acquiring head (cumulativity)
+                __syncwarp();
+                if (lane == 0) red_release_gpu_add_u32(p.sk_flags + slot_idx * kSkFlagStride, 1u);
+                continue;
+            }
+            if (take) {
+                // Head: add the next pair's partial sums (now in the stage
+                // buffers, same layout) before scaling.
+                const uint32_t slot_s = smem_u32(smem) + (uint32_t)(q * 32 + lane) * 16u;
+#pragma unroll
+                for (int cp = 0; cp < BN / 128; ++cp) {
+                    uint32_t va0[32], va1[32];
+                    tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
+                    tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
+                    tmem_ld_wait();
+                    if (cp == BN / 128 - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
+                    }
+                    const uint32_t part_s = slot_s + (uint32_t)((c0 + cp * 2) * 8 * 128) * 16u;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        uint4 x[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) x[i] = ld_shared_v4(part_s + (uint32_t)((4 * g + i) * 128) * 16u);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            uint32_t* v = (g < 2 ? va0 : va1) + 16 * (g & 1) + 4 * i;
+                            v[0] = __float_as_uint(__uint_as_float(v[0]) + __uint_as_float(x[i].x));
+                            v[1] = __float_as_uint(__uint_as_float(v[1]) + __uint_as_float(x[i].y));
+                            v[2] = __float_as_uint(__uint_as_float(v[2]) + __uint_as_float(x[i].z));
+                            v[3] = __float_as_uint(__uint_as_float(v[3]) + __uint_as_float(x[i].w));
+                        }
+                    }
+                    uint32_t bh[32];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        bh[i] = pack_bf16x2(__uint_as_float(va0[2 * i]) * alpha, __uint_as_float(va0[2 * i + 1]) * alpha);
+                        bh[16 + i] =
+                            pack_bf16x2(__uint_as_float(va1[2 * i]) * alpha, __uint_as_float(va1[2 * i + 1]) * alpha);
+                    }
+                    store_chunk(c0 + cp * 2, bh);
+                    store_chunk(c0 + cp * 2 + 1, bh + 16);
+                }
+                continue;
+            }
+            // Whole tile: read the warp's BN / 2 columns 64 at a time and
+            // convert them to BF16 in registers; release the accumulator after
+            // the last read, then stage and store.
             uint32_t bf[BN / 4];
 #pragma unroll
             for (int cp = 0; cp < BN / 128; ++cp) {
@@ -817,25 +1011,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 }
             }
 #pragma unroll
-            for (int h = 0; h < BN / 64; ++h) {
-                const int ch = c0 + h;
-                if (ch * 32 >= b_cols || q * 32 >= a_rows) continue;   // uniform per warp
-                const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
-                if (lane == 0) bulk_wait_group_read<1>();
-                __syncwarp();
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const uint4 w = make_uint4(bf[h * 16 + 4 * j], bf[h * 16 + 4 * j + 1], bf[h * 16 + 4 * j + 2],
-                                               bf[h * 16 + 4 * j + 3]);
-                    st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
-                }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    tma_store_2d(&tmC, box, n0 + ch * 32, a_row0 + q * 32);
-                    bulk_commit_group();
-                }
-            }
+            for (int h = 0; h < BN / 64; ++h) store_chunk(c0 + h, bf + h * 16);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
@@ -931,6 +1107,44 @@ int pair_clusters_resident() {
     return cached[d];
 }
 
+// How the pair kernel covers an m x n x k product: resident pairs, whole
+// tiles, and the stream-K k-tiles of the rest (0 when the tiles fill whole
+// waves, or a tile has a single k-tile and cannot be split).
+struct PairPlan {
+    int clusters = 0;
+    int64_t tiles = 0;
+    int dp_tiles = 0;
+    int64_t sk_units = 0;
+};
+
+bool pair_plan(int64_t m, int64_t n, int64_t k, PairPlan& pl) {
+    if (m <= 128) return false;
+    const int clusters_max = pair_clusters_resident();
+    const int sms = num_sms();
+    if (clusters_max <= 0 || sms < 2) return false;
+    const int64_t tiles = ((m + 255) / 256) * ((n + PairUse::BN - 1) / PairUse::BN);
+    if (tiles >= ((int64_t)1 << 31)) return false;
+    pl.tiles = tiles;
+    pl.clusters = (int)std::min<int64_t>(tiles, std::min(clusters_max, sms / 2));
+    const int64_t num_kt = (k / 64 + 3) / 4;
+    const int64_t P = pl.clusters;
+    if (tiles > P && tiles % P != 0 && num_kt > 1 && P <= 256 && (2 * P) * num_kt < ((int64_t)1 << 31)) {
+        pl.dp_tiles = (int)((tiles / P - 1) * P);
+        pl.sk_units = (tiles - pl.dp_tiles) * num_kt;
+    } else {
+        pl.dp_tiles = (int)tiles;
+        pl.sk_units = 0;
+    }
+    return true;
+}
+
+// Workspace of the stream-K tail: the counters (one 64-byte line per CTA),
+// then one FP32 128 x BN slot per CTA.
+constexpr size_t kSkFlagsBytes = 256 * 2 * kSkFlagStride * sizeof(uint32_t);   // up to 256 pairs
+size_t sk_workspace_bytes(int clusters) {
+    return kSkFlagsBytes + (size_t)clusters * 2 * 128 * PairUse::BN * sizeof(float);
+}
+
 nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                            int clusters, cudaStream_t s) {
     cudaLaunchAttribute attr[2];
@@ -969,6 +1183,12 @@ bool make_out_map(CUtensorMap* map, const void* base, int64_t rows, int64_t cols
 bool ptr_ok(const void* p) { return p && aligned16(p); }
 
 }  // namespace
+
+size_t gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+    PairPlan pl;
+    if (m <= 0 || n <= 0 || k <= 0 || !pair_plan(m, n, k, pl) || pl.sk_units == 0) return 0;
+    return sk_workspace_bytes(pl.clusters);
+}
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -976,7 +1196,6 @@ using namespace nvfp4;
 extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                                      const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c,
                                      int64_t ldc, int64_t m, int64_t n, int64_t k, void* workspace, void* stream) {
-    (void)workspace;
     if (m < 0 || n <= 0 || k <= 0 || ldc < n) return NVFP4_ERR_INVALID_ARGUMENT;
     if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !c)
         return NVFP4_ERR_INVALID_ARGUMENT;
@@ -985,6 +1204,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     if (!ptr_ok(a_codes) || !ptr_ok(a_scales) || !ptr_ok(b_codes) || !ptr_ok(b_scales) || !ptr_ok(c) ||
         (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(b_global) & 3u) || ldc % 8 != 0)
         return NVFP4_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(workspace) & 15u) return NVFP4_ERR_MISALIGNED;
     if (m == 0) return NVFP4_OK;
     const int sms = num_sms();
     if (sms <= 0) return NVFP4_ERR_NO_DEVICE;
@@ -1020,27 +1240,28 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         const int grid = (int)std::min<int64_t>((int64_t)p.tiles_n, sms);
         return launch<CfgDecW, false>(ta, tb, tc, p, grid, s);
     }
-    if (m > 128) {
-        // prefill-class: 2-SM pair tiles of 256 x 224
-        const int clusters_max = pair_clusters_resident();
-        if (clusters_max > 0) {
-            if (!make_codes_map(&ta, a_codes, m, k / 2, 128) ||
-                !make_codes_map(&tb, b_codes, n, k / 2, PairUse::BH) || !make_out_map(&tc, c, m, n, ldc))
-                return NVFP4_ERR_CUDA;
-            p.sfa = a_scales;
-            p.sfb = b_scales;
-            p.sfb_rb_per_group = (int)((n + 127) / 128);
-            p.ga = a_global;
-            p.gb = b_global;
-            p.rows_a = (int)m;
-            p.rows_b = (int)n;
-            p.tiles_m = (int)((m + 255) / 256);
-            p.tiles_n = (int)((n + PairUse::BN - 1) / PairUse::BN);
-            const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
-            if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
-            const int clusters = (int)std::min<int64_t>(tiles, std::min(clusters_max, sms / 2));
-            return launch_pair(ta, tb, tc, p, clusters, s);
-        }
+    PairPlan pl;
+    if (pair_plan(m, n, k, pl)) {
+        // prefill-class: 2-SM pair tiles of 256 x 256, stream-K over the last waves
+        if (!make_codes_map(&ta, a_codes, m, k / 2, 128) ||
+            !make_codes_map(&tb, b_codes, n, k / 2, PairUse::BH) || !make_out_map(&tc, c, m, n, ldc))
+            return NVFP4_ERR_CUDA;
+        p.sfa = a_scales;
+        p.sfb = b_scales;
+        p.sfb_rb_per_group = (int)((n + 127) / 128);
+        p.ga = a_global;
+        p.gb = b_global;
+        p.rows_a = (int)m;
+        p.rows_b = (int)n;
+        p.tiles_m = (int)((m + 255) / 256);
+        p.tiles_n = (int)((n + PairUse::BN - 1) / PairUse::BN);
+        // without a workspace every tile stays whole
+        const bool sk = pl.sk_units > 0 && workspace != nullptr;
+        p.dp_tiles = sk ? pl.dp_tiles : (int)pl.tiles;
+        p.sk_units = sk ? pl.sk_units : 0;
+        p.sk_flags = sk ? reinterpret_cast<uint32_t*>(workspace) : nullptr;
+        p.partial = sk ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + kSkFlagsBytes) : nullptr;
+        return launch_pair(ta, tb, tc, p, pl.clusters, s);
     }
     constexpr int BN = CfgWide::BN;
     if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN) ||

@@ -49,18 +49,21 @@ def test_tiny_workload_end_to_end():
     (128, 256, 256),     # one full tile
     (200, 320, 320),     # ragged m, ragged n tile, partial last k-tile
     (256, 512, 1024),    # several tiles
-    (65, 200, 64),       # smallest k; just above the swap threshold
-    (64, 200, 128),      # swap path, BN 64
-    (33, 304, 192),      # swap path, BN 64 with 33 tokens
-    (17, 136, 64),       # swap path, BN 32
-    (16, 64, 256),       # swap path, BN 16
+    (65, 200, 64),       # smallest k; just above the decode-tile threshold (m <= 64)
+    (64, 200, 128),      # decode tiles: 64 token rows, ragged second weight tile
+    (33, 304, 192),      # decode tiles with 33 tokens
+    (17, 136, 64),       # decode tiles, one weight tile of 136 rows
+    (16, 64, 256),       # decode tiles, 16 tokens x 64 weight rows
     (1, 64, 320),        # single token
     (300, 16, 448),      # narrow n
     (129, 264, 128),     # 2-SM pair tile with one valid row in its second half
     (520, 776, 512),     # pair tiles: ragged m (3 row tiles) and n (4th column tile 8 wide)
     (1000, 2072, 576),   # many pair tiles, both edges ragged, partial last k-tile
-    (2304, 2336, 256),   # more pair tiles than resident pairs: a partial second wave
+    (2304, 2336, 256),   # more pair tiles than resident pairs, one k-tile: a partial second wave
     (2560, 4000, 128),   # ditto, with the last wave at the ragged n edge
+    (2304, 2336, 512),   # 90 pair tiles, two k-tiles: every tile shared out stream-K
+    (4608, 4352, 1088),  # 306 tiles: 222 whole, the k-tiles of 84 shared out; partial last k-tile
+    (2350, 4104, 768),   # 170 tiles: stream-K tiles at both ragged edges (last column tile 8 wide)
 ])
 def test_gemm_matches_oracle(m, n, k):
     (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 0)
@@ -79,6 +82,36 @@ def test_gemm_output_row_stride():
     ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
     assert_gemm_close(to_host_f64(out[:, :96]), ref, "strided")
     assert torch.all(out[:, 96:] == 7.0)                  # nothing written past n
+
+
+def test_stream_k_workspace_reuse_and_without_workspace():
+    """A shape that splits tiles between pairs: repeated calls on one
+    workspace, and a call with no workspace (every tile whole), all match the
+    oracle; the workspace counters return to zero after each call."""
+    import torch
+    m, n, k = 2304, 2336, 512
+    need = nv.nvfp4_workspace_bytes(nv.OP_GEMM, m, n, k, 0)
+    assert need > 0
+    assert nv.nvfp4_workspace_bytes(nv.OP_GEMM, 64, n, k, 0) == 0          # decode tiles: none
+    (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 3)
+    ta, tw = nvfp4_from_host(ac, asf, ga), nvfp4_from_host(wc, wsf, gw)
+    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream().cuda_stream
+    for it in range(3):
+        c = torch.full((m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+        for ws_ptr in (ws.data_ptr(), None):
+            st = nv.nvfp4_gemm(ta.codes.data_ptr(), ta.scales.data_ptr(), ta.global_scale.data_ptr(),
+                               tw.codes.data_ptr(), tw.scales.data_ptr(), tw.global_scale.data_ptr(), c.data_ptr(),
+                               n, m, n, k, ws_ptr, stream)
+            assert st == 0
+            _sync()
+            assert int(ws[:32768].to(torch.int64).sum()) == 0
+            assert_gemm_close(to_host_f64(c), ref, f"stream-K call {it}, workspace {ws_ptr is not None}")
+    # a misaligned workspace is refused before anything runs
+    assert nv.nvfp4_gemm(ta.codes.data_ptr(), ta.scales.data_ptr(), ta.global_scale.data_ptr(),
+                         tw.codes.data_ptr(), tw.scales.data_ptr(), tw.global_scale.data_ptr(), c.data_ptr(),
+                         n, m, n, k, ws.data_ptr() + 4, stream) == 3     # NVFP4_ERR_MISALIGNED
 
 
 @pytest.fixture(scope="module")
