@@ -580,11 +580,11 @@ __device__ __forceinline__ void static_for(F&& f) {
 struct PairWork {
     int t = -1, kb = 0, ke = 0;        // current item: tile t, k-tiles [kb, ke)
     int u = -1;                        // next stream-K unit (sk_units < 2^31, host), -1 in the whole-tile phase
-    __device__ bool next(const GemmArgs& p, int cluster) {
+    __device__ bool next(const GemmArgs& p, int cluster, int dp_tiles) {
         const int P = (int)(gridDim.x >> 1);
         if (u < 0) {
             t = t < 0 ? cluster : t + P;
-            if (t < p.dp_tiles) {
+            if (t < dp_tiles) {
                 kb = 0;
                 ke = p.num_kt;
                 return true;
@@ -594,7 +594,7 @@ struct PairWork {
         const int u1 = (int)(p.sk_units * (cluster + 1) / P);
         if (u >= u1) return false;
         const int j = u / p.num_kt;
-        t = p.dp_tiles + j;
+        t = dp_tiles + j;
         kb = u - j * p.num_kt;
         ke = min(p.num_kt, kb + (u1 - u));
         u += ke - kb;
@@ -612,8 +612,15 @@ __device__ __forceinline__ bool sk_wait_ready(const uint32_t* ready, uint64_t li
     return true;
 }
 
-template <class P>
-struct alignas(8) PairTail {
+struct PairGroups {                  // grouped form: per-expert prefixes of pair tiles and scale blocks
+    int total_tiles;
+    int tile_prefix[kMaxGroups + 1];
+    int blk_prefix[kMaxGroups + 1];
+};
+struct PairNoGroups {};
+
+template <class P, bool GROUPED = false>
+struct alignas(8) PairTail : std::conditional_t<GROUPED, PairGroups, PairNoGroups> {
     uint64_t full[P::STAGES];        // leader: both CTAs' A/B bytes
     uint64_t empty[P::STAGES];       // each CTA: released by the leader's MMA commit
     uint64_t sfl[P::STAGES];         // each CTA: its own scale bytes landed
@@ -626,7 +633,60 @@ struct alignas(8) PairTail {
     volatile int abort_flag;
 };
 
-template <class P>
+// Where pair tile t lies, for the CTA of rank `rank`.  Plain: tiles run over
+// (256-row m-tile fastest, n-tile).  Grouped: expert e owns tiles
+// [tile_prefix[e], tile_prefix[e + 1]), ceil(n_e / 256) m-tiles per n-tile, m
+// fastest; its rows start at offsets[e] and its 128-row scale blocks at
+// blk_prefix[e]; the rows of a CTA past the expert's end belong to the next
+// expert and are neither scaled from its blocks nor stored.
+struct PairTile {
+    int a_row;       // first A (and output) row of this CTA's half
+    int a_rows;      // valid rows of the half (<= 0: none)
+    int sfa_rb;      // 128-row A scale block of the half
+    bool sfa_ok;     // that block holds this half's rows
+    int n0;          // first output column
+    int b_row0;      // first B tensor-map row of the pair tile
+    int group;
+};
+template <int BN, bool GROUPED, class TAIL>
+__device__ __forceinline__ PairTile pair_tile(const GemmArgs& p, const TAIL* tail, int t, uint32_t rank) {
+    PairTile pt;
+    int tm, tn, n_e, blocks;
+    if constexpr (GROUPED) {
+        int lo = 0, hi = p.num_groups;   // largest e with tile_prefix[e] <= t
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tail->tile_prefix[mid] <= t) lo = mid; else hi = mid;
+        }
+        const int e = lo, r0 = p.offsets[e];
+        n_e = p.offsets[e + 1] - r0;
+        const int mt2 = (n_e + 255) / 256;
+        const int local = t - tail->tile_prefix[e];
+        tm = local % mt2;
+        tn = local / mt2;
+        pt.a_row = r0 + tm * 256 + 128 * (int)rank;
+        pt.sfa_rb = tail->blk_prefix[e] + 2 * tm + (int)rank;
+        blocks = (n_e + 127) / 128;
+        pt.b_row0 = e * p.rows_b + tn * BN;
+        pt.group = e;
+    } else {
+        const int tiles_m2 = (p.rows_a + 255) / 256;
+        tm = t % tiles_m2;
+        tn = t / tiles_m2;
+        n_e = p.rows_a;
+        pt.a_row = tm * 256 + 128 * (int)rank;
+        pt.sfa_rb = 2 * tm + (int)rank;
+        blocks = (p.rows_a + 127) / 128;
+        pt.b_row0 = tn * BN;
+        pt.group = 0;
+    }
+    pt.a_rows = n_e - (tm * 256 + 128 * (int)rank);
+    pt.sfa_ok = 2 * tm + (int)rank < blocks;
+    pt.n0 = tn * BN;
+    return pt;
+}
+
+template <class P, bool GROUPED>
 __global__ void __launch_bounds__(kPairThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
@@ -635,7 +695,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_smem = smem + STAGES * P::STAGE_BYTES;
-    PairTail<P>* tail = reinterpret_cast<PairTail<P>*>(epi_smem + P::EPI_BYTES);
+    PairTail<P, GROUPED>* tail = reinterpret_cast<PairTail<P, GROUPED>*>(epi_smem + P::EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_ctarank();
     const bool leader = rank == 0;
@@ -668,12 +728,54 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tmem_relinquish_pair();
     }
     pdl_wait();
+    if constexpr (GROUPED) {
+        // per-expert prefixes (the offsets may come from the previous kernel)
+        if (warp == 2) {
+            const int E = p.num_groups;
+            const int per = (E + 31) / 32;
+            int t_loc = 0, b_loc = 0;
+            for (int i = 0; i < per; ++i) {
+                const int e = lane * per + i;
+                if (e < E) {
+                    const int n_e = p.offsets[e + 1] - p.offsets[e];
+                    t_loc += (n_e + 255) / 256 * p.tiles_n;
+                    b_loc += (n_e + 127) / 128;
+                }
+            }
+            int t_inc = t_loc, b_inc = b_loc;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int tv = __shfl_up_sync(0xFFFFFFFFu, t_inc, o);
+                const int bv = __shfl_up_sync(0xFFFFFFFFu, b_inc, o);
+                if (lane >= o) {
+                    t_inc += tv;
+                    b_inc += bv;
+                }
+            }
+            int t_run = t_inc - t_loc, b_run = b_inc - b_loc;
+            for (int i = 0; i < per; ++i) {
+                const int e = lane * per + i;
+                if (e < E) {
+                    tail->tile_prefix[e] = t_run;
+                    tail->blk_prefix[e] = b_run;
+                    const int n_e = p.offsets[e + 1] - p.offsets[e];
+                    t_run += (n_e + 255) / 256 * p.tiles_n;
+                    b_run += (n_e + 127) / 128;
+                }
+            }
+            if (lane == 31) {
+                tail->tile_prefix[E] = t_inc;
+                tail->blk_prefix[E] = b_inc;
+                tail->total_tiles = t_inc;
+            }
+        }
+    }
     tc_fence_before();
-    cluster_sync();          // both CTAs' barriers initialized, tensor memory allocated
+    cluster_sync();          // both CTAs' barriers initialized, tensor memory allocated (and prefixes written)
     tc_fence_after();
     const uint32_t tmem = tail->tmem_base;
-    const int tiles_m2 = (p.rows_a + 255) / 256;
-    const int sfa_blocks = (p.rows_a + 127) / 128;
+    int dp_tiles = p.dp_tiles;               // grouped: every tile whole
+    if constexpr (GROUPED) dp_tiles = tail->total_tiles;
 
     if (warp == 0) {
         if (lane == 0) {
@@ -681,16 +783,16 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             PairWork w;
-            while (ok && w.next(p, cluster)) {
-                const int t = w.t;
-                const int tm = t % tiles_m2, tn = t / tiles_m2;
-                const int a_row = tm * 256 + 128 * (int)rank;
-                const int g0 = tn * BN + BH * (int)rank;          // first B row of this CTA's half
-                const bool sfa_ok = a_row / 128 < sfa_blocks;
-                const int a0 = (tn * BN) / 128;                   // B scales: all BN rows of the tile
-                const int nsfb = max(0, min(((tn * BN) % 128 + BN + 127) / 128, p.sfb_rb_per_group - a0));
-                const uint8_t* sfa_src = p.sfa + (int64_t)(a_row / 128) * p.sfa_rb_stride;
-                const uint8_t* sfb_src = p.sfb + (int64_t)a0 * p.sfb_rb_stride;
+            while (ok && w.next(p, cluster, dp_tiles)) {
+                const PairTile pt = pair_tile<BN, GROUPED>(p, tail, w.t, rank);
+                const int a_row = pt.a_row;
+                const int g0 = pt.b_row0 + BH * (int)rank;        // first B row of this CTA's half
+                const bool sfa_ok = pt.sfa_ok;
+                const int a0 = pt.n0 / 128;                       // B scales: all BN rows of the tile
+                const int nsfb = max(0, min((pt.n0 % 128 + BN + 127) / 128, p.sfb_rb_per_group - a0));
+                const uint8_t* sfa_src = p.sfa + (int64_t)pt.sfa_rb * p.sfa_rb_stride;
+                const uint8_t* sfb_src =
+                    p.sfb + (int64_t)pt.group * p.sfb_group_stride + (int64_t)a0 * p.sfb_rb_stride;
                 for (int kt = w.kb; kt < w.ke; ++kt) {
                     if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
                         ok = false;
@@ -730,7 +832,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             int it = 0;
             bool ok = true;
             PairWork w;
-            for (; ok && w.next(p, cluster); ++it) {
+            for (; ok && w.next(p, cluster, dp_tiles); ++it) {
                 const uint32_t ab = (uint32_t)(it % P::ACC), au = (uint32_t)(it / P::ACC);
                 if (!mbar_wait(&tail->acc_empty[ab], (au & 1u) ^ 1u, limit) || tail->abort_flag) {
                     ok = false;
@@ -778,11 +880,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t ready_step = (uint32_t)(smem_u32(&tail->sf_ready[1]) - smem_u32(&tail->sf_ready[0]));
         uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
         bool ok = true;
-        PairWork w;
-        while (ok && w.next(p, cluster)) {
-            const int tn = w.t / tiles_m2;
-            const int off = (tn * BN) % 128;                  // first tile row inside the first scale block
-            for (int kt = w.kb; kt < w.ke; ++kt) {
+        PairWork wk;
+        while (ok && wk.next(p, cluster, dp_tiles)) {
+            const int off = pair_tile<BN, GROUPED>(p, tail, wk.t, rank).n0 % 128;   // first tile row in its first scale block
+            for (int kt = wk.kb; kt < wk.ke; ++kt) {
                 // read this k-tile's scale words as soon as they land, then wait
                 // for the tensor-memory buffer: only the stores stay on the
                 // MMA's critical path
@@ -856,8 +957,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t empty_step = (uint32_t)sizeof(uint64_t);
         int it = 0;
         PairWork w;
-        for (; w.next(p, cluster); ++it) {
-            const int tm = w.t % tiles_m2, tn = w.t / tiles_m2;
+        for (; w.next(p, cluster, dp_tiles); ++it) {
             const uint32_t ab = (uint32_t)(it % P::ACC), au = (uint32_t)(it / P::ACC);
             // stream-K roles of this item: a continuation hands its partial sums
             // to the previous pair; a head adds those of the next pair
@@ -891,15 +991,36 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int a_row0 = tm * 256 + 128 * (int)rank;
-            const int n0 = tn * BN;
-            const int a_rows = p.rows_a - a_row0;
+            const PairTile pt = pair_tile<BN, GROUPED>(p, tail, w.t, rank);
+            const int a_row0 = pt.a_row;
+            const int n0 = pt.n0;
+            const int a_rows = pt.a_rows;
             const int b_cols = min(BN, p.rows_b - n0);
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
-            const float alpha = __fmul_rn(p.ga[0], p.gb[0]);
+            const float alpha = __fmul_rn(p.ga[pt.group], p.gb[pt.group]);
             // One 32-column chunk (16 BF16 pairs per lane) through a staging box to C.
             auto store_chunk = [&](int ch, const uint32_t* w16) {
                 if (ch * 32 >= b_cols || q * 32 >= a_rows) return;   // uniform per warp
+                if (GROUPED && q * 32 + 32 > a_rows) {
+                    // the expert's last rows: the next rows of C belong to the next
+                    // expert, so no 32-row box; each lane stores its own row
+                    if (q * 32 + lane < a_rows) {
+                        __nv_bfloat16* crow = p.c + (int64_t)(a_row0 + q * 32 + lane) * p.ldc + n0 + ch * 32;
+                        if (b_cols - ch * 32 >= 32) {
+#pragma unroll
+                            for (int j = 0; j < 4; ++j)
+                                *reinterpret_cast<uint4*>(crow + 8 * j) =
+                                    make_uint4(w16[4 * j], w16[4 * j + 1], w16[4 * j + 2], w16[4 * j + 3]);
+                        } else {
+                            const int ncols = b_cols - ch * 32;
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (i < ncols)
+                                    crow[i] = __ushort_as_bfloat16((unsigned short)(w16[i >> 1] >> (16 * (i & 1))));
+                        }
+                    }
+                    return;
+                }
                 const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
                 if (lane == 0) bulk_wait_group_read<1>();
                 __syncwarp();
@@ -1066,15 +1187,17 @@ nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtens
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args));
 }
 
+template <bool GROUPED>
 constexpr size_t kPairSmem =
-    1024 + (size_t)PairUse::STAGES * PairUse::STAGE_BYTES + PairUse::EPI_BYTES + sizeof(PairTail<PairUse>);
-static_assert(kPairSmem <= 232448, "shared memory");
+    1024 + (size_t)PairUse::STAGES * PairUse::STAGE_BYTES + PairUse::EPI_BYTES + sizeof(PairTail<PairUse, GROUPED>);
+static_assert(kPairSmem<true> <= 232448, "shared memory");
 
+template <bool GROUPED>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters);
     cfg.blockDim = dim3(kPairThreads);
-    cfg.dynamicSmemBytes = kPairSmem;
+    cfg.dynamicSmemBytes = kPairSmem<GROUPED>;
     cfg.stream = s;
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
@@ -1088,6 +1211,7 @@ cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute
 }
 
 // Number of CTA pairs that can be resident at once (one CTA per SM), per device.
+template <bool GROUPED = false>
 int pair_clusters_resident() {
     static std::mutex mu;
     static int cached[64] = {};
@@ -1095,11 +1219,12 @@ int pair_clusters_resident() {
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return 0;
     std::lock_guard<std::mutex> lk(mu);
     if (cached[d] == 0) {
-        auto kern = gemm_pair_kernel<PairUse>;
-        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem) != cudaSuccess)
+        auto kern = gemm_pair_kernel<PairUse, GROUPED>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem<GROUPED>) !=
+            cudaSuccess)
             return 0;
         cudaLaunchAttribute attr[2];
-        cudaLaunchConfig_t cfg = pair_config(1, nullptr, attr);
+        cudaLaunchConfig_t cfg = pair_config<GROUPED>(1, nullptr, attr);
         int n = 0;
         if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) return 0;
         cached[d] = n;
@@ -1145,11 +1270,12 @@ size_t sk_workspace_bytes(int clusters) {
     return kSkFlagsBytes + (size_t)clusters * 2 * 128 * PairUse::BN * sizeof(float);
 }
 
+template <bool GROUPED = false>
 nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                            int clusters, cudaStream_t s) {
     cudaLaunchAttribute attr[2];
-    cudaLaunchConfig_t cfg = pair_config(clusters, s, attr);
-    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairUse>, ta, tb, tc, args));
+    cudaLaunchConfig_t cfg = pair_config<GROUPED>(clusters, s, attr);
+    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairUse, GROUPED>, ta, tb, tc, args));
 }
 
 // Kernel configurations: 64 < m <= 128 and the grouped form use 128 x 192
@@ -1326,6 +1452,23 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     p.err = device_error_word();
     if (!p.err) return NVFP4_ERR_CUDA;
     CUtensorMap ta, tb, tc;
+    // Experts of 192 rows or more on average (prefill-sized MoE): 256 x 256
+    // pair tiles, every tile whole; smaller groups would mostly pad a 256-row
+    // tile, so they take the 128 x 192 single-SM tiles.
+    const int clusters_max = pair_clusters_resident<true>();
+    if (clusters_max > 0 && sms >= 2 && total_rows >= 192 * (int64_t)num_experts) {
+        if (!make_codes_map(&ta, a_codes, total_rows, k / 2, 128) ||
+            !make_codes_map(&tb, b_codes, n * num_experts, k / 2, PairUse::BH) ||
+            !make_out_map(&tc, c, total_rows, n, n))
+            return NVFP4_ERR_CUDA;
+        p.tiles_n = (int)((n + PairUse::BN - 1) / PairUse::BN);
+        p.dp_tiles = 0;
+        p.sk_units = 0;
+        // upper bound of the tile count: sum_e ceil(n_e / 256) <= total_rows / 256 + num_experts
+        const int64_t max_tiles = (total_rows / 256 + num_experts) * (int64_t)p.tiles_n;
+        const int clusters = (int)std::min<int64_t>(max_tiles, std::min(clusters_max, sms / 2));
+        return launch_pair<true>(ta, tb, tc, p, clusters, s);
+    }
     if (!make_codes_map(&ta, a_codes, total_rows, k / 2, 128) ||
         !make_codes_map(&tb, b_codes, n * num_experts, k / 2, BN) || !make_out_map(&tc, c, total_rows, n, n))
         return NVFP4_ERR_CUDA;

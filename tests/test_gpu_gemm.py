@@ -154,10 +154,16 @@ def test_decode_workload_full(m, decode_weights):
     assert_gemm_close(to_host_f64(c), ref, f"decode m={m}")
 
 
-def test_grouped_gemm_ragged_experts():
-    sizes = [0, 5, 128, 130, 0, 1, 257, 64]
+@pytest.mark.parametrize("sizes,k,n", [
+    ([0, 5, 128, 130, 0, 1, 257, 64], 320, 200),               # small experts: 128 x 192 single-SM tiles
+    # experts of >= 192 rows on average: 256 x 256 pair tiles; an expert of 129
+    # rows (one valid row in the second half), of exactly 256, of 1, of 0, and
+    # ragged n (last column tile 8 wide) with a partial last k-tile
+    ([300, 0, 129, 256, 511, 1, 385, 200], 576, 520),
+    ([256] * 3 + [255, 257], 1024, 256),
+])
+def test_grouped_gemm_ragged_experts(sizes, k, n):
     off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
-    k, n = 320, 200
     a = W.gaussian_bf16((int(off[-1]), k), 0, 44, 1.0, outlier_frac=0.01)
     ac, asf, ga = O.quantize_1d_grouped(a, off)
     E = len(sizes)
