@@ -121,11 +121,13 @@ nvfp4_status_t nvfp4_workspace_init(void* workspace, size_t bytes, void* stream)
  *                every byte of each group's padded scale block is written.
  *   global_scale device, FP32 [max(1, num_groups)].
  *   workspace    nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_ACT, rows, 0, k, num_groups).
- * One tensor (group_offsets NULL): one cooperative launch, one CTA per SM
- * (amax pass, a grid barrier through the workspace, quantize pass); the
- * launch waits until every SM can take its CTA.  Row groups: two kernels, a
- * per-group amax reduction, then the quantizer (launched with programmatic
- * dependent launch so its start overlaps the reduction's end).
+ * When k % 64 == 0 (and, with groups, num_groups <= 1024): one cooperative
+ * launch, one CTA per SM -- an amax pass (per group, folded into the
+ * workspace), a grid barrier through the workspace, a quantize pass; the
+ * launch waits until every SM can take its CTA.  Otherwise two kernels: a
+ * per-group (or whole-tensor) amax reduction, then the quantizer (launched
+ * with programmatic dependent launch so its start overlaps the reduction's
+ * end).
  * After nvfp4_get_last_device_error reports NVFP4_ERR_TIMEOUT, initialize the
  * workspace again before reusing it.
  */
@@ -141,15 +143,15 @@ nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_
  * owns every byte of device memory and hands out no allocator, or a
  * latency-critical path that may not call cudaMalloc (it can synchronize the
  * whole device).
- *   Scratch: a fixed 41216-byte array in the library's device image (each GPU
+ *   Scratch: a fixed 49408-byte array in the library's device image (each GPU
  *   that loads the library holds it until the process exits), enough for at
  *   most 1024 row groups; num_groups > 1024 returns
  *   NVFP4_ERR_UNSUPPORTED_SHAPE.
  *   The first call on a device looks up the array's device address with that
  *   device current; make that first call before any stream capture.
- *   Each call first clears, with an asynchronous memset on stream, the part of
- *   the array that must start at zero; otherwise it behaves exactly like
- *   nvfp4_quantize_act (same arguments, results, errors).
+ *   Each call first clears the array with an asynchronous memset on stream;
+ *   otherwise it behaves exactly like nvfp4_quantize_act (same arguments,
+ *   results, errors).
  *   All calls on a device share the one array and it keeps the last call's
  *   contents: calls that overlap on the GPU (e.g. on two streams without an
  *   ordering between them) race and produce wrong results.

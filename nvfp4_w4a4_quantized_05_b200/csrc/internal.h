@@ -32,22 +32,23 @@ constexpr int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 
 inline nvfp4_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
 
-// Workspace layout of the quantizers (bytes):
-//   [0, 4)         CTA completion counter (two-kernel path) or grid-barrier
-//                  arrivals (one-launch path), uint32
-//   [4, 8)         grid-barrier departures (one-launch path), uint32
-//   [16, 16+4G)    per-group amax as FP32 bit patterns (uint32)
-//   [pad_off, +4(G+1))  per-group first scale row (int32), written each call
-//   [part_off, +128*kMaxFusedCtas)  one-launch path: the word of CTA c at
-//                  part_off + 128 c (one per 128-byte line, so that pollers
-//                  spread over the L2 slices)
+// Workspace layout of the quantizers (bytes); G = number of row groups:
+//   [0, 128 * kMaxFusedCtas)  one-launch path: the word of CTA c at 128 c,
+//                  generation << 32 | BF16 amax bits (uint64; one per 128-byte
+//                  line, so that pollers spread over the L2 slices).  At a
+//                  fixed place, so that every call on the workspace, with or
+//                  without groups, steps the same generation count.
+//   [T, T + 4)     two-kernel path: CTA completion counter (uint32), T = quant_ws_two_off()
+//   [T + 16, T + 16 + 4G)  two-kernel path: per-group amax as FP32 bit patterns (uint32)
+//   [pad_off, +4(G+1))     per-group first scale row (int32), written each call
+//   [gword_off, +8G)       one-launch grouped path: per-group generation << 32 | amax bits (uint64)
 constexpr int kMaxFusedCtas = 256;
-constexpr int kPartStrideWords = 32;
-constexpr int64_t quant_ws_amax_off() { return 16; }
-constexpr int64_t quant_ws_pad_off(int groups) { return round_up(16 + 4 * (int64_t)groups, 16); }
-constexpr int64_t quant_ws_part_off(int groups) { return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 128); }
-constexpr int64_t quant_ws_bytes(int groups) {
-    return round_up(quant_ws_part_off(groups) + 4 * (int64_t)kPartStrideWords * kMaxFusedCtas, 256);
+constexpr int kPartStrideWords = 16;   // uint64 words: 128 bytes
+constexpr int64_t quant_ws_two_off() { return 128 * (int64_t)kMaxFusedCtas; }
+constexpr int64_t quant_ws_pad_off(int groups) { return round_up(quant_ws_two_off() + 16 + 4 * (int64_t)groups, 16); }
+constexpr int64_t quant_ws_gword_off(int groups) {
+    return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 128);
 }
+constexpr int64_t quant_ws_bytes(int groups) { return round_up(quant_ws_gword_off(groups) + 8 * (int64_t)groups, 256); }
 
 }  // namespace nvfp4

@@ -436,17 +436,23 @@ constexpr int kTaskVals = 1024;                  // values per warp task
 constexpr int kTaskBytes = kTaskVals * 2;
 constexpr int kStage = 3;                        // task slots per warp
 
+constexpr int kMaxFusedGroups = 1024;            // row groups the one-launch form takes
+
 struct FusedArgs {
     const uint16_t* x;
     int64_t ld;
     int rows, k, nseg, scale_cols;
-    int tasks;        // round128(rows) * nseg
+    int tasks;        // padded rows * nseg: one tensor round128(rows); grouped an upper bound,
+                      // the exact count follows from the offsets on the device
     int full_segs;    // segments that need no guards: k / 1024
     uint32_t sc4x512; // (scale_cols / 4) * 512: bytes of one 128-row band of scale tiles
-    float* gscale;
+    float* gscale;    // [groups]
     uint8_t* codes;
     uint8_t* scales;
-    uint32_t* part;   // per-CTA generation | amax words, 32 words apart
+    uint64_t* part;   // per-CTA generation << 32 | amax words, kPartStrideWords apart
+    uint64_t* gword;  // grouped: per-group generation << 32 | amax words
+    const int32_t* offsets;   // grouped: [groups + 1]; nullptr for one tensor
+    int groups;
     uint64_t limit;
     unsigned* err;
 };
@@ -477,50 +483,147 @@ __device__ __forceinline__ LaneC make_lanec(int lane) {
     return lc;
 }
 
-// Task positions walk one task at a time, row-major over (row, segment).
-struct SrcCursor {   // which box a task's values come from
-    int row, seg;
-    __device__ __forceinline__ void init(const FusedArgs& a, int t) {
-        row = t / a.nseg;
-        seg = t - row * a.nseg;
+// Tasks run over padded rows: the scale layout gives each group of rows
+// (one group for one tensor) a whole number of 128-row scale blocks.  Group
+// e owns padded rows [128 blk[e], 128 blk[e + 1]); padded row pr of it is
+// tensor row off[e] + pr - 128 blk[e] while that is below off[e + 1], and
+// padding (zero values: zero scale bytes, no codes) after.
+struct GroupTab {       // offsets and block prefixes, in shared memory
+    const int* off;     // [G + 1]
+    const int* blk;     // [G + 1]
+    int G;
+};
+struct RowMap {
+    int e;        // group of the current padded row
+    int pbeg;     // its first padded row
+    int pend;     // its first padded row past the group
+    int base;     // tensor row = padded row + base
+    int rlast;    // the group's rows end at this tensor row
+    __device__ __forceinline__ void one(int rows) {
+        e = 0;
+        pbeg = 0;
+        pend = 0x7FFFFFFF;
+        base = 0;
+        rlast = rows;
     }
-    __device__ __forceinline__ void next(const FusedArgs& a) {
-        if (++seg == a.nseg) {
-            seg = 0;
-            ++row;
+    __device__ __forceinline__ void set(const GroupTab& gt, int g) {
+        e = g;
+        pbeg = 128 * gt.blk[g];
+        pend = 128 * gt.blk[g + 1];
+        base = gt.off[g] - 128 * gt.blk[g];
+        rlast = gt.off[g + 1];
+    }
+    // the last group whose first padded row is at or before pr (it holds pr:
+    // empty groups start where the next one does)
+    __device__ __forceinline__ void seek(const GroupTab& gt, int pr) {
+        int lo = 0, hi = gt.G;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (128 * gt.blk[mid] <= pr) lo = mid; else hi = mid;
         }
+        set(gt, lo);
+    }
+    __device__ __forceinline__ void step(const GroupTab& gt, int pr) {
+        while (pr >= pend && e + 1 < gt.G) set(gt, e + 1);
+    }
+    __device__ __forceinline__ void step_back(const GroupTab& gt, int pr) {
+        while (pr < pbeg && e > 0) set(gt, e - 1);
     }
 };
-struct DstCursor {   // where a task's codes and scale words go (32-bit byte offsets)
+
+// Task positions walk one task at a time, row-major over (padded row, segment).
+template <bool GROUPED>
+struct SrcCursor {   // which values a task holds
     int row, seg;
-    uint32_t co;     // row * k / 2 + seg * 512
-    uint32_t so;     // scale word of the segment's first four blocks
-    __device__ __forceinline__ void set_row(const FusedArgs& a) {
-        const uint32_t r = (uint32_t)row;
-        co = r * (uint32_t)(a.k >> 1) + ((uint32_t)seg << 9);
-        so = (r >> 7) * a.sc4x512 + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + ((uint32_t)seg << 13);
-    }
-    __device__ __forceinline__ void init(const FusedArgs& a, int t) {
+    RowMap m;
+    __device__ __forceinline__ void init(const FusedArgs& a, const GroupTab& gt, int t) {
         row = t / a.nseg;
         seg = t - row * a.nseg;
-        set_row(a);
+        if constexpr (GROUPED) m.seek(gt, row); else m.one(a.rows);
     }
-    __device__ __forceinline__ void next(const FusedArgs& a) {
+    __device__ __forceinline__ void next(const FusedArgs& a, const GroupTab& gt) {
         if (++seg == a.nseg) {
             seg = 0;
             ++row;
+            if constexpr (GROUPED) m.step(gt, row);
+        }
+    }
+    __device__ __forceinline__ void prev(const FusedArgs& a, const GroupTab& gt) {
+        if (seg-- == 0) {
+            seg = a.nseg - 1;
+            --row;
+            if constexpr (GROUPED) m.step_back(gt, row);
+        }
+    }
+    __device__ __forceinline__ bool valid() const { return row + m.base < m.rlast; }
+    __device__ __forceinline__ int real() const { return row + m.base; }
+};
+template <bool GROUPED>
+struct DstCursor {   // where a task's codes and scale words go (32-bit byte offsets)
+    int row, seg;
+    RowMap m;
+    uint32_t co;     // tensor row * k / 2 + seg * 512 (used for rows that hold values)
+    uint32_t so;     // scale word of the segment's first four blocks (padded row)
+    __device__ __forceinline__ void set_row(const FusedArgs& a) {
+        const uint32_t r = (uint32_t)row;
+        co = (uint32_t)(row + m.base) * (uint32_t)(a.k >> 1) + ((uint32_t)seg << 9);
+        so = (r >> 7) * a.sc4x512 + (r & 31u) * 16u + ((r >> 5) & 3u) * 4u + ((uint32_t)seg << 13);
+    }
+    __device__ __forceinline__ void init(const FusedArgs& a, const GroupTab& gt, int t) {
+        row = t / a.nseg;
+        seg = t - row * a.nseg;
+        if constexpr (GROUPED) m.seek(gt, row); else m.one(a.rows);
+        set_row(a);
+    }
+    __device__ __forceinline__ void next(const FusedArgs& a, const GroupTab& gt) {
+        if (++seg == a.nseg) {
+            seg = 0;
+            ++row;
+            if constexpr (GROUPED) m.step(gt, row);
             set_row(a);
         } else {
             co += kTaskVals / 2;
             so += 8192u;   // 16 scale tiles of 512 bytes per segment
         }
     }
+    __device__ __forceinline__ void prev(const FusedArgs& a, const GroupTab& gt) {
+        if (seg-- == 0) {
+            seg = a.nseg - 1;
+            --row;
+            if constexpr (GROUPED) m.step_back(gt, row);
+            set_row(a);
+        } else {
+            co -= kTaskVals / 2;
+            so -= 8192u;
+        }
+    }
+    __device__ __forceinline__ bool valid() const { return row + m.base < m.rlast; }
 };
 
-// Quantize the task held in slot sb.  FULL: the whole task is inside the tensor.
-template <bool FULL>
-__device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb, const DstCursor& t,
-                                              const LaneC& lc, const BlockQ& c, const uint64_t* rtab) {
+// Per-group quantizer constants: the global scale g and the bracket constants.
+struct GroupQ {
+    float g;
+    BlockQ c;
+};
+__device__ __forceinline__ GroupQ make_groupq(uint32_t amax_bits) {
+    GroupQ q;
+    const float amax = __uint_as_float(amax_bits << 16);
+    q.g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kGlobalDen);
+    q.c = make_blockq(q.g);
+    return q;
+}
+// (r, r) for scale byte sf, d = float(sf) g, r = d == 0 ? 0 : min(1 / d, FLT_MAX):
+// the same value the table of the one-tensor form holds.
+__device__ __forceinline__ uint64_t block_rr(uint32_t sf, float g) {
+    const float d = __fmul_rn(e4m3_to_f32(sf), g);
+    return pack_rr((d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX));
+}
+
+// Quantize the task held in slot sb.  FULL: the whole task is inside the
+// tensor.  One tensor: r from the per-CTA table; grouped: r computed per block.
+template <bool FULL, bool GROUPED>
+__device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
+                                              const LaneC& lc, const GroupQ& gq, const uint64_t* rtab) {
     uint4 u[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4*>(sb + lc.ld_off[i]);
@@ -531,8 +634,15 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
     const uint32_t m = bmax_abs(__byte_perm(m0, m1, 0x5410), __byte_perm(m0, m1, 0x7632));
     const float b0 = __uint_as_float((m << 16) & 0x7FFF0000u);
     const float b1 = __uint_as_float(m & 0x7FFF0000u);
-    const uint32_t pair = block_sf2(b0, b1, c);   // scale bytes of blocks 2 lane, 2 lane + 1
-    const uint64_t rr0 = rtab[pair & 0xFFu], rr1 = rtab[pair >> 8];
+    const uint32_t pair = block_sf2(b0, b1, gq.c);   // scale bytes of blocks 2 lane, 2 lane + 1
+    uint64_t rr0, rr1;
+    if constexpr (GROUPED) {
+        rr0 = block_rr(pair & 0xFFu, gq.g);
+        rr1 = block_rr(pair >> 8, gq.g);
+    } else {
+        rr0 = rtab[pair & 0xFFu];
+        rr1 = rtab[pair >> 8];
+    }
     uint4 q;
     q.x = quant8(u[0], rr0);
     q.y = quant8(u[1], rr0);
@@ -546,36 +656,38 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
         *reinterpret_cast<uint4*>(dst) = q;
         if (even) *sw = word;
     } else {
-        // Rows past the tensor and values past k arrived as zeros: their scale
-        // bytes are 0, as the padded scale tile wants; no codes are stored there.
-        if (t.row < a.rows && t.seg * kTaskVals + 32 * lc.lane < a.k) *reinterpret_cast<uint4*>(dst) = q;
+        // Padding rows and values past k arrived as zeros: their scale bytes
+        // are 0, as the padded scale tile wants; no codes are stored there.
+        if (t.valid() && t.seg * kTaskVals + 32 * lc.lane < a.k) *reinterpret_cast<uint4*>(dst) = q;
         if (even && t.seg * (kTaskVals / 16) + 2 * lc.lane < a.scale_cols) *sw = word;
     }
 }
-__device__ __forceinline__ void quantize_any(const FusedArgs& a, const char* sb, const DstCursor& t,
-                                             const LaneC& lc, const BlockQ& c, const uint64_t* rtab) {
-    if (t.row < a.rows && t.seg < a.full_segs)
-        quantize_slot<true>(a, sb, t, lc, c, rtab);
+template <bool GROUPED>
+__device__ __forceinline__ void quantize_any(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
+                                             const LaneC& lc, const GroupQ& gq, const uint64_t* rtab) {
+    if (t.valid() && t.seg < a.full_segs)
+        quantize_slot<true, GROUPED>(a, sb, t, lc, gq, rtab);
     else
-        quantize_slot<false>(a, sb, t, lc, c, rtab);
+        quantize_slot<false, GROUPED>(a, sb, t, lc, gq, rtab);
 }
 
-// Grid barrier and amax reduction in one: CTA c publishes its word (part
-// + 32 c, one per 128-byte line) = gen << 16 | (its BF16 amax bits), so a reader that sees this call's
-// generation also sees the amax.  gen is one more (mod 2^16) than the
-// generation of the CTA's own word from the previous call (0 in a fresh
-// workspace), the same for every CTA.  Warp 0 of each CTA polls all G words
-// until every one carries gen; false if that wait ran out (error word set).
-__device__ __forceinline__ bool grid_amax(uint32_t* part, int G, uint32_t gen, uint64_t limit, unsigned* err,
+// Grid barrier (and, for one tensor, the amax reduction) in one: CTA c
+// publishes its word (part + kPartStrideWords c, one per 128-byte line) =
+// gen << 32 | (its BF16 amax bits; 0 in the grouped form), so a reader that
+// sees this call's generation also sees the amax.  gen is one more (mod 2^32)
+// than the generation of the CTA's own word from the previous call (0 in a
+// fresh workspace), the same for every CTA.  Warp 0 of each CTA polls all G
+// words until every one carries gen; false if that wait ran out (error word set).
+__device__ __forceinline__ bool grid_amax(const uint64_t* part, int G, uint32_t gen, uint64_t limit, unsigned* err,
                                           int lane, uint32_t& amax_bits) {
     const uint64_t t0 = globaltimer_ns();
     while (true) {
         bool mine = true;
         uint32_t mx = 0;
         for (int i = lane; i < G; i += 32) {
-            const uint32_t w = ld_relaxed_gpu_u32(part + kPartStrideWords * i);
-            mine = mine && (w >> 16) == gen;
-            mx = max(mx, w & 0xFFFFu);
+            const uint64_t w = ld_relaxed_gpu_u64(part + kPartStrideWords * i);
+            mine = mine && (uint32_t)(w >> 32) == gen;
+            mx = max(mx, (uint32_t)w & 0xFFFFu);
         }
         if (__all_sync(kFull, mine)) {
 #pragma unroll
@@ -590,6 +702,27 @@ __device__ __forceinline__ bool grid_amax(uint32_t* part, int G, uint32_t gen, u
     }
 }
 
+// Grouped form: fold a warp's amax bits m of group e into the group's word.
+// The first fold of this call (word of an older generation) replaces the
+// stale value; later ones take the max.
+__device__ __forceinline__ void fold_group_amax(uint64_t* w, uint32_t gen, uint32_t m) {
+    uint64_t old = ld_relaxed_gpu_u64(w);
+    while (true) {
+        const uint32_t cur = (uint32_t)(old >> 32) == gen ? (uint32_t)old : 0u;
+        const uint64_t nw = ((uint64_t)gen << 32) | max(cur, m);
+        if (nw == old) return;
+        const uint64_t prev = atom_cas_gpu_u64(w, old, nw);
+        if (prev == old) return;
+        old = prev;
+    }
+}
+// Grouped form: the amax bits of group e after the barrier (0 for a group no
+// row of which was seen this call, i.e. an empty group).
+__device__ __forceinline__ uint32_t group_amax(const uint64_t* w, uint32_t gen) {
+    const uint64_t v = ld_relaxed_gpu_u64(w);
+    return (uint32_t)(v >> 32) == gen ? (uint32_t)v : 0u;
+}
+
 // A warp's slot ring: slot s is kTaskBytes at base + (warp + 32 s) * kTaskBytes,
 // filled by one TMA box and completed on bar[s].
 struct Ring {
@@ -601,13 +734,15 @@ struct Ring {
     __device__ __forceinline__ char* slot(int s) const { return base + (warp + 32 * s) * kTaskBytes; }
 };
 // Lane 0 starts the copy of task t into slot s; the warp's reads of the slot's
-// previous task are done (the caller's __syncwarp).
-__device__ __forceinline__ void stage(const CUtensorMap* tmap, Ring& r, int s, const SrcCursor& t, uint64_t pol,
-                                      int lane) {
+// previous task are done (the caller's __syncwarp).  Padding rows read past
+// the tensor, where the copy fills zeros.
+template <bool GROUPED>
+__device__ __forceinline__ void stage(const CUtensorMap* tmap, const FusedArgs& a, Ring& r, int s,
+                                      const SrcCursor<GROUPED>& t, uint64_t pol, int lane) {
     if (lane == 0) {
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&r.bar[s], r.box_bytes);
-        tma_load_3d(r.slot(s), tmap, &r.bar[s], 0, t.seg * (kTaskVals / 64), t.row, pol);
+        tma_load_3d(r.slot(s), tmap, &r.bar[s], 0, t.seg * (kTaskVals / 64), t.valid() ? t.real() : a.rows, pol);
     }
 }
 // Wait (bounded) until the copy into slot s has landed.
@@ -617,11 +752,12 @@ __device__ __forceinline__ void land(Ring& r, int s, const FusedArgs& a) {
 }
 
 // Pass 1 copy: the warp starts the cp.async copy of task t into slot s.
-__device__ __forceinline__ void stage_cp(const FusedArgs& a, const Ring& r, int s, const SrcCursor& t,
+template <bool GROUPED>
+__device__ __forceinline__ void stage_cp(const FusedArgs& a, const Ring& r, int s, const SrcCursor<GROUPED>& t,
                                          const LaneC& lc, uint64_t pol) {
-    const uint16_t* p = a.x + (int64_t)t.row * a.ld + t.seg * kTaskVals + 8 * lc.lane;
+    const bool row_in = t.valid();
+    const uint16_t* p = a.x + (int64_t)(row_in ? t.real() : 0) * a.ld + t.seg * kTaskVals + 8 * lc.lane;
     const uint32_t d = smem_u32(r.slot(s));
-    const bool row_in = t.row < a.rows;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const bool in = row_in && t.seg * kTaskVals + 256 * i + 8 * lc.lane < a.k;
@@ -629,51 +765,77 @@ __device__ __forceinline__ void stage_cp(const FusedArgs& a, const Ring& r, int 
     }
 }
 
+// Per-warp state of pass 2: the constants of the group being quantized.
+template <bool GROUPED>
+struct Pass2Q {
+    GroupQ q;
+    int e = -1;
+    __device__ __forceinline__ const GroupQ& at(const FusedArgs& a, const DstCursor<GROUPED>& t, uint32_t gen) {
+        if constexpr (GROUPED) {
+            if (t.m.e != e) {   // warp-uniform
+                e = t.m.e;
+                q = make_groupq(group_amax(a.gword + e, gen));
+            }
+        }
+        return q;
+    }
+};
+
 // Pass 2 of one warp with tasks tw .. tw + n - 1, the last nres = min(kStage, n)
 // of them still on chip: task n - nres + k is in slot (n - nres + k) % kStage.
-// Quantizing it frees the slot for task k of the n - nres others, and then
-// task q of the others follows task q - kStage through the same slot.
-__device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const FusedArgs& a, Ring& r,
-                                            const uint64_t* rtab, const BlockQ& c, int tw, int n, const LaneC& lc) {
+// The nl = n - nres others come back newest first -- task nl - 1, nl - 2, ...,
+// 0 -- because pass 1 read them in increasing order, so the later ones are the
+// likeliest to be still in L2 when the tensor is larger than L2.  Quantizing
+// on-chip task k frees its slot for the k-th of those, and then the q-th
+// follows the (q - kStage)-th through the same slot.
+template <bool GROUPED>
+__device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const FusedArgs& a, const GroupTab& gt, Ring& r,
+                                            const uint64_t* rtab, Pass2Q<GROUPED>& pq, uint32_t gen, int tw, int n,
+                                            const LaneC& lc) {
     const uint64_t pol = l2_policy_evict_first();   // last use
     const int nres = n < kStage ? n : kStage;
     const int nl = n - nres;
-    DstCursor rp, lq;
-    SrcCursor lp;
-    rp.init(a, tw + n - nres);
-    lq.init(a, tw);
-    lp.init(a, tw);
+    DstCursor<GROUPED> rp, lq;
+    SrcCursor<GROUPED> lp;
+    rp.init(a, gt, tw + n - nres);
+    if (nl > 0) {
+        lq.init(a, gt, tw + nl - 1);
+        lp.init(a, gt, tw + nl - 1);
+    }
     int s = (n - nres) % kStage;
     for (int k = 0; k < nres; ++k) {
-        quantize_any(a, r.slot(s), rp, lc, c, rtab);
-        rp.next(a);
+        quantize_any<GROUPED>(a, r.slot(s), rp, lc, pq.at(a, rp, gen), rtab);
+        rp.next(a, gt);
         __syncwarp();   // every lane is done reading the slot
         if (k < nl) {
-            stage(tmap, r, s, lp, pol, lc.lane);
-            lp.next(a);
+            stage<GROUPED>(tmap, a, r, s, lp, pol, lc.lane);
+            lp.prev(a, gt);
         }
         s = (s + 1 == kStage) ? 0 : s + 1;
     }
-    // s is back at the slot of the first on-chip task, where task 0 lands.
+    // s is back at the slot of the first on-chip task, where the first refill lands.
     for (int q = 0; q < nl; ++q) {
         land(r, s, a);
-        quantize_any(a, r.slot(s), lq, lc, c, rtab);
-        lq.next(a);
+        quantize_any<GROUPED>(a, r.slot(s), lq, lc, pq.at(a, lq, gen), rtab);
+        lq.prev(a, gt);
         __syncwarp();
         if (q + kStage < nl) {
-            stage(tmap, r, s, lp, pol, lc.lane);
-            lp.next(a);
+            stage<GROUPED>(tmap, a, r, s, lp, pol, lc.lane);
+            lp.prev(a, gt);
         }
         s = (s + 1 == kStage) ? 0 : s + 1;
     }
 }
 
+template <bool GROUPED>
 __global__ void __launch_bounds__(kFThreads, 1)
     quant1d_fused_kernel(const __grid_constant__ CUtensorMap tmap, FusedArgs a, uint32_t box_bytes) {
     extern __shared__ __align__(1024) uint8_t dsm[];   // kStage task slots per warp (+ alignment pad)
     __shared__ __align__(8) uint64_t sbar[kStage * kFWarps];
     __shared__ uint64_t rtab[128];
     __shared__ uint32_t red[kFWarps];
+    __shared__ int s_off[GROUPED ? kMaxFusedGroups + 1 : 1];
+    __shared__ int s_blk[GROUPED ? kMaxFusedGroups + 1 : 1];
     __shared__ uint32_t s_amax, s_gen;
     __shared__ int s_ok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -682,12 +844,45 @@ __global__ void __launch_bounds__(kFThreads, 1)
     const int cnt = (int)((int64_t)a.tasks * (blockIdx.x + 1) / G) - t0;
     // Warp w takes a contiguous run of the CTA's tasks.
     const int tw = t0 + cnt * warp / kFWarps;
-    const int n = t0 + cnt * (warp + 1) / kFWarps - tw;
-    uint32_t gen = 0;
-    if (tid == 0) gen = ((ld_relaxed_gpu_u32(a.part + kPartStrideWords * blockIdx.x) >> 16) + 1u) & 0xFFFFu;
+    int n = t0 + cnt * (warp + 1) / kFWarps - tw;
+    if (tid == 0) s_gen = (uint32_t)(ld_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x) >> 32) + 1u;
     if (tid < kStage * kFWarps) mbar_init(&sbar[tid], 1);
+    GroupTab gt;
+    gt.off = s_off;
+    gt.blk = s_blk;
+    gt.G = a.groups;
+    if constexpr (GROUPED) {
+        // offsets and the exclusive prefix of the groups' 128-row block counts
+        // (a.groups <= kMaxFusedGroups = kFThreads)
+        const int e = tid;
+        int nb = 0;
+        if (e < a.groups) {
+            const int o0 = a.offsets[e], o1 = a.offsets[e + 1];
+            s_off[e] = o0;
+            if (e == a.groups - 1) s_off[a.groups] = o1;
+            nb = (o1 - o0 + 127) / 128;
+        }
+        int inc = nb;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFull, inc, o);
+            if (lane >= o) inc += v;
+        }
+        if (lane == 31) red[warp] = (uint32_t)inc;
+        __syncthreads();
+        int wbase = 0;
+        for (int w = 0; w < warp; ++w) wbase += (int)red[w];
+        if (e < a.groups) s_blk[e] = wbase + inc - nb;
+        if (e == a.groups - 1) s_blk[a.groups] = wbase + inc;
+    }
     fence_mbar_init();
     __syncthreads();
+    const uint32_t gen = s_gen;
+    if constexpr (GROUPED) {
+        // the exact task count: tasks past it belong to no group
+        const int real = 128 * s_blk[a.groups] * a.nseg;
+        n = max(0, min(tw + n, real) - tw);
+    }
     Ring r;
     r.base = reinterpret_cast<char*>(dsm) + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u);   // 128-byte swizzle: 1 KB aligned
     r.bar = &sbar[warp * kStage];
@@ -702,13 +897,15 @@ __global__ void __launch_bounds__(kFThreads, 1)
     {
         const uint64_t pol_keep = l2_policy_evict_normal();   // read again in pass 2
         const uint64_t pol_last = l2_policy_evict_first();    // stays on chip: not read again
-        SrcCursor sp;                                         // next task to copy
-        sp.init(a, tw);
+        SrcCursor<GROUPED> sp, lp;                            // next task to copy; next task to land
+        sp.init(a, gt, tw);
+        lp.init(a, gt, tw);
+        int cur = lp.m.e;                                     // grouped: the group acc belongs to
 #pragma unroll
         for (int i = 0; i < kStage; ++i) {
             if (i < n) {
-                stage_cp(a, r, i, sp, lc, i >= n - kStage ? pol_last : pol_keep);
-                sp.next(a);
+                stage_cp<GROUPED>(a, r, i, sp, lc, i >= n - kStage ? pol_last : pol_keep);
+                sp.next(a, gt);
             }
             cp_async_commit();
         }
@@ -718,38 +915,62 @@ __global__ void __launch_bounds__(kFThreads, 1)
         for (int i = 0; i < n; ++i) {
             cp_async_wait<kStage - 1>();
             __syncwarp();   // every lane's copies into the slot have landed
+            if constexpr (GROUPED) {
+                if (lp.m.e != cur) {   // warp-uniform: a new group starts with this task
+                    uint32_t m = absmax_bits(acc);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+                    if (lane == 0) fold_group_amax(a.gword + cur, gen, m);
+                    cur = lp.m.e;
+                    acc = 0;
+                }
+                lp.next(a, gt);
+            }
             const char* sb = r.slot(s);
 #pragma unroll
             for (int q = 0; q < 4; ++q)
                 acc = bmax_abs(acc, absmax8_packed(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q])));
             if (i + kStage < n) {
                 __syncwarp();   // every lane is done reading the slot
-                stage_cp(a, r, s, sp, lc, i + kStage >= n - kStage ? pol_last : pol_keep);
-                sp.next(a);
+                stage_cp<GROUPED>(a, r, s, sp, lc, i + kStage >= n - kStage ? pol_last : pol_keep);
+                sp.next(a, gt);
             }
             cp_async_commit();
             s = (s + 1 == kStage) ? 0 : s + 1;
         }
         cp_async_wait<0>();
         __syncwarp();
-    }
-    uint32_t m = absmax_bits(acc);
+        if constexpr (GROUPED) {
+            if (n > 0) {
+                uint32_t m = absmax_bits(acc);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
-    if (lane == 0) red[warp] = m;
+                for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+                if (lane == 0) fold_group_amax(a.gword + cur, gen, m);
+            }
+        }
+    }
+    if constexpr (!GROUPED) {
+        uint32_t m = absmax_bits(acc);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+        if (lane == 0) red[warp] = m;
+    }
     __syncthreads();
 
-    // ---- grid barrier: publish this CTA's amax, gather everyone's
+    // ---- grid barrier: publish this CTA's word, gather everyone's
     if (tid == 0) {
-        uint32_t b = red[0];
-        for (int w = 1; w < kFWarps; ++w) b = max(b, red[w]);
-        st_relaxed_gpu_u32(a.part + kPartStrideWords * blockIdx.x, (gen << 16) | b);
-        s_gen = gen;
+        uint32_t b = 0;
+        if constexpr (!GROUPED)
+            for (int w = 0; w < kFWarps; ++w) b = max(b, red[w]);
+        // grouped: every warp's folds (ordered before this by the CTA barrier)
+        // become visible with the word
+        if constexpr (GROUPED) fence_acq_rel_gpu();
+        st_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x, ((uint64_t)gen << 32) | b);
     }
-    __syncthreads();
     if (warp == 0) {
         uint32_t amax_bits = 0;
-        const bool got = grid_amax(a.part, G, s_gen, a.limit, a.err, lane, amax_bits);
+        const bool got = grid_amax(a.part, G, gen, a.limit, a.err, lane, amax_bits);
+        if constexpr (GROUPED) fence_acq_rel_gpu();   // the group words after every CTA's word
         if (lane == 0) {
             s_ok = got ? 1 : 0;
             s_amax = amax_bits;
@@ -758,13 +979,17 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __syncthreads();
     const bool ok = s_ok != 0;
     if (ok) {
-        const float amax = __uint_as_float(s_amax << 16);
-        const float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kGlobalDen);
-        if (blockIdx.x == 0 && tid == 0) a.gscale[0] = g;
-        fill_rtab(rtab, g, tid);
-        const BlockQ c = make_blockq(g);
-        __syncthreads();
-        fused_pass2(&tmap, a, r, rtab, c, tw, n, lc);
+        Pass2Q<GROUPED> pq;
+        if constexpr (GROUPED) {
+            for (int e = blockIdx.x * kFThreads + tid; e < a.groups; e += G * kFThreads)
+                a.gscale[e] = make_groupq(group_amax(a.gword + e, gen)).g;
+        } else {
+            pq.q = make_groupq(s_amax);
+            if (blockIdx.x == 0 && tid == 0) a.gscale[0] = pq.q.g;
+            fill_rtab(rtab, pq.q.g, tid);
+            __syncthreads();
+        }
+        fused_pass2<GROUPED>(&tmap, a, gt, r, rtab, pq, gen, tw, n, lc);
     }
     pdl_launch_dependents();
 }
@@ -856,14 +1081,18 @@ cudaError_t launch_pdl(const void* func, dim3 grid, dim3 block, void** args, cud
     return cudaLaunchKernelExC(&cfg, func, args);
 }
 
-// One-launch quantization of one tensor.  Returns NVFP4_ERR_UNSUPPORTED_SHAPE
-// (nothing launched) when the tensor does not fit its layout -- k % 64 != 0, or
-// codes / scales too large for 32-bit offsets -- or the device cannot hold one
-// such CTA per SM; the caller then takes the two-kernel path.
-nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes, uint8_t* scales,
-                         float* gscale, void* workspace, cudaStream_t s) {
+// One-launch quantization of one tensor, or of row groups (offsets != nullptr,
+// at most kMaxFusedGroups).  Returns NVFP4_ERR_UNSUPPORTED_SHAPE (nothing
+// launched) when the tensor does not fit its layout -- k % 64 != 0, or codes /
+// scales too large for 32-bit offsets -- or the device cannot hold one such
+// CTA per SM; the caller then takes the two-kernel path.
+nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const int32_t* offsets, int groups,
+                         uint8_t* codes, uint8_t* scales, float* gscale, void* workspace, cudaStream_t s) {
     constexpr int kSmemMax = kStage * kFWarps * kTaskBytes + 1024;
-    if (k % 64 != 0 || round_up(rows, 128) * k >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const bool grouped = offsets != nullptr;
+    if (grouped && groups > kMaxFusedGroups) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t prow = round_up(rows + (grouped ? 127 * (int64_t)groups : 0), 128);   // padded rows, at most
+    if (k % 64 != 0 || prow * k >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     static std::mutex mu;
     static int ready[64] = {};   // per device: 0 unknown, 1 usable, -1 not usable
     int dev = -1;
@@ -871,14 +1100,18 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     {
         std::lock_guard<std::mutex> lk(mu);
         if (ready[dev] == 0) {
-            int occ = 0;
+            int occ0 = 0, occ1 = 0;
             const bool ok =
                 tensor_map_encoder() != nullptr &&
-                cudaFuncSetAttribute(quant1d_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemMax) ==
-                    cudaSuccess &&
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, quant1d_fused_kernel, kFThreads, kSmemMax) ==
-                    cudaSuccess &&
-                occ >= 1;
+                cudaFuncSetAttribute(quant1d_fused_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSmemMax) == cudaSuccess &&
+                cudaFuncSetAttribute(quant1d_fused_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSmemMax) == cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ0, quant1d_fused_kernel<false>, kFThreads,
+                                                              kSmemMax) == cudaSuccess &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, quant1d_fused_kernel<true>, kFThreads,
+                                                              kSmemMax) == cudaSuccess &&
+                occ0 >= 1 && occ1 >= 1;
             ready[dev] = ok ? 1 : -1;
         }
         if (ready[dev] < 0) {
@@ -908,7 +1141,7 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     a.k = (int)k;
     a.nseg = (int)((k + kTaskVals - 1) / kTaskVals);
     a.scale_cols = (int)(k / 16);
-    a.tasks = (int)(round_up(rows, 128) * a.nseg);
+    a.tasks = (int)(prow * a.nseg);
     a.full_segs = (int)(k / kTaskVals);
     a.sc4x512 = (uint32_t)(a.scale_cols / 4) * 512u;
     // One CTA per SM, for every tensor: the grid-barrier generations live in
@@ -920,14 +1153,17 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     a.gscale = gscale;
     a.codes = codes;
     a.scales = scales;
-    a.part = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_part_off(1));
+    a.part = reinterpret_cast<uint64_t*>(workspace);
+    a.gword = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_gword_off(groups));
+    a.offsets = offsets;
+    a.groups = grouped ? groups : 1;
     a.limit = wait_limit_ns();
     a.err = device_error_word();
     if (!a.err) return NVFP4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)G);
     cfg.blockDim = dim3(kFThreads);
-    cfg.dynamicSmemBytes = (size_t)depth * kFWarps * kTaskBytes + 1024;
+    cfg.dynamicSmemBytes = (size_t)(depth > 0 ? depth : 1) * kFWarps * kTaskBytes + 1024;
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs resident at once (grid barrier)
@@ -935,7 +1171,9 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&tmap, &a, &box_bytes};
-    return cuda_status(cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(&quant1d_fused_kernel), args));
+    const void* kern = grouped ? reinterpret_cast<const void*>(&quant1d_fused_kernel<true>)
+                               : reinterpret_cast<const void*>(&quant1d_fused_kernel<false>);
+    return cuda_status(cudaLaunchKernelExC(&cfg, kern, args));
 }
 
 nvfp4_status_t run_amax(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const int32_t* offsets, int groups,
@@ -947,7 +1185,7 @@ nvfp4_status_t run_amax(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, 
     a.groups.offsets = offsets;
     a.groups.rows = (int)rows;
     a.num_groups = groups;
-    a.ws = reinterpret_cast<uint32_t*>(workspace);
+    a.ws = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_two_off());
     a.pad_rows = offsets ? reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_pad_off(groups))
                          : nullptr;
     a.gscale = gscale;
@@ -986,8 +1224,9 @@ extern "C" nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_
     if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const uint16_t* xb = reinterpret_cast<const uint16_t*>(x);
-    if (!group_offsets) {
-        const nvfp4_status_t fs = run_fused(xb, rows, k, ld, codes, scales, global_scale, workspace, s);
+    {
+        const nvfp4_status_t fs =
+            run_fused(xb, rows, k, ld, group_offsets, groups, codes, scales, global_scale, workspace, s);
         if (fs != NVFP4_ERR_UNSUPPORTED_SHAPE) return fs;
     }
     nvfp4_status_t st = run_amax(xb, rows, k, ld, group_offsets, groups, workspace, global_scale, s);
@@ -1072,7 +1311,7 @@ extern "C" nvfp4_status_t nvfp4_probe_cvt(const float* in, uint8_t* out_e2m1, ui
 namespace nvfp4 {
 namespace {
 constexpr int kStaticMaxGroups = 1024;
-constexpr int64_t kStaticScratchBytes = quant_ws_bytes(kStaticMaxGroups);   // 41216 bytes
+constexpr int64_t kStaticScratchBytes = quant_ws_bytes(kStaticMaxGroups);   // 49408 bytes
 std::mutex g_static_mu;
 void* g_static_ptr[64] = {};
 }  // namespace
@@ -1112,9 +1351,9 @@ extern "C" nvfp4_status_t nvfp4_quantize_act_static(const void* x, int64_t rows,
     void* ws = static_scratch();
     if (!ws) return NVFP4_ERR_CUDA;
     const int groups = group_offsets ? num_groups : 1;
-    // The CTA counter and the amax slots must start at zero; the array keeps
-    // whatever the previous call on this device left in it.
+    // The workspace must be as a fresh one (zeros); the array keeps whatever
+    // the previous call on this device left in it.
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (cudaMemsetAsync(ws, 0, (size_t)quant_ws_pad_off(groups), s) != cudaSuccess) return NVFP4_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, (size_t)quant_ws_bytes(groups), s) != cudaSuccess) return NVFP4_ERR_CUDA;
     return nvfp4_quantize_act(x, rows, k, ld, group_offsets, num_groups, codes, scales, global_scale, ws, stream);
 }

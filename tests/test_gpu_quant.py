@@ -187,7 +187,7 @@ def test_workspace_reusable_across_calls():
         assert st == 0
         torch.cuda.synchronize()
         nv.check_device_error()
-        assert int(ws[:16].abs().sum()) == 0
+        assert int(ws[32768:32784].abs().sum()) == 0      # the two-kernel path's counters
         assert np.array_equal(codes.cpu().numpy(), oc) and np.array_equal(scales.cpu().numpy(), osf)
         assert g.cpu().numpy()[0] == np.float32(og)
 
@@ -204,11 +204,65 @@ def _assert_same_grouped(xb, off):
     assert bad.size == 0, f"{bad.size} scale bytes differ, first at {bad[:4]}"
 
 
-def test_grouped_quantize_ragged_groups():
+@pytest.mark.parametrize("k", [2048, 960, 4160, 2064])
+def test_grouped_quantize_ragged_groups(k):
+    # k % 64 == 0: the one-launch grouped form (k < 1024: narrow tasks; 4160:
+    # a partial last task); 2064: the two-kernel form
     sizes = [0, 5, 128, 130, 0, 1, 257, 64]
     off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
-    xb = W.gaussian_bf16((int(off[-1]), 2048), 0, 43, 1.0, outlier_frac=0.01)
+    xb = W.gaussian_bf16((int(off[-1]), k), 0, 43, 1.0, outlier_frac=0.01)
     _assert_same_grouped(xb, off)
+
+
+@pytest.mark.parametrize("groups", [1024, 1100])
+def test_grouped_quantize_many_groups(groups):
+    """Up to 1024 groups take the one-launch form, more the two-kernel form;
+    group sizes 0..40 with runs of empty groups, and one all-zero group."""
+    rng = np.random.default_rng(groups)
+    sizes = rng.integers(0, 41, groups)
+    sizes[10:20] = 0
+    sizes[-3:] = 0
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    xb = W.gaussian_bf16((int(off[-1]), 128), 0, 45, 1.0, outlier_frac=0.01)
+    z = int(np.argmax(sizes > 5))
+    xb[off[z]:off[z + 1]] = 0
+    _assert_same_grouped(xb, off)
+
+
+def test_grouped_and_single_calls_share_a_workspace():
+    """Grouped and one-tensor calls alternate on one workspace (sized for the
+    groups): every result is the oracle's."""
+    import torch
+    dev = device()
+    sizes = [300, 0, 129, 256]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    rows, k = int(off[-1]), 1024
+    ws = torch.zeros(nv.nvfp4_workspace_bytes(nv.OP_QUANTIZE_ACT, rows, 0, k, len(sizes)), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream().cuda_stream
+    offd = torch.from_numpy(off).to(dev)
+    for it in range(4):
+        xb = W.gaussian_bf16((rows, k), it, 46, 1.0 + it, outlier_frac=0.01)
+        x = bf16_to_device(xb)
+        codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=dev)
+        if it % 2 == 0:
+            scales = torch.zeros(nv.nvfp4_grouped_scale_bytes(rows, len(sizes), k), dtype=torch.uint8, device=dev)
+            g = torch.empty(len(sizes), dtype=torch.float32, device=dev)
+            st = nv.nvfp4_quantize_act(x.data_ptr(), rows, k, k, offd.data_ptr(), len(sizes), codes.data_ptr(),
+                                       scales.data_ptr(), g.data_ptr(), ws.data_ptr(), stream)
+            oc, osf, og = O.quantize_1d_grouped(xb, off)
+        else:
+            scales = torch.zeros(nv.nvfp4_scale_bytes(rows, k), dtype=torch.uint8, device=dev)
+            g = torch.empty(1, dtype=torch.float32, device=dev)
+            st = nv.nvfp4_quantize_act(x.data_ptr(), rows, k, k, None, 0, codes.data_ptr(), scales.data_ptr(),
+                                       g.data_ptr(), ws.data_ptr(), stream)
+            oc, osf, og = O.quantize_1d(xb)
+        assert st == 0
+        torch.cuda.synchronize()
+        nv.check_device_error()
+        assert np.array_equal(codes.cpu().numpy(), oc)
+        assert np.array_equal(scales.cpu().numpy()[:np.asarray(osf).size], np.asarray(osf).reshape(-1))
+        assert np.array_equal(g.cpu().numpy().view(np.uint32), np.atleast_1d(np.float32(og)).view(np.uint32))
 
 
 def test_grouped_quantize_moe_workload():
