@@ -346,7 +346,7 @@ class Moe:
         self.c = [c0] + [torch.empty_like(c0) for _ in range(R - 1)]
         self.flops = 2.0 * self.rows * N * K
         self.qbytes = quant_bytes(self.rows, K, E)
-        self.launches_per_step = 3                    # per-group amax, quantize, grouped GEMM
+        self.launches_per_step = 2                    # one-launch grouped quantizer, grouped GEMM
 
     def quantize(self, i):
         j = i % self.R
