@@ -58,7 +58,6 @@ namespace nvfp4 {
 namespace {
 
 constexpr int kThreads = 320;         // 10 warps, roles above
-constexpr int kPairThreads = 448;     // pair kernel: 14 warps (8 epilogue warps, scale warps 10-13)
 constexpr uint32_t kTmemCols = 512;
 constexpr int kMaxStages = 8;
 constexpr int kMaxScaleBufs = 8;
@@ -514,7 +513,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // per tensor-memory lane quarter), 10-13 scale staging.  Tensor memory per CTA
 // (256 x 256 tiles): one 256-column accumulator and four packed scale buffers
 // of 48 columns (16 for A, 8 per k-step for B).
-template <int BN_, int STAGES_, int NSB_, int ACC_>
+template <int BN_, int STAGES_, int NSB_, int ACC_, int EPI_WARPS_ = 8>
 struct PairCfg {
     static constexpr int BN = BN_;                    // pair tile width
     static constexpr int BH = BN / 2;                 // B rows loaded per CTA
@@ -530,11 +529,16 @@ struct PairCfg {
     static constexpr uint32_t SF_COLS = 16 + 4 * NBC;
     static constexpr uint32_t SF_STRIDE = SF_COLS;     // packed buffers, written with 8-column stores
     static constexpr uint32_t SF_BASE = ACC * BN;      // accumulator buffers first
-    static constexpr int EPI_WARPS = 8;               // two per tensor-memory lane quarter
-    static constexpr uint32_t EPI_BYTES = EPI_WARPS * 2 * 2048;
+    static constexpr int EPI_WARPS = EPI_WARPS_;      // 8 or 16: two or four per tensor-memory lane quarter
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS + 4);   // producer, MMA, epilogue, scale staging
+    static constexpr int EPI_COLS = BN * 4 / EPI_WARPS;         // accumulator columns one epilogue warp drains
+    static constexpr int EPI_CP = EPI_COLS / 64;                // ... in 64-column reads
+    static constexpr int EPI_BOXES = EPI_WARPS == 8 ? 2 : 1;     // 2 KB output staging boxes per epilogue warp
+    static constexpr uint32_t EPI_BYTES = EPI_WARPS * EPI_BOXES * 2048;
     static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
     static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols, "tensor memory budget");
-    static_assert(BN % 128 == 0, "each epilogue warp of a quarter drains BN / 2 columns, 64 at a time");
+    static_assert(EPI_WARPS == 8 || EPI_WARPS == 16, "epilogue warps");
+    static_assert(EPI_COLS % 64 == 0, "each epilogue warp drains whole 64-column reads");
     static_assert(SF_BASE % 8 == 0 && SF_STRIDE % 8 == 0, "8-column stores start at a multiple of 8");
     static_assert(BN % 64 == 0 && (BN <= 192 || BN == 256),
                   "a B tile starts at row 0 or 64 of a scale block and spans <= 2 blocks");
@@ -559,14 +563,13 @@ using PairUse = PairCfg<256, 5, 4, 1>;
 // its first k-tiles [0, ke) last in its share (the "head", owner of the
 // output); pair c + 1 computes the rest [kb, num_kt) first in its own share
 // (the "continuation").  The continuation's epilogue stores its FP32
-// accumulator to a workspace slot and counts its 8 epilogue warps in a
+// accumulator to a workspace slot and counts its epilogue warps in a
 // per-CTA counter; once the head's MMAs are done, one thread of its epilogue
-// waits (bounded) for the count of 8, copies the slot into the now idle stage
+// waits (bounded) for the full count, copies the slot into the now idle stage
 // buffers with bulk copies and returns the counter to zero for the next
 // launch; the epilogue adds the copy to its own accumulator before scaling
 // and storing as usual.
 constexpr int kSkFlagStride = 16;      // uint32 words: one 64-byte line per CTA
-constexpr uint32_t kSkWarps = 8;       // epilogue warps per CTA
 
 // Calls f(std::integral_constant<int, i>) for i = 0 .. N-1 (compile-time indices).
 template <int N, int I = 0, class F>
@@ -602,10 +605,11 @@ struct PairWork {
     }
 };
 
-// Bounded wait until all epilogue warps of the continuation have counted in.
-__device__ __forceinline__ bool sk_wait_ready(const uint32_t* ready, uint64_t limit_ns, volatile int* abort_flag) {
+// Bounded wait until all `warps` epilogue warps of the continuation have counted in.
+__device__ __forceinline__ bool sk_wait_ready(const uint32_t* ready, uint32_t warps, uint64_t limit_ns,
+                                              volatile int* abort_flag) {
     const uint64_t t0 = globaltimer_ns();
-    while (ld_acquire_gpu_u32(ready) < kSkWarps) {
+    while (ld_acquire_gpu_u32(ready) < warps) {
         if (*abort_flag || globaltimer_ns() - t0 > limit_ns) return false;
         __nanosleep(128);
     }
@@ -687,7 +691,7 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& p, const TAIL* tai
 }
 
 template <class P, bool GROUPED>
-__global__ void __launch_bounds__(kPairThreads, 1)
+__global__ void __launch_bounds__(P::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
     constexpr int BN = P::BN, BH = P::BH, STAGES = P::STAGES, NBC = P::NBC;
@@ -949,10 +953,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // MMAs wait only for the reads (measured on the prefill shape: 4 warps
         // 143 us, 8 warps 139 us, 8 warps reading 64 columns at a time 135 us,
         // converting all of them before the stores 133 us; 16 warps were slower).
+        constexpr int NCP = P::EPI_CP;
         const int q = warp & 3;
-        const int half = (warp - 2) >> 2;
-        const int c0 = half * (BN / 64);
-        const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * 4096u;
+        const int c0 = ((warp - 2) >> 2) * (2 * NCP);      // first 32-column chunk of this warp
+        const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * (P::EPI_BOXES * 2048u);
         const uint32_t empty0 = mapa_shared(smem_u32(&tail->acc_empty[0]), 0);
         const uint32_t empty_step = (uint32_t)sizeof(uint64_t);
         int it = 0;
@@ -969,7 +973,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 // buffers are free, so one bulk copy brings the next pair's partial
                 // sums (128 x BN FP32) on chip while the accumulator is read.
                 if (warp == 2 && lane == 0) {
-                    wait_ok = sk_wait_ready(p.sk_flags + slot_idx * kSkFlagStride, limit, &tail->abort_flag);
+                    wait_ok = sk_wait_ready(p.sk_flags + slot_idx * kSkFlagStride, (uint32_t)P::EPI_WARPS, limit,
+                                            &tail->abort_flag);
                     if (wait_ok) {
                         fence_proxy_async_global();
                         constexpr uint32_t kPart = 128u * BN * 4u, kPiece = 16384u;
@@ -1021,8 +1026,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     }
                     return;
                 }
-                const uint32_t box = stg + (uint32_t)(ch & 1) * 2048u;
-                if (lane == 0) bulk_wait_group_read<1>();
+                const uint32_t box = stg + (P::EPI_BOXES == 2 ? (uint32_t)(ch & 1) * 2048u : 0u);
+                if (lane == 0) {
+                    if constexpr (P::EPI_BOXES == 2) bulk_wait_group_read<1>(); else bulk_wait_group_read<0>();
+                }
                 __syncwarp();
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
@@ -1042,12 +1049,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 // pieces), then one count per warp.
                 float4* slot = reinterpret_cast<float4*>(p.partial + (size_t)slot_idx * (128 * BN)) + q * 32 + lane;
 #pragma unroll
-                for (int cp = 0; cp < BN / 128; ++cp) {
+                for (int cp = 0; cp < NCP; ++cp) {
                     uint32_t va0[32], va1[32];
                     tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
                     tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
                     tmem_ld_wait();
-                    if (cp == BN / 128 - 1) {
+                    if (cp == NCP - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
@@ -1071,12 +1078,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 // buffers, same layout) before scaling.
                 const uint32_t slot_s = smem_u32(smem) + (uint32_t)(q * 32 + lane) * 16u;
 #pragma unroll
-                for (int cp = 0; cp < BN / 128; ++cp) {
+                for (int cp = 0; cp < NCP; ++cp) {
                     uint32_t va0[32], va1[32];
                     tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
                     tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
                     tmem_ld_wait();
-                    if (cp == BN / 128 - 1) {
+                    if (cp == NCP - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
@@ -1111,14 +1118,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             // Whole tile: read the warp's BN / 2 columns 64 at a time and
             // convert them to BF16 in registers; release the accumulator after
             // the last read, then stage and store.
-            uint32_t bf[BN / 4];
+            uint32_t bf[NCP * 32];
 #pragma unroll
-            for (int cp = 0; cp < BN / 128; ++cp) {
+            for (int cp = 0; cp < NCP; ++cp) {
                 uint32_t va0[32], va1[32];
                 tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
                 tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
                 tmem_ld_wait();
-                if (cp == BN / 128 - 1) {
+                if (cp == NCP - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
@@ -1132,7 +1139,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                 }
             }
 #pragma unroll
-            for (int h = 0; h < BN / 64; ++h) store_chunk(c0 + h, bf + h * 16);
+            for (int h = 0; h < 2 * NCP; ++h) store_chunk(c0 + h, bf + h * 16);
         }
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
@@ -1196,7 +1203,7 @@ template <bool GROUPED>
 cudaLaunchConfig_t pair_config(int clusters, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * clusters);
-    cfg.blockDim = dim3(kPairThreads);
+    cfg.blockDim = dim3(PairUse::THREADS);
     cfg.dynamicSmemBytes = kPairSmem<GROUPED>;
     cfg.stream = s;
     attr[0].id = cudaLaunchAttributeClusterDimension;
