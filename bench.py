@@ -244,6 +244,25 @@ class Prefill:
     def result(self, i):
         return self.c[i % self.R]
 
+    def next_layer_steps(self, nv, torch):
+        """The next layer's dynamic quantization of this GEMM's output C, two
+        ways, over the same rotating sets: the GEMM then the one-launch
+        quantizer (amax and quantize passes over C), or the GEMM emitting C's
+        global scale then the quantize pass alone."""
+        qc = [nv.quantize_act(c) for c in self.c]
+        gs = [torch.empty(1, dtype=torch.float32, device=c.device) for c in self.c]
+
+        def one_phase(i):
+            j = i % self.R
+            self.nv.gemm(self.qa[j], self.w[j], out=self.c[j])
+            self.nv.quantize_act(self.c[j], out=qc[j])
+
+        def two_phase(i):
+            j = i % self.R
+            self.nv.gemm_emit_scale(self.qa[j], self.w[j], out=self.c[j], out_scale=gs[j])
+            self.nv.quantize_act_scaled(self.c[j], gs[j], out=qc[j])
+        return one_phase, two_phase
+
     def gemm_label(self):
         if self.m <= 64:
             return "gemm_kernel (tcgen05 mxf4nvf4; 64 token rows x 192 weight rows per tile)"
@@ -685,6 +704,17 @@ def run_ours(args):
         line["weight_quantize"] = {"workload": f"bf16 [{wl.wn},{wl.k}] N(0,0.02) -> nvfp4, 16x16 blocks",
                                    "gbs": w_gbs, "frac_hbm": w_gbs / peaks["hbm_gbs"], "avg_ms": w_avg * 1e3,
                                    "algorithmic_bytes": wl.wqbytes, "kernels": "amax_kernel + quant2d_kernel"}
+    if type(wl) is Prefill:
+        one_phase, two_phase = wl.next_layer_steps(nv, torch)
+        time.sleep(REST_S)
+        t1 = graph_seconds(torch, cs, one_phase, wl.R, kiters)
+        time.sleep(REST_S)
+        t2 = graph_seconds(torch, cs, two_phase, wl.R, kiters)
+        line["next_layer_quant"] = {
+            "what": "GEMM + dynamic quantization of its BF16 output C [m, n] for the next layer",
+            "one_phase_ms": t1 * 1e3, "two_phase_ms": t2 * 1e3, "gemm_alone_ms": g_avg * 1e3,
+            "note": "one phase: GEMM, then the one-launch quantizer (amax pass + quantize pass over C); two phase: "
+                    "GEMM emitting C's global scale from its epilogue, then the quantize pass alone"}
     if isinstance(wl, Decode):
         line["weight_stream"] = {"gbs": wl.wbytes / g_avg / 1e9, "frac_hbm": wl.wbytes / g_avg / 1e9 / peaks["hbm_gbs"],
                                  "bytes": wl.wbytes}

@@ -92,7 +92,7 @@ size_t nvfp4_grouped_scale_bytes(int64_t total_rows, int num_groups, int64_t k);
 
 /* Workspace bytes an operation needs (operations below); 0 if none. */
 enum { NVFP4_OP_QUANTIZE_ACT = 0, NVFP4_OP_QUANTIZE_WEIGHT_2D = 1, NVFP4_OP_GEMM = 2,
-       NVFP4_OP_GROUPED_GEMM = 3 };
+       NVFP4_OP_GROUPED_GEMM = 3, NVFP4_OP_GEMM_EMIT_SCALE = 4 };
 size_t nvfp4_workspace_bytes(int op, int64_t rows, int64_t n, int64_t k, int num_groups);
 
 /* Zero a workspace before its first use (cudaMemsetAsync on stream). */
@@ -135,6 +135,20 @@ nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_
                                   const int32_t* group_offsets, int num_groups,
                                   uint8_t* codes, uint8_t* scales, float* global_scale,
                                   void* workspace, void* stream);
+
+/* nvfp4_quantize_act_scaled -- the quantize pass of nvfp4_quantize_act with
+ * the global scale given (one tensor): codes and scales exactly as
+ * nvfp4_quantize_act would write them if the tensor's amax were
+ * global_scale[0] * 2688.  With the scale from nvfp4_gemm_emit_scale on the
+ * GEMM's own output, the result equals nvfp4_quantize_act of that output,
+ * for one read of it instead of two.
+ *   x, rows, k, ld, codes, scales: as nvfp4_quantize_act (one tensor).
+ *   global_scale: device FP32 [1], > 0 and finite; read, not written.
+ * One launch; no workspace.  The launch waits for the previous work on
+ * stream (it may be the kernel that wrote x). */
+nvfp4_status_t nvfp4_quantize_act_scaled(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                         const float* global_scale, uint8_t* codes, uint8_t* scales,
+                                         void* stream);
 
 /* nvfp4_quantize_act_static -- nvfp4_quantize_act without the workspace
  * argument: this entry point allocates nothing and takes no scratch from the
@@ -186,7 +200,8 @@ nvfp4_status_t nvfp4_quantize_weight_2d(const void* w, int64_t n, int64_t k, int
  *   a_codes, a_scales, a_global: device; output of nvfp4_quantize_act on [m, k].
  *   b_codes, b_scales, b_global: device; output of either quantizer on [n, k].
  *   c: device BF16 [m, n], row stride ldc elements (ldc >= n, ldc % 8 == 0).
- *   m >= 0, n > 0, k > 0, k % 64 == 0.
+ *   m >= 0, n > 0, k > 0, k % 64 == 0.  m == 0 reads and writes nothing (the
+ *   operand pointers may then be NULL).
  *   workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, 0) bytes, 16-byte
  *   aligned, zeroed before first use (see above); NULL is allowed.  For m > 128
  *   the kernel runs on pairs of SMs with 256 x 256 output tiles; when the tiles
@@ -203,6 +218,25 @@ nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
                           const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
                           void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
                           void* workspace, void* stream);
+
+/* nvfp4_gemm_emit_scale -- nvfp4_gemm that also takes the amax of its BF16
+ * output in the epilogue and writes the global scale the next layer's
+ * dynamic quantizer needs: c_global_scale[0] = max|C| / (6 * 448), or 1 when
+ * C is all zeros (C as stored, after BF16 rounding).  With
+ * nvfp4_quantize_act_scaled it splits dynamic activation quantization into
+ * its two passes so that the amax pass costs no read of C: the output-side
+ * fusion of the pages' W4A4 pipeline ("NVFP4 Dynamic Quantization in
+ * Practice"; the dequantization / extra-pass overhead of "W4A8 vs NVFP4
+ * quantization on GPUs").
+ *   Arguments as nvfp4_gemm, plus c_global_scale: device FP32 [1].
+ *   workspace: nvfp4_workspace_bytes(NVFP4_OP_GEMM_EMIT_SCALE, m, n, k, 0)
+ *   bytes, 16-byte aligned, zeroed before first use; required (not NULL).
+ *   The first 256 bytes hold a running maximum and a CTA count that every
+ *   call returns to zero; the rest serves as nvfp4_gemm's workspace. */
+nvfp4_status_t nvfp4_gemm_emit_scale(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                                     const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
+                                     void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
+                                     float* c_global_scale, void* workspace, void* stream);
 
 /* nvfp4_grouped_gemm -- one GEMM per expert over row groups (mixture of
  * experts: "NVFP4 Dynamic Quantization in Practice", "The Practical

@@ -23,17 +23,18 @@ __all__ = [
     "lib", "Nvfp4Error", "NVFP4Tensor",
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_grouped_scale_bytes", "nvfp4_workspace_bytes",
     "nvfp4_workspace_init", "nvfp4_quantize_act", "nvfp4_quantize_act_static", "nvfp4_quantize_weight_2d",
-    "nvfp4_gemm",
+    "nvfp4_gemm", "nvfp4_gemm_emit_scale", "nvfp4_quantize_act_scaled",
     "nvfp4_grouped_gemm", "nvfp4_get_last_device_error", "nvfp4_set_wait_limit_ns", "nvfp4_probe_cvt",
     "nvfp4_probe_bounded_wait", "nvfp4_status_string", "nvfp4_version",
     "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
-    "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM",
+    "gemm_emit_scale", "quantize_act_scaled",
+    "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM", "OP_GEMM_EMIT_SCALE",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libnvfp4.so")
 
-OP_QUANTIZE_ACT, OP_QUANTIZE_WEIGHT_2D, OP_GEMM, OP_GROUPED_GEMM = 0, 1, 2, 3
+OP_QUANTIZE_ACT, OP_QUANTIZE_WEIGHT_2D, OP_GEMM, OP_GROUPED_GEMM, OP_GEMM_EMIT_SCALE = 0, 1, 2, 3, 4
 STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
           5: "TIMEOUT", 6: "NO_DEVICE"}
 
@@ -60,6 +61,8 @@ _SIGNATURES = {
     "nvfp4_quantize_act_static": (_i32, [_vp, _i64, _i64, _i64, _vp, _i32, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_weight_2d": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
+    "nvfp4_gemm_emit_scale": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "nvfp4_quantize_act_scaled": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_get_last_device_error": (_i32, [_vp]),
     "nvfp4_set_wait_limit_ns": (_u64, [_u64]),
@@ -156,6 +159,16 @@ def nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc,
                stream=0) -> int:
     return lib().nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
                             workspace, stream)
+
+
+def nvfp4_gemm_emit_scale(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
+                          c_global_scale, workspace, stream=0) -> int:
+    return lib().nvfp4_gemm_emit_scale(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
+                                       c_global_scale, workspace, stream)
+
+
+def nvfp4_quantize_act_scaled(x, rows, k, ld, global_scale, codes, scales, stream=0) -> int:
+    return lib().nvfp4_quantize_act_scaled(x, rows, k, ld, global_scale, codes, scales, stream)
 
 
 def nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_codes, b_scales, b_global, c, n, k,
@@ -300,6 +313,55 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out=None):
                     _ptr(b.global_scale), _ptr(c), c.stride(0), a.rows, b.rows, a.k, _ptr(ws), _stream_ptr(torch, dev))
     _check(st, "nvfp4_gemm")
     return c
+
+
+def gemm_emit_scale(a: NVFP4Tensor, b: NVFP4Tensor, out=None, out_scale=None):
+    """gemm() that also returns the global scale of its BF16 output for the
+    next dynamic quantizer: (C, g) with g = max|C| / 2688 (1 for an all-zero
+    C), a device FP32 [1] tensor."""
+    import torch
+    if a.k != b.k:
+        raise ValueError("k mismatch")
+    dev = a.codes.device
+    c = out if out is not None else torch.empty((a.rows, b.rows), dtype=torch.bfloat16, device=dev)
+    g = out_scale if out_scale is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    nbytes = nvfp4_workspace_bytes(OP_GEMM_EMIT_SCALE, a.rows, b.rows, a.k, 0)
+    key = (dev.index, OP_GEMM_EMIT_SCALE, 0, torch.cuda.current_stream(dev).cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    st = nvfp4_gemm_emit_scale(_ptr(a.codes), _ptr(a.scales), _ptr(a.global_scale), _ptr(b.codes), _ptr(b.scales),
+                               _ptr(b.global_scale), _ptr(c), c.stride(0), a.rows, b.rows, a.k, _ptr(g), _ptr(ws),
+                               _stream_ptr(torch, dev))
+    _check(st, "nvfp4_gemm_emit_scale")
+    return c, g
+
+
+def quantize_act_scaled(x, global_scale, out: Optional[NVFP4Tensor] = None) -> NVFP4Tensor:
+    """The quantize pass alone, with a given device FP32 [1] global scale (from
+    gemm_emit_scale on the GEMM that produced x)."""
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along k")
+    rows, k = x.shape
+    dev = x.device
+    if out is not None:
+        if out.rows != rows or out.k != k or out.scales.numel() < nvfp4_scale_bytes(rows, k) or out.offsets is not None:
+            raise ValueError("out does not match the input shape")
+        codes, scales = out.codes, out.scales
+    else:
+        codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty(nvfp4_scale_bytes(rows, k), dtype=torch.uint8, device=dev)
+    st = nvfp4_quantize_act_scaled(_ptr(x), rows, k, x.stride(0), _ptr(global_scale), _ptr(codes), _ptr(scales),
+                                   _stream_ptr(torch, dev))
+    _check(st, "nvfp4_quantize_act_scaled")
+    if out is not None:
+        out.global_scale = global_scale
+        return out
+    return NVFP4Tensor(codes, scales, global_scale, rows, k)
 
 
 def grouped_gemm(a: NVFP4Tensor, b_codes, b_scales, b_global, n: int, out=None):

@@ -117,6 +117,7 @@ extern "C" size_t nvfp4_workspace_bytes(int op, int64_t rows, int64_t n, int64_t
         case NVFP4_OP_QUANTIZE_ACT: return (size_t)quant_ws_bytes(num_groups > 1 ? num_groups : 1);
         case NVFP4_OP_QUANTIZE_WEIGHT_2D: return (size_t)quant_ws_bytes(1);
         case NVFP4_OP_GEMM: return gemm_workspace_bytes(rows, n, k);
+        case NVFP4_OP_GEMM_EMIT_SCALE: return (size_t)kEmitScaleWsBytes + gemm_workspace_bytes(rows, n, k);
         case NVFP4_OP_GROUPED_GEMM: return 0;
     }
     return 0;

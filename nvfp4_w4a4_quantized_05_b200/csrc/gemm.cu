@@ -90,7 +90,34 @@ struct GemmArgs {
     int64_t sk_units;
     float* partial;            // per CTA of each pair: FP32 [BN / 4][128] x 4 partial sums
     uint32_t* sk_flags;        // per CTA of each pair: a ready counter, kSkFlagStride words apart
+    // optional: the amax of the BF16 output, as the next quantizer's global scale
+    uint32_t* c_amax;          // [0] running max |C| (BF16 bits), [1] CTAs done; both 0 between calls
+    float* c_gscale;           // receives amax(C) / 2688 (1 when amax is 0)
 };
+
+// The largest |value| of packed BF16 pairs, as a 16-bit pattern.
+__device__ __forceinline__ uint32_t bf16x2_abs_bits(uint32_t packed) {
+    const uint32_t m = packed & 0x7FFF7FFFu;
+    return max(m & 0xFFFFu, m >> 16);
+}
+// An epilogue warp's running output maximum (packed), folded into the call's word.
+__device__ __forceinline__ void fold_c_amax(const GemmArgs& p, uint32_t cam) {
+    uint32_t m = bf16x2_abs_bits(cam);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if ((threadIdx.x & 31) == 0 && m != 0u) atomicMax(&p.c_amax[0], m);
+}
+// Thread 0 of every CTA, after all its epilogue warps have folded: the last
+// CTA turns the maximum into the global scale and returns both words to zero.
+__device__ __forceinline__ void finish_c_amax(const GemmArgs& p) {
+    __threadfence();
+    if (atomicAdd(&p.c_amax[1], 1u) == gridDim.x - 1) {
+        __threadfence();
+        const float amax = __uint_as_float(atomicExch(&p.c_amax[0], 0u) << 16);
+        p.c_gscale[0] = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);   // 6 x 448, as the quantizer
+        atomicExch(&p.c_amax[1], 0u);
+    }
+}
 
 struct alignas(8) SmemTail {
     uint64_t full[kMaxStages];
@@ -194,7 +221,8 @@ struct Cfg {
     static_assert(SF_COLS == 32 || SF_COLS == 48, "scale staging writes 32 (+16) columns per k-tile");
 };
 
-template <class C, bool GROUPED>
+// EMIT (plain form only): also fold max |C| and write C's global scale.
+template <class C, bool GROUPED, bool EMIT = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
@@ -429,6 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;                       // tensor-memory lane quarter of this warp
         const int rloc = q * 32 + lane;               // A-side row inside the tile
         const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * 4096u;
+        uint32_t cam = 0;                             // running max |C| of this lane's rows (packed)
         int it = 0;
         for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++it) {
             const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
@@ -464,6 +493,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                         w.y = pack_bf16x2(__uint_as_float(v[8 * j + 2]) * alpha, __uint_as_float(v[8 * j + 3]) * alpha);
                         w.z = pack_bf16x2(__uint_as_float(v[8 * j + 4]) * alpha, __uint_as_float(v[8 * j + 5]) * alpha);
                         w.w = pack_bf16x2(__uint_as_float(v[8 * j + 6]) * alpha, __uint_as_float(v[8 * j + 7]) * alpha);
+                        if (EMIT && a_ok)
+                            cam = max_abs_bf16x2(max_abs_bf16x2(cam, max_abs_bf16x2(w.x, w.y)), max_abs_bf16x2(w.z, w.w));
                         // 64-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ ((r >> 1) & 3)
                         st_shared_v4(box + (uint32_t)lane * 64u + (uint32_t)((j ^ ((lane >> 1) & 3)) * 16), w);
                     }
@@ -485,12 +516,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0) mbar_arrive(&tail->acc_empty[ab]);
         }
+        if (EMIT) fold_c_amax(p, cam);
         if (lane == 0) bulk_wait_group_all();   // stores done before the CTA's shared memory goes away
         __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
+    if (EMIT && threadIdx.x == 0) finish_c_amax(p);
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
@@ -690,7 +723,7 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& p, const TAIL* tai
     return pt;
 }
 
-template <class P, bool GROUPED>
+template <class P, bool GROUPED, bool EMIT = false>
 __global__ void __launch_bounds__(P::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
@@ -959,6 +992,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * (P::EPI_BOXES * 2048u);
         const uint32_t empty0 = mapa_shared(smem_u32(&tail->acc_empty[0]), 0);
         const uint32_t empty_step = (uint32_t)sizeof(uint64_t);
+        uint32_t cam = 0;                             // running max |C| of this lane's rows (packed)
         int it = 0;
         PairWork w;
         for (; w.next(p, cluster, dp_tiles); ++it) {
@@ -1025,6 +1059,10 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                         }
                     }
                     return;
+                }
+                if (EMIT && q * 32 + lane < a_rows) {   // the output maximum, chunk by chunk
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) cam = max_abs_bf16x2(cam, w16[j]);
                 }
                 const uint32_t box = stg + (P::EPI_BOXES == 2 ? (uint32_t)(ch & 1) * 2048u : 0u);
                 if (lane == 0) {
@@ -1141,12 +1179,14 @@ __global__ void __launch_bounds__(P::THREADS, 1)
 #pragma unroll
             for (int h = 0; h < 2 * NCP; ++h) store_chunk(c0 + h, bf + h * 16);
         }
+        if (EMIT) fold_c_amax(p, cam);
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
     }
 
     tc_fence_before();
     __syncthreads();
+    if (EMIT && threadIdx.x == 0) finish_c_amax(p);
     cluster_sync();          // no CTA leaves while its peer may still touch its shared memory
     if (warp == 1) {
         tc_fence_after();
@@ -1171,10 +1211,10 @@ bool make_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <class C, bool GROUPED>
+template <class C, bool GROUPED, bool EMIT = false>
 nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                       int grid, cudaStream_t s) {
-    auto kern = gemm_kernel<C, GROUPED>;
+    auto kern = gemm_kernel<C, GROUPED, EMIT>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -1277,12 +1317,19 @@ size_t sk_workspace_bytes(int clusters) {
     return kSkFlagsBytes + (size_t)clusters * 2 * 128 * PairUse::BN * sizeof(float);
 }
 
-template <bool GROUPED = false>
+template <bool GROUPED = false, bool EMIT = false>
 nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                            int clusters, cudaStream_t s) {
+    auto kern = gemm_pair_kernel<PairUse, GROUPED, EMIT>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [&] {
+        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem<GROUPED>);
+    });
+    if (attr_err != cudaSuccess) return NVFP4_ERR_CUDA;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pair_config<GROUPED>(clusters, s, attr);
-    return cuda_status(cudaLaunchKernelEx(&cfg, gemm_pair_kernel<PairUse, GROUPED>, ta, tb, tc, args));
+    return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args));
 }
 
 // Kernel configurations: 64 < m <= 128 and the grouped form use 128 x 192
@@ -1326,24 +1373,39 @@ size_t gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
 
 using namespace nvfp4;
 
-extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
-                                     const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c,
-                                     int64_t ldc, int64_t m, int64_t n, int64_t k, void* workspace, void* stream) {
+namespace nvfp4 {
+namespace {
+__global__ void set_one_kernel(float* g) { g[0] = 1.0f; }
+
+// The dense GEMM.  c_amax / c_gscale (optional): also fold max |C| and write
+// the global scale of C for the next quantizer (see nvfp4_gemm_emit_scale).
+nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                         const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c, int64_t ldc,
+                         int64_t m, int64_t n, int64_t k, void* workspace, uint32_t* c_amax, float* c_gscale,
+                         void* stream) {
     if (m < 0 || n <= 0 || k <= 0 || ldc < n) return NVFP4_ERR_INVALID_ARGUMENT;
-    if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !c)
-        return NVFP4_ERR_INVALID_ARGUMENT;
     if (k % 64 != 0 || m >= ((int64_t)1 << 31) || n >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (m == 0) {   // nothing to read or write (the operand pointers may be NULL)
+        if (c_gscale) {   // an empty C: amax 0, global scale 1
+            set_one_kernel<<<1, 1, 0, s>>>(c_gscale);
+            return cuda_status(cudaGetLastError());
+        }
+        return NVFP4_OK;
+    }
+    if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !c)
+        return NVFP4_ERR_INVALID_ARGUMENT;
     if (!ptr_ok(a_codes) || !ptr_ok(a_scales) || !ptr_ok(b_codes) || !ptr_ok(b_scales) || !ptr_ok(c) ||
         (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(b_global) & 3u) || ldc % 8 != 0)
         return NVFP4_ERR_MISALIGNED;
     if (reinterpret_cast<uintptr_t>(workspace) & 15u) return NVFP4_ERR_MISALIGNED;
-    if (m == 0) return NVFP4_OK;
     const int sms = num_sms();
     if (sms <= 0) return NVFP4_ERR_NO_DEVICE;
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int64_t sf_rb_stride = 128 * (k / 16);
     GemmArgs p = {};
+    p.c_amax = c_amax;
+    p.c_gscale = c_gscale;
     p.num_ks = (int)(k / 64);
     p.num_kt = (p.num_ks + 3) / 4;
     p.c = reinterpret_cast<__nv_bfloat16*>(c);
@@ -1371,7 +1433,7 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         p.tiles_m = 1;
         p.tiles_n = (int)((n + CfgDecW::BN - 1) / CfgDecW::BN);
         const int grid = (int)std::min<int64_t>((int64_t)p.tiles_n, sms);
-        return launch<CfgDecW, false>(ta, tb, tc, p, grid, s);
+        return c_amax ? launch<CfgDecW, false, true>(ta, tb, tc, p, grid, s) : launch<CfgDecW, false>(ta, tb, tc, p, grid, s);
     }
     PairPlan pl;
     if (pair_plan(m, n, k, pl)) {
@@ -1394,7 +1456,8 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
         p.sk_units = sk ? pl.sk_units : 0;
         p.sk_flags = sk ? reinterpret_cast<uint32_t*>(workspace) : nullptr;
         p.partial = sk ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + kSkFlagsBytes) : nullptr;
-        return launch_pair(ta, tb, tc, p, pl.clusters, s);
+        return c_amax ? launch_pair<false, true>(ta, tb, tc, p, pl.clusters, s)
+                      : launch_pair<false>(ta, tb, tc, p, pl.clusters, s);
     }
     constexpr int BN = CfgWide::BN;
     if (!make_codes_map(&ta, a_codes, m, k / 2, 128) || !make_codes_map(&tb, b_codes, n, k / 2, BN) ||
@@ -1412,7 +1475,29 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int grid = (int)std::min<int64_t>(tiles, sms);
-    return launch<CfgWide, false>(ta, tb, tc, p, grid, s);
+    return c_amax ? launch<CfgWide, false, true>(ta, tb, tc, p, grid, s) : launch<CfgWide, false>(ta, tb, tc, p, grid, s);
+}
+}  // namespace
+}  // namespace nvfp4
+
+extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
+                                     const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c,
+                                     int64_t ldc, int64_t m, int64_t n, int64_t k, void* workspace, void* stream) {
+    return gemm_impl(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k, workspace, nullptr,
+                     nullptr, stream);
+}
+
+extern "C" nvfp4_status_t nvfp4_gemm_emit_scale(const uint8_t* a_codes, const uint8_t* a_scales,
+                                                const float* a_global, const uint8_t* b_codes,
+                                                const uint8_t* b_scales, const float* b_global, void* c, int64_t ldc,
+                                                int64_t m, int64_t n, int64_t k, float* c_global_scale,
+                                                void* workspace, void* stream) {
+    if (!c_global_scale || !workspace) return NVFP4_ERR_INVALID_ARGUMENT;
+    if ((reinterpret_cast<uintptr_t>(c_global_scale) & 3u) || (reinterpret_cast<uintptr_t>(workspace) & 15u))
+        return NVFP4_ERR_MISALIGNED;
+    uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+    return gemm_impl(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
+                     ws + kEmitScaleWsBytes, reinterpret_cast<uint32_t*>(ws), c_global_scale, stream);
 }
 
 extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,

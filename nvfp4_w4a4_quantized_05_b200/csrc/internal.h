@@ -22,6 +22,9 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 // Scratch bytes nvfp4_gemm wants for an m x n x k product on the current
 // device (the stream-K tail of the pair kernel); 0 when it needs none.
 size_t gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
+// nvfp4_gemm_emit_scale's workspace: its output-amax words first, then the
+// plain GEMM's workspace.
+constexpr int64_t kEmitScaleWsBytes = 256;
 
 // Current limit of the bounded waits, in ns.
 uint64_t wait_limit_ns();

@@ -1299,6 +1299,42 @@ extern "C" nvfp4_status_t nvfp4_probe_cvt(const float* in, uint8_t* out_e2m1, ui
     return cuda_status(cudaGetLastError());
 }
 
+extern "C" nvfp4_status_t nvfp4_quantize_act_scaled(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                                    const float* global_scale, uint8_t* codes, uint8_t* scales,
+                                                    void* stream) {
+    if (rows < 0 || k <= 0 || ld < k) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (!x || !codes || !scales || !global_scale) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t nseg = (k + 511) / 512;
+    if (rows * (k / 8) >= (int64_t)1 << 40 || round_up(rows, 128) * nseg >= ((int64_t)1 << 31) ||
+        rows >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u) || ld % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
+    if (rows == 0) return NVFP4_OK;
+    Quant1dArgs q;
+    q.x = reinterpret_cast<const uint16_t*>(x);
+    q.ld = ld;
+    q.k = (int)k;
+    q.nseg = (int)nseg;
+    q.scale_cols = (int)(round_up(k / 16, 4));
+    q.groups.offsets = nullptr;
+    q.groups.rows = (int)rows;
+    q.pad_rows = nullptr;
+    q.gscale = global_scale;
+    q.codes = codes;
+    q.scales = scales;
+    const int64_t tasks = round_up(rows, 128) * q.nseg;
+    const int qx = clamp_grid((tasks + kWarps * kQuantUnroll - 1) / (kWarps * kQuantUnroll), (int64_t)num_sms() * 4);
+    // A plain launch: x may come from the previous kernel on the stream, whose
+    // end this kernel must not overlap (its first loads precede its
+    // griddepcontrol.wait, which returns at once without the launch attribute).
+    quant1d_kernel<<<dim3(qx, 1), kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(q);
+    return cuda_status(cudaGetLastError());
+}
+
 // ---- quantization without a caller-provided workspace --------------------------------
 //
 // Some callers cannot allocate device memory at the point where they quantize:

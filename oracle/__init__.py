@@ -50,6 +50,7 @@ def lib():
             "orc_sf_offset": (_i64, [_i64, _i64, _i64]),
             "orc_global_scale": (ctypes.c_float, [ctypes.c_float]),
             "orc_quantize_1d": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _u8p, _u8p, _f32p]),
+            "orc_quantize_1d_given_g": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_float, _u8p, _u8p]),
             "orc_grouped_scale_rows": (_i64, [_i32p, ctypes.c_int]),
             "orc_quantize_1d_grouped": (ctypes.c_int, [_u16p, _i32p, ctypes.c_int, _i64, _i64,
                                                        _u8p, _u8p, _f32p]),
@@ -145,6 +146,19 @@ def quantize_1d(x_bf16: np.ndarray):
     if rc != 0:
         raise ValueError(f"orc_quantize_1d failed ({rc})")
     return codes, sf, float(g[0])
+
+
+def quantize_1d_given_g(x_bf16: np.ndarray, g: float):
+    """1D quantization with the global scale g given (the two-phase form's
+    second pass): steps 3-8 of the block quantizer with g from the caller."""
+    x = _bf16(x_bf16)
+    rows, k = x.shape
+    codes = np.zeros((rows, k // 2), np.uint8)
+    sf = np.zeros(scale_rows(rows) * scale_cols(k), np.uint8)
+    rc = lib().orc_quantize_1d_given_g(x, rows, k, k, float(np.float32(g)), codes, sf)
+    if rc != 0:
+        raise ValueError(f"orc_quantize_1d_given_g failed ({rc})")
+    return codes, sf
 
 
 def grouped_scale_rows(offsets: np.ndarray) -> int:

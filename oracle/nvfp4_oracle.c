@@ -202,6 +202,18 @@ int64_t orc_grouped_scale_rows(const int32_t* off, int num_groups) {
     return t;
 }
 
+/* The same block quantizer with the global scale g given by the caller: the
+   second pass of a two-phase form whose amax was taken elsewhere (by the GEMM
+   that produced x).  g must be positive and finite. */
+int orc_quantize_1d_given_g(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, float g,
+                            uint8_t* codes, uint8_t* sf) {
+    if (rows < 0 || k <= 0 || k % 16 != 0 || ld < k || !(g > 0.0f) || !isfinite(g)) return 1;
+    if (check_finite_rows(x, 0, rows, k, ld)) return 2;
+    memset(sf, 0, (size_t)(orc_scale_rows(rows) * orc_scale_cols(k)));
+    quantize_rows_1d(x, 0, rows, k, ld, g, codes, sf, 0);
+    return 0;
+}
+
 int orc_quantize_1d_grouped(const uint16_t* x, const int32_t* off, int num_groups,
                             int64_t k, int64_t ld, uint8_t* codes, uint8_t* sf,
                             float* g_out) {

@@ -72,6 +72,9 @@ int orc_quantize_1d(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
  * start at sum_{j<e} orc_scale_rows(off[j+1]-off[j]).  sf must hold
  * orc_grouped_scale_rows(...) * orc_scale_cols(k) bytes.                    */
 int64_t orc_grouped_scale_rows(const int32_t* off, int num_groups);
+/* 1D quantization with a caller-given global scale g (> 0, finite). */
+int orc_quantize_1d_given_g(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, float g,
+                            uint8_t* codes, uint8_t* sf);
 int orc_quantize_1d_grouped(const uint16_t* x, const int32_t* off, int num_groups,
                             int64_t k, int64_t ld, uint8_t* codes, uint8_t* sf,
                             float* g_out);

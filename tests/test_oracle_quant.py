@@ -208,3 +208,24 @@ def test_scale_layout_is_a_bijection():
         R, C = O.scale_rows(rows), O.scale_cols(k)
         offs = {O.sf_offset(r, c, k) for r in range(R) for c in range(C)}
         assert offs == set(range(R * C))
+
+
+def test_given_scale_matches_dynamic_and_moves_the_scale_exponent():
+    """The given-scale quantizer (second pass of the two-phase form) equals
+    the dynamic one when given the tensor's own global scale.  With g doubled
+    every block scale drops by exactly one E4M3 exponent step (all blocks here
+    stay in the normal range) and, d = dec(sf) g being unchanged, every code
+    stays the same."""
+    x = W.gaussian_bf16((64, 256), 0, 71, 1.0)
+    c0, s0, g0 = O.quantize_1d(x)
+    c1, s1 = O.quantize_1d_given_g(x, g0)
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1)
+    c2, s2 = O.quantize_1d_given_g(x, np.float32(2.0) * np.float32(g0))
+    assert np.array_equal(c0, c2)
+    used = s0 != 0                                   # padding bytes stay 0
+    d0 = np.array([O.e4m3_decode(int(b)) for b in s0[used]])
+    d2 = np.array([O.e4m3_decode(int(b)) for b in s2[used]])
+    assert d0.min() >= 2.0 ** -5                     # halving keeps every scale normal
+    assert np.array_equal(d2, d0 / 2)
+    with pytest.raises(ValueError):
+        O.quantize_1d_given_g(x, 0.0)
