@@ -666,6 +666,7 @@ struct alignas(8) PairTail : std::conditional_t<GROUPED, PairGroups, PairNoGroup
     uint64_t sf_ready[P::NSB];       // leader: 8 scale warps staged a buffer
     uint64_t sf_free[P::NSB];        // each CTA: MMAs reading a scale buffer done
     uint64_t sk_bar;                 // each CTA: the next pair's partial sums landed (stream-K head)
+    uint32_t cmax[P::EPI_WARPS * 32];   // output-maximum variant: each epilogue lane's running max |C|
     uint32_t tmem_base;
     volatile int abort_flag;
 };
@@ -992,7 +993,10 @@ __global__ void __launch_bounds__(P::THREADS, 1)
         const uint32_t stg = smem_u32(epi_smem) + (uint32_t)(warp - 2) * (P::EPI_BOXES * 2048u);
         const uint32_t empty0 = mapa_shared(smem_u32(&tail->acc_empty[0]), 0);
         const uint32_t empty_step = (uint32_t)sizeof(uint64_t);
-        uint32_t cam = 0;                             // running max |C| of this lane's rows (packed)
+        // output-maximum variant: the lane's running max |C| lives in shared
+        // memory, not in a register held across the whole loop
+        uint32_t* cmax = &tail->cmax[(warp - 2) * 32 + lane];
+        if (EMIT) *cmax = 0u;
         int it = 0;
         PairWork w;
         for (; w.next(p, cluster, dp_tiles); ++it) {
@@ -1059,10 +1063,6 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                         }
                     }
                     return;
-                }
-                if (EMIT && q * 32 + lane < a_rows) {   // the output maximum, chunk by chunk
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) cam = max_abs_bf16x2(cam, w16[j]);
                 }
                 const uint32_t box = stg + (P::EPI_BOXES == 2 ? (uint32_t)(ch & 1) * 2048u : 0u);
                 if (lane == 0) {
@@ -1148,6 +1148,12 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                         bh[16 + i] =
                             pack_bf16x2(__uint_as_float(va1[2 * i]) * alpha, __uint_as_float(va1[2 * i + 1]) * alpha);
                     }
+                    if (EMIT && q * 32 + lane < a_rows) {
+                        uint32_t cm = *cmax;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) cm = max_abs_bf16x2(cm, bh[i]);
+                        *cmax = cm;
+                    }
                     store_chunk(c0 + cp * 2, bh);
                     store_chunk(c0 + cp * 2 + 1, bh + 16);
                 }
@@ -1157,6 +1163,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
             // convert them to BF16 in registers; release the accumulator after
             // the last read, then stage and store.
             uint32_t bf[NCP * 32];
+            uint32_t cm = 0;   // output-maximum variant: this tile's max |C| in the lane's row
 #pragma unroll
             for (int cp = 0; cp < NCP; ++cp) {
                 uint32_t va0[32], va1[32];
@@ -1174,12 +1181,14 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                                                   __uint_as_float(va0[2 * i + 1]) * alpha);
                     bf[cp * 32 + 16 + i] = pack_bf16x2(__uint_as_float(va1[2 * i]) * alpha,
                                                        __uint_as_float(va1[2 * i + 1]) * alpha);
+                    if (EMIT) cm = max_abs_bf16x2(cm, max_abs_bf16x2(bf[cp * 32 + i], bf[cp * 32 + 16 + i]));
                 }
             }
+            if (EMIT && q * 32 + lane < a_rows) *cmax = max_abs_bf16x2(*cmax, cm);
 #pragma unroll
             for (int h = 0; h < 2 * NCP; ++h) store_chunk(c0 + h, bf + h * 16);
         }
-        if (EMIT) fold_c_amax(p, cam);
+        if (EMIT) fold_c_amax(p, *cmax);
         if (lane == 0) bulk_wait_group_all();
         __syncwarp();
     }
