@@ -1086,23 +1086,21 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                 // group g of row r at slot[g * 128 + r] (lane-contiguous 16-byte
                 // pieces), then one count per warp.
                 float4* slot = reinterpret_cast<float4*>(p.partial + (size_t)slot_idx * (128 * BN)) + q * 32 + lane;
-#pragma unroll
-                for (int cp = 0; cp < NCP; ++cp) {
-                    uint32_t va0[32], va1[32];
-                    tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32, va0);
-                    tmem_ld_32x32b_x32(tq + (c0 + cp * 2) * 32 + 32, va1);
+                // 32 columns at a time: this rare path keeps few values live
+#pragma unroll 1
+                for (int ch = 0; ch < 2 * NCP; ++ch) {
+                    uint32_t va[32];
+                    tmem_ld_32x32b_x32(tq + (c0 + ch) * 32, va);
                     tmem_ld_wait();
-                    if (cp == NCP - 1) {
+                    if (ch == 2 * NCP - 1) {
                         tc_fence_before();
                         __syncwarp();
                         if (lane == 0) mbar_arrive_cluster(empty0 + ab * empty_step);
                     }
-                    float4* part = slot + (c0 + cp * 2) * 8 * 128;   // one base, immediate offsets
+                    float4* part = slot + (c0 + ch) * 8 * 128;   // one base, immediate offsets
                     static_for<8>([&](auto ic) {
                         constexpr int i = decltype(ic)::value;
-                        st_global_v4_at<i * 2048>(part, va0[4 * i], va0[4 * i + 1], va0[4 * i + 2], va0[4 * i + 3]);
-                        st_global_v4_at<(8 + i) * 2048>(part, va1[4 * i], va1[4 * i + 1], va1[4 * i + 2],
-                                                        va1[4 * i + 3]);
+                        st_global_v4_at<i * 2048>(part, va[4 * i], va[4 * i + 1], va[4 * i + 2], va[4 * i + 3]);
                     });
                 }
                 // the warp barrier orders every lane's stores before lane 0's
