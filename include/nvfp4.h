@@ -136,6 +136,21 @@ nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_
                                   uint8_t* codes, uint8_t* scales, float* global_scale,
                                   void* workspace, void* stream);
 
+/* nvfp4_quantize_act_smooth -- nvfp4_quantize_act of one tensor with a
+ * per-channel pre-scaling folded in (SmoothQuant style: per-channel factors
+ * move activation outliers into the weights; the pages discuss such
+ * outlier handling next to NVFP4's block scales): the tensor quantized is
+ * x'[r][c] = fp32(x[r][c]) * smooth[c] (one IEEE product), and every step --
+ * amax, global scale, block scales, codes -- runs on x'.  The weights take
+ * the inverse factors before their (offline) quantization.
+ *   smooth: device FP32 [k], positive and finite; every product finite.
+ *   k % 64 == 0 and k <= 6144 (the factors sit in shared memory); else
+ *   NVFP4_ERR_UNSUPPORTED_SHAPE.  Other arguments as nvfp4_quantize_act with
+ *   group_offsets NULL (same workspace).  One cooperative launch. */
+nvfp4_status_t nvfp4_quantize_act_smooth(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                         const float* smooth, uint8_t* codes, uint8_t* scales,
+                                         float* global_scale, void* workspace, void* stream);
+
 /* nvfp4_quantize_act_scaled -- the quantize pass of nvfp4_quantize_act with
  * the global scale given (one tensor): codes and scales exactly as
  * nvfp4_quantize_act would write them if the tensor's amax were

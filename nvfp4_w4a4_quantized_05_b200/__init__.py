@@ -23,11 +23,11 @@ __all__ = [
     "lib", "Nvfp4Error", "NVFP4Tensor",
     "nvfp4_codes_bytes", "nvfp4_scale_bytes", "nvfp4_grouped_scale_bytes", "nvfp4_workspace_bytes",
     "nvfp4_workspace_init", "nvfp4_quantize_act", "nvfp4_quantize_act_static", "nvfp4_quantize_weight_2d",
-    "nvfp4_gemm", "nvfp4_gemm_emit_scale", "nvfp4_quantize_act_scaled",
+    "nvfp4_gemm", "nvfp4_gemm_emit_scale", "nvfp4_quantize_act_scaled", "nvfp4_quantize_act_smooth",
     "nvfp4_grouped_gemm", "nvfp4_get_last_device_error", "nvfp4_set_wait_limit_ns", "nvfp4_probe_cvt",
     "nvfp4_probe_bounded_wait", "nvfp4_status_string", "nvfp4_version",
     "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
-    "gemm_emit_scale", "quantize_act_scaled",
+    "gemm_emit_scale", "quantize_act_scaled", "quantize_act_smooth",
     "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM", "OP_GEMM_EMIT_SCALE",
 ]
 
@@ -63,6 +63,7 @@ _SIGNATURES = {
     "nvfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_gemm_emit_scale": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp]),
     "nvfp4_quantize_act_scaled": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
+    "nvfp4_quantize_act_smooth": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_get_last_device_error": (_i32, [_vp]),
     "nvfp4_set_wait_limit_ns": (_u64, [_u64]),
@@ -165,6 +166,10 @@ def nvfp4_gemm_emit_scale(a_codes, a_scales, a_global, b_codes, b_scales, b_glob
                           c_global_scale, workspace, stream=0) -> int:
     return lib().nvfp4_gemm_emit_scale(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
                                        c_global_scale, workspace, stream)
+
+
+def nvfp4_quantize_act_smooth(x, rows, k, ld, smooth, codes, scales, global_scale, workspace, stream=0) -> int:
+    return lib().nvfp4_quantize_act_smooth(x, rows, k, ld, smooth, codes, scales, global_scale, workspace, stream)
 
 
 def nvfp4_quantize_act_scaled(x, rows, k, ld, global_scale, codes, scales, stream=0) -> int:
@@ -336,6 +341,34 @@ def gemm_emit_scale(a: NVFP4Tensor, b: NVFP4Tensor, out=None, out_scale=None):
                                _stream_ptr(torch, dev))
     _check(st, "nvfp4_gemm_emit_scale")
     return c, g
+
+
+def quantize_act_smooth(x, smooth, out: Optional[NVFP4Tensor] = None) -> NVFP4Tensor:
+    """Dynamic 1D quantization of x' = x * smooth[column] (per-channel
+    pre-scaling, SmoothQuant style) for a BF16 [rows, k] CUDA tensor and a
+    device FP32 [k] factor vector."""
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along k")
+    rows, k = x.shape
+    if smooth.dtype != torch.float32 or smooth.numel() != k or not smooth.is_cuda:
+        raise TypeError("smooth must be a float32 CUDA tensor of k factors")
+    dev = x.device
+    if out is not None:
+        if out.rows != rows or out.k != k or out.scales.numel() < nvfp4_scale_bytes(rows, k) or out.offsets is not None:
+            raise ValueError("out does not match the input shape")
+        codes, scales, g = out.codes, out.scales, out.global_scale
+    else:
+        codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty(nvfp4_scale_bytes(rows, k), dtype=torch.uint8, device=dev)
+        g = torch.empty(1, dtype=torch.float32, device=dev)
+    ws = _workspace(torch, dev, OP_QUANTIZE_ACT)
+    st = nvfp4_quantize_act_smooth(_ptr(x), rows, k, x.stride(0), _ptr(smooth), _ptr(codes), _ptr(scales), _ptr(g),
+                                   _ptr(ws), _stream_ptr(torch, dev))
+    _check(st, "nvfp4_quantize_act_smooth")
+    return out if out is not None else NVFP4Tensor(codes, scales, g, rows, k)
 
 
 def quantize_act_scaled(x, global_scale, out: Optional[NVFP4Tensor] = None) -> NVFP4Tensor:

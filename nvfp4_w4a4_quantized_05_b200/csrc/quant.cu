@@ -437,6 +437,7 @@ constexpr int kTaskBytes = kTaskVals * 2;
 constexpr int kStage = 3;                        // task slots per warp
 
 constexpr int kMaxFusedGroups = 1024;            // row groups the one-launch form takes
+constexpr int kMaxSmoothK = 6144;                // k of the pre-scaled form (its factors sit in shared memory)
 
 struct FusedArgs {
     const uint16_t* x;
@@ -453,6 +454,7 @@ struct FusedArgs {
     uint64_t* gword;  // grouped: per-group generation << 32 | amax words
     const int32_t* offsets;   // grouped: [groups + 1]; nullptr for one tensor
     int groups;
+    const float* smooth;      // pre-scaled form: per-column factors [k]; nullptr otherwise
     uint64_t limit;
     unsigned* err;
 };
@@ -600,14 +602,41 @@ struct DstCursor {   // where a task's codes and scale words go (32-bit byte off
     __device__ __forceinline__ bool valid() const { return row + m.base < m.rlast; }
 };
 
+// Eight BF16 values, each times its column factor (x' = x s, one IEEE product),
+// then times r -> eight packed E2M1 codes.
+__device__ __forceinline__ uint32_t quant8_smooth(const uint4& v, const float4& s0, const float4& s1, uint64_t rr) {
+    const float r = __uint_as_float((uint32_t)rr);
+    float x[8];
+    x[0] = __fmul_rn(__fmul_rn(__uint_as_float(v.x << 16), s0.x), r);
+    x[1] = __fmul_rn(__fmul_rn(__uint_as_float(v.x & 0xFFFF0000u), s0.y), r);
+    x[2] = __fmul_rn(__fmul_rn(__uint_as_float(v.y << 16), s0.z), r);
+    x[3] = __fmul_rn(__fmul_rn(__uint_as_float(v.y & 0xFFFF0000u), s0.w), r);
+    x[4] = __fmul_rn(__fmul_rn(__uint_as_float(v.z << 16), s1.x), r);
+    x[5] = __fmul_rn(__fmul_rn(__uint_as_float(v.z & 0xFFFF0000u), s1.y), r);
+    x[6] = __fmul_rn(__fmul_rn(__uint_as_float(v.w << 16), s1.z), r);
+    x[7] = __fmul_rn(__fmul_rn(__uint_as_float(v.w & 0xFFFF0000u), s1.w), r);
+    return cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
+}
+// max |x s| over the eight values of a unit.
+__device__ __forceinline__ float absmax8_smooth(const uint4& v, const float4& s0, const float4& s1) {
+    float m = fabsf(__fmul_rn(__uint_as_float(v.x << 16), s0.x));
+    m = fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.x & 0xFFFF0000u), s0.y)));
+    m = fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.y << 16), s0.z)));
+    m = fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.y & 0xFFFF0000u), s0.w)));
+    m = fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.z << 16), s1.x)));
+    m = fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.z & 0xFFFF0000u), s1.y)));
+    m = fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.w << 16), s1.z)));
+    return fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.w & 0xFFFF0000u), s1.w)));
+}
+
 // Per-group quantizer constants: the global scale g and the bracket constants.
 struct GroupQ {
     float g;
     BlockQ c;
 };
-__device__ __forceinline__ GroupQ make_groupq(uint32_t amax_bits) {
+__device__ __forceinline__ GroupQ make_groupq(uint32_t amax_fbits) {   // FP32 bits of the amax
     GroupQ q;
-    const float amax = __uint_as_float(amax_bits << 16);
+    const float amax = __uint_as_float(amax_fbits);
     q.g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kGlobalDen);
     q.c = make_blockq(q.g);
     return q;
@@ -621,19 +650,28 @@ __device__ __forceinline__ uint64_t block_rr(uint32_t sf, float g) {
 
 // Quantize the task held in slot sb.  FULL: the whole task is inside the
 // tensor.  One tensor: r from the per-CTA table; grouped: r computed per block.
-template <bool FULL, bool GROUPED>
+template <bool FULL, bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
-                                              const LaneC& lc, const GroupQ& gq, const uint64_t* rtab) {
+                                              const LaneC& lc, const GroupQ& gq, const uint64_t* rtab,
+                                              const float* ssm) {
     uint4 u[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4*>(sb + lc.ld_off[i]);
-    // Packed maxima of |x| per block, then both blocks' halves against each other:
-    // m = (amax of block 2 lane + 1 in the high half, of block 2 lane in the low).
-    const uint32_t m0 = bmax_abs(absmax8_packed(u[0]), absmax8_packed(u[1]));
-    const uint32_t m1 = bmax_abs(absmax8_packed(u[2]), absmax8_packed(u[3]));
-    const uint32_t m = bmax_abs(__byte_perm(m0, m1, 0x5410), __byte_perm(m0, m1, 0x7632));
-    const float b0 = __uint_as_float((m << 16) & 0x7FFF0000u);
-    const float b1 = __uint_as_float(m & 0x7FFF0000u);
+    float b0, b1;
+    const float4* sv = nullptr;   // pre-scaled form: the factors of this lane's 32 columns
+    if constexpr (SMOOTH) sv = reinterpret_cast<const float4*>(ssm + t.seg * kTaskVals + 32 * lc.lane);
+    if constexpr (SMOOTH) {
+        b0 = fmaxf(absmax8_smooth(u[0], sv[0], sv[1]), absmax8_smooth(u[1], sv[2], sv[3]));
+        b1 = fmaxf(absmax8_smooth(u[2], sv[4], sv[5]), absmax8_smooth(u[3], sv[6], sv[7]));
+    } else {
+        // Packed maxima of |x| per block, then both blocks' halves against each other:
+        // m = (amax of block 2 lane + 1 in the high half, of block 2 lane in the low).
+        const uint32_t m0 = bmax_abs(absmax8_packed(u[0]), absmax8_packed(u[1]));
+        const uint32_t m1 = bmax_abs(absmax8_packed(u[2]), absmax8_packed(u[3]));
+        const uint32_t m = bmax_abs(__byte_perm(m0, m1, 0x5410), __byte_perm(m0, m1, 0x7632));
+        b0 = __uint_as_float((m << 16) & 0x7FFF0000u);
+        b1 = __uint_as_float(m & 0x7FFF0000u);
+    }
     const uint32_t pair = block_sf2(b0, b1, gq.c);   // scale bytes of blocks 2 lane, 2 lane + 1
     uint64_t rr0, rr1;
     if constexpr (GROUPED) {
@@ -644,10 +682,17 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
         rr1 = rtab[pair >> 8];
     }
     uint4 q;
-    q.x = quant8(u[0], rr0);
-    q.y = quant8(u[1], rr0);
-    q.z = quant8(u[2], rr1);
-    q.w = quant8(u[3], rr1);
+    if constexpr (SMOOTH) {
+        q.x = quant8_smooth(u[0], sv[0], sv[1], rr0);
+        q.y = quant8_smooth(u[1], sv[2], sv[3], rr0);
+        q.z = quant8_smooth(u[2], sv[4], sv[5], rr1);
+        q.w = quant8_smooth(u[3], sv[6], sv[7], rr1);
+    } else {
+        q.x = quant8(u[0], rr0);
+        q.y = quant8(u[1], rr0);
+        q.z = quant8(u[2], rr1);
+        q.w = quant8(u[3], rr1);
+    }
     const uint32_t word = __byte_perm(pair, __shfl_down_sync(kFull, pair, 1), 0x5410);
     const bool even = (lc.lane & 1) == 0;
     uint8_t* dst = a.codes + t.co + 16 * lc.lane;
@@ -662,18 +707,19 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
         if (even && t.seg * (kTaskVals / 16) + 2 * lc.lane < a.scale_cols) *sw = word;
     }
 }
-template <bool GROUPED>
+template <bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void quantize_any(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
-                                             const LaneC& lc, const GroupQ& gq, const uint64_t* rtab) {
+                                             const LaneC& lc, const GroupQ& gq, const uint64_t* rtab,
+                                             const float* ssm) {
     if (t.valid() && t.seg < a.full_segs)
-        quantize_slot<true, GROUPED>(a, sb, t, lc, gq, rtab);
+        quantize_slot<true, GROUPED, SMOOTH>(a, sb, t, lc, gq, rtab, ssm);
     else
-        quantize_slot<false, GROUPED>(a, sb, t, lc, gq, rtab);
+        quantize_slot<false, GROUPED, SMOOTH>(a, sb, t, lc, gq, rtab, ssm);
 }
 
 // Grid barrier (and, for one tensor, the amax reduction) in one: CTA c
 // publishes its word (part + kPartStrideWords c, one per 128-byte line) =
-// gen << 32 | (its BF16 amax bits; 0 in the grouped form), so a reader that
+// gen << 32 | (the FP32 bits of its amax; 0 in the grouped form), so a reader that
 // sees this call's generation also sees the amax.  gen is one more (mod 2^32)
 // than the generation of the CTA's own word from the previous call (0 in a
 // fresh workspace), the same for every CTA.  Warp 0 of each CTA polls all G
@@ -687,7 +733,7 @@ __device__ __forceinline__ bool grid_amax(const uint64_t* part, int G, uint32_t 
         for (int i = lane; i < G; i += 32) {
             const uint64_t w = ld_relaxed_gpu_u64(part + kPartStrideWords * i);
             mine = mine && (uint32_t)(w >> 32) == gen;
-            mx = max(mx, (uint32_t)w & 0xFFFFu);
+            mx = max(mx, (uint32_t)w);
         }
         if (__all_sync(kFull, mine)) {
 #pragma unroll
@@ -788,10 +834,10 @@ struct Pass2Q {
 // likeliest to be still in L2 when the tensor is larger than L2.  Quantizing
 // on-chip task k frees its slot for the k-th of those, and then the q-th
 // follows the (q - kStage)-th through the same slot.
-template <bool GROUPED>
+template <bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const FusedArgs& a, const GroupTab& gt, Ring& r,
                                             const uint64_t* rtab, Pass2Q<GROUPED>& pq, uint32_t gen, int tw, int n,
-                                            const LaneC& lc) {
+                                            const LaneC& lc, const float* ssm) {
     const uint64_t pol = l2_policy_evict_first();   // last use
     const int nres = n < kStage ? n : kStage;
     const int nl = n - nres;
@@ -804,7 +850,7 @@ __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const Fused
     }
     int s = (n - nres) % kStage;
     for (int k = 0; k < nres; ++k) {
-        quantize_any<GROUPED>(a, r.slot(s), rp, lc, pq.at(a, rp, gen), rtab);
+        quantize_any<GROUPED, SMOOTH>(a, r.slot(s), rp, lc, pq.at(a, rp, gen), rtab, ssm);
         rp.next(a, gt);
         __syncwarp();   // every lane is done reading the slot
         if (k < nl) {
@@ -816,7 +862,7 @@ __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const Fused
     // s is back at the slot of the first on-chip task, where the first refill lands.
     for (int q = 0; q < nl; ++q) {
         land(r, s, a);
-        quantize_any<GROUPED>(a, r.slot(s), lq, lc, pq.at(a, lq, gen), rtab);
+        quantize_any<GROUPED, SMOOTH>(a, r.slot(s), lq, lc, pq.at(a, lq, gen), rtab, ssm);
         lq.prev(a, gt);
         __syncwarp();
         if (q + kStage < nl) {
@@ -827,7 +873,8 @@ __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const Fused
     }
 }
 
-template <bool GROUPED>
+// SMOOTH: the pre-scaled form (one tensor): x' = x s[column] is quantized.
+template <bool GROUPED, bool SMOOTH = false>
 __global__ void __launch_bounds__(kFThreads, 1)
     quant1d_fused_kernel(const __grid_constant__ CUtensorMap tmap, FusedArgs a, uint32_t box_bytes) {
     extern __shared__ __align__(1024) uint8_t dsm[];   // kStage task slots per warp (+ alignment pad)
@@ -836,6 +883,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __shared__ uint32_t red[kFWarps];
     __shared__ int s_off[GROUPED ? kMaxFusedGroups + 1 : 1];
     __shared__ int s_blk[GROUPED ? kMaxFusedGroups + 1 : 1];
+    __shared__ __align__(16) float s_smooth[SMOOTH ? kMaxSmoothK : 4];
     __shared__ uint32_t s_amax, s_gen;
     __shared__ int s_ok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -875,6 +923,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
         if (e < a.groups) s_blk[e] = wbase + inc - nb;
         if (e == a.groups - 1) s_blk[a.groups] = wbase + inc;
     }
+    if constexpr (SMOOTH) {
+        // the factors, zero past k up to the last task's end (k <= kMaxSmoothK)
+        const int kt = a.nseg * kTaskVals;
+        for (int i = tid; i < kt; i += kFThreads) s_smooth[i] = i < a.k ? a.smooth[i] : 0.0f;
+    }
     fence_mbar_init();
     __syncthreads();
     const uint32_t gen = s_gen;
@@ -893,7 +946,8 @@ __global__ void __launch_bounds__(kFThreads, 1)
 
     // ---- pass 1: amax through the slot ring; the last kStage tasks stay on chip
     const LaneC lc = make_lanec(lane);
-    uint32_t acc = 0;
+    uint32_t acc = 0;      // packed BF16 running max |x|
+    float accf = 0.0f;     // pre-scaled form: running max |x s|
     {
         const uint64_t pol_keep = l2_policy_evict_normal();   // read again in pass 2
         const uint64_t pol_last = l2_policy_evict_first();    // stays on chip: not read again
@@ -915,21 +969,33 @@ __global__ void __launch_bounds__(kFThreads, 1)
         for (int i = 0; i < n; ++i) {
             cp_async_wait<kStage - 1>();
             __syncwarp();   // every lane's copies into the slot have landed
-            if constexpr (GROUPED) {
-                if (lp.m.e != cur) {   // warp-uniform: a new group starts with this task
-                    uint32_t m = absmax_bits(acc);
+            int seg_now = 0;
+            if constexpr (GROUPED || SMOOTH) {
+                if constexpr (GROUPED) {
+                    if (lp.m.e != cur) {   // warp-uniform: a new group starts with this task
+                        uint32_t m = absmax_bits(acc) << 16;   // FP32 bits
 #pragma unroll
-                    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
-                    if (lane == 0) fold_group_amax(a.gword + cur, gen, m);
-                    cur = lp.m.e;
-                    acc = 0;
+                        for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+                        if (lane == 0) fold_group_amax(a.gword + cur, gen, m);
+                        cur = lp.m.e;
+                        acc = 0;
+                    }
                 }
+                seg_now = lp.seg;
                 lp.next(a, gt);
             }
             const char* sb = r.slot(s);
+            if constexpr (SMOOTH) {
+                const float4* sv = reinterpret_cast<const float4*>(s_smooth + seg_now * kTaskVals + 32 * lane);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                acc = bmax_abs(acc, absmax8_packed(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q])));
+                for (int q = 0; q < 4; ++q)
+                    accf = fmaxf(accf, absmax8_smooth(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q]), sv[2 * q],
+                                                      sv[2 * q + 1]));
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    acc = bmax_abs(acc, absmax8_packed(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q])));
+            }
             if (i + kStage < n) {
                 __syncwarp();   // every lane is done reading the slot
                 stage_cp<GROUPED>(a, r, s, sp, lc, i + kStage >= n - kStage ? pol_last : pol_keep);
@@ -942,7 +1008,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         __syncwarp();
         if constexpr (GROUPED) {
             if (n > 0) {
-                uint32_t m = absmax_bits(acc);
+                uint32_t m = absmax_bits(acc) << 16;
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
                 if (lane == 0) fold_group_amax(a.gword + cur, gen, m);
@@ -950,7 +1016,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
         }
     }
     if constexpr (!GROUPED) {
-        uint32_t m = absmax_bits(acc);
+        uint32_t m = SMOOTH ? __float_as_uint(accf) : absmax_bits(acc) << 16;   // FP32 bits
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
         if (lane == 0) red[warp] = m;
@@ -989,7 +1055,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
             fill_rtab(rtab, pq.q.g, tid);
             __syncthreads();
         }
-        fused_pass2<GROUPED>(&tmap, a, gt, r, rtab, pq, gen, tw, n, lc);
+        fused_pass2<GROUPED, SMOOTH>(&tmap, a, gt, r, rtab, pq, gen, tw, n, lc, s_smooth);
     }
     pdl_launch_dependents();
 }
@@ -1087,10 +1153,12 @@ cudaError_t launch_pdl(const void* func, dim3 grid, dim3 block, void** args, cud
 // scales too large for 32-bit offsets -- or the device cannot hold one such
 // CTA per SM; the caller then takes the two-kernel path.
 nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const int32_t* offsets, int groups,
-                         uint8_t* codes, uint8_t* scales, float* gscale, void* workspace, cudaStream_t s) {
+                         uint8_t* codes, uint8_t* scales, float* gscale, void* workspace, cudaStream_t s,
+                         const float* smooth = nullptr) {
     constexpr int kSmemMax = kStage * kFWarps * kTaskBytes + 1024;
     const bool grouped = offsets != nullptr;
     if (grouped && groups > kMaxFusedGroups) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (smooth && (grouped || round_up(k, kTaskVals) > kMaxSmoothK)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int64_t prow = round_up(rows + (grouped ? 127 * (int64_t)groups : 0), 128);   // padded rows, at most
     if (k % 64 != 0 || prow * k >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     static std::mutex mu;
@@ -1100,18 +1168,22 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     {
         std::lock_guard<std::mutex> lk(mu);
         if (ready[dev] == 0) {
-            int occ0 = 0, occ1 = 0;
+            int occ0 = 0, occ1 = 0, occ2 = 0;
             const bool ok =
                 tensor_map_encoder() != nullptr &&
                 cudaFuncSetAttribute(quant1d_fused_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSmemMax) == cudaSuccess &&
                 cudaFuncSetAttribute(quant1d_fused_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSmemMax) == cudaSuccess &&
+                cudaFuncSetAttribute(quant1d_fused_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     kSmemMax) == cudaSuccess &&
                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ0, quant1d_fused_kernel<false>, kFThreads,
                                                               kSmemMax) == cudaSuccess &&
                 cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ1, quant1d_fused_kernel<true>, kFThreads,
                                                               kSmemMax) == cudaSuccess &&
-                occ0 >= 1 && occ1 >= 1;
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ2, quant1d_fused_kernel<false, true>, kFThreads,
+                                                              kSmemMax) == cudaSuccess &&
+                occ0 >= 1 && occ1 >= 1 && occ2 >= 1;
             ready[dev] = ok ? 1 : -1;
         }
         if (ready[dev] < 0) {
@@ -1157,6 +1229,7 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     a.gword = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_gword_off(groups));
     a.offsets = offsets;
     a.groups = grouped ? groups : 1;
+    a.smooth = smooth;
     a.limit = wait_limit_ns();
     a.err = device_error_word();
     if (!a.err) return NVFP4_ERR_CUDA;
@@ -1171,8 +1244,9 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     void* args[] = {&tmap, &a, &box_bytes};
-    const void* kern = grouped ? reinterpret_cast<const void*>(&quant1d_fused_kernel<true>)
-                               : reinterpret_cast<const void*>(&quant1d_fused_kernel<false>);
+    const void* kern = grouped  ? reinterpret_cast<const void*>(&quant1d_fused_kernel<true>)
+                       : smooth ? reinterpret_cast<const void*>(&quant1d_fused_kernel<false, true>)
+                                : reinterpret_cast<const void*>(&quant1d_fused_kernel<false>);
     return cuda_status(cudaLaunchKernelExC(&cfg, kern, args));
 }
 
@@ -1297,6 +1371,21 @@ extern "C" nvfp4_status_t nvfp4_probe_cvt(const float* in, uint8_t* out_e2m1, ui
     const int grid = clamp_grid((n + 255) / 256, (int64_t)num_sms() * 16);
     probe_cvt_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(in, out_e2m1, out_e4m3, n);
     return cuda_status(cudaGetLastError());
+}
+
+extern "C" nvfp4_status_t nvfp4_quantize_act_smooth(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                                    const float* smooth, uint8_t* codes, uint8_t* scales,
+                                                    float* global_scale, void* workspace, void* stream) {
+    if (rows < 0 || k <= 0 || ld < k) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (!x || !smooth || !codes || !scales || !global_scale || !workspace) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 64 != 0 || round_up(k, kTaskVals) > kMaxSmoothK || rows >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(workspace) ||
+        (reinterpret_cast<uintptr_t>(smooth) & 3u) || (reinterpret_cast<uintptr_t>(global_scale) & 3u) || ld % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
+    return run_fused(reinterpret_cast<const uint16_t*>(x), rows, k, ld, nullptr, 1, codes, scales, global_scale,
+                     workspace, reinterpret_cast<cudaStream_t>(stream), smooth);
 }
 
 extern "C" nvfp4_status_t nvfp4_quantize_act_scaled(const void* x, int64_t rows, int64_t k, int64_t ld,

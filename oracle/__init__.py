@@ -51,6 +51,7 @@ def lib():
             "orc_global_scale": (ctypes.c_float, [ctypes.c_float]),
             "orc_quantize_1d": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _u8p, _u8p, _f32p]),
             "orc_quantize_1d_given_g": (ctypes.c_int, [_u16p, _i64, _i64, _i64, ctypes.c_float, _u8p, _u8p]),
+            "orc_quantize_1d_smooth": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _f32p, _u8p, _u8p, _f32p]),
             "orc_grouped_scale_rows": (_i64, [_i32p, ctypes.c_int]),
             "orc_quantize_1d_grouped": (ctypes.c_int, [_u16p, _i32p, ctypes.c_int, _i64, _i64,
                                                        _u8p, _u8p, _f32p]),
@@ -159,6 +160,24 @@ def quantize_1d_given_g(x_bf16: np.ndarray, g: float):
     if rc != 0:
         raise ValueError(f"orc_quantize_1d_given_g failed ({rc})")
     return codes, sf
+
+
+def quantize_1d_smooth(x_bf16: np.ndarray, s: np.ndarray):
+    """1D quantization of x' = fp32(x) * s[column] (SmoothQuant-style
+    per-channel pre-scaling folded into the quantizer).  Returns (codes,
+    scales, g)."""
+    x = _bf16(x_bf16)
+    rows, k = x.shape
+    sv = np.ascontiguousarray(s, dtype=np.float32)
+    if sv.shape != (k,):
+        raise ValueError("s must have one factor per column")
+    codes = np.zeros((rows, k // 2), np.uint8)
+    sf = np.zeros(scale_rows(rows) * scale_cols(k), np.uint8)
+    g = np.zeros(1, np.float32)
+    rc = lib().orc_quantize_1d_smooth(x, rows, k, k, sv, codes, sf, g)
+    if rc != 0:
+        raise ValueError(f"orc_quantize_1d_smooth failed ({rc})")
+    return codes, sf, float(g[0])
 
 
 def grouped_scale_rows(offsets: np.ndarray) -> int:

@@ -196,6 +196,49 @@ int orc_quantize_1d(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     return 0;
 }
 
+/* SmoothQuant-style per-channel pre-scaling folded into the 1D quantizer:
+ * the values quantized are x'[r][c] = fp32(x[r][c]) * s[c] (one IEEE
+ * product), and every step of orc_quantize_1d then runs on x' (amax, global
+ * scale, block amax, block scale, codes).  s: k positive finite factors;
+ * every product must be finite. */
+int orc_quantize_1d_smooth(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const float* s,
+                           uint8_t* codes, uint8_t* sf, float* g_out) {
+    if (rows < 0 || k <= 0 || k % 16 != 0 || ld < k) return 1;
+    for (int64_t j = 0; j < k; ++j)
+        if (!(s[j] > 0.0f) || !isfinite(s[j])) return 1;
+    if (check_finite_rows(x, 0, rows, k, ld)) return 2;
+    float amax = 0.0f;
+    int bad = 0;
+    #pragma omp parallel for reduction(max:amax) reduction(|:bad) schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            float v = orc_bf16_to_f32(x[r * ld + j]) * s[j];
+            if (!isfinite(v)) bad = 1;
+            if (fabsf(v) > amax) amax = fabsf(v);
+        }
+    if (bad) return 2;
+    float g = orc_global_scale(amax);
+    int64_t scale_cols = orc_scale_cols(k);
+    memset(sf, 0, (size_t)(orc_scale_rows(rows) * scale_cols));
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < k / 16; ++b) {
+            float xv[16];
+            uint8_t c[16];
+            float bamax = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                xv[i] = orc_bf16_to_f32(x[r * ld + b * 16 + i]) * s[b * 16 + i];
+                if (fabsf(xv[i]) > bamax) bamax = fabsf(xv[i]);
+            }
+            sf[orc_sf_offset(r, b, scale_cols)] = quantize_block(xv, 16, bamax, g, c);
+            for (int i = 0; i < 8; ++i)
+                codes[r * (k / 2) + b * 8 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+    *g_out = g;
+    return 0;
+}
+
 int64_t orc_grouped_scale_rows(const int32_t* off, int num_groups) {
     int64_t t = 0;
     for (int e = 0; e < num_groups; ++e) t += orc_scale_rows((int64_t)off[e + 1] - off[e]);

@@ -75,6 +75,9 @@ int64_t orc_grouped_scale_rows(const int32_t* off, int num_groups);
 /* 1D quantization with a caller-given global scale g (> 0, finite). */
 int orc_quantize_1d_given_g(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, float g,
                             uint8_t* codes, uint8_t* sf);
+/* 1D quantization of x'[r][c] = fp32(x[r][c]) * s[c] (per-channel pre-scaling, SmoothQuant style). */
+int orc_quantize_1d_smooth(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const float* s,
+                           uint8_t* codes, uint8_t* sf, float* g_out);
 int orc_quantize_1d_grouped(const uint16_t* x, const int32_t* off, int num_groups,
                             int64_t k, int64_t ld, uint8_t* codes, uint8_t* sf,
                             float* g_out);

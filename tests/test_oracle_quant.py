@@ -229,3 +229,26 @@ def test_given_scale_matches_dynamic_and_moves_the_scale_exponent():
     assert np.array_equal(d2, d0 / 2)
     with pytest.raises(ValueError):
         O.quantize_1d_given_g(x, 0.0)
+
+
+def test_smooth_quantizer_pins():
+    """Per-channel pre-scaling folded into the quantizer.  s = 1 is the plain
+    quantizer.  With powers of two per channel every product is exact, so the
+    result is the plain quantizer of the BF16 tensor x * 2^j[c] (in range).
+    A uniform factor 2^j moves only g: codes and scale bytes stay."""
+    x = W.laplace_outliers_bf16((48, 512), 0, 72)
+    c0, s0, g0 = O.quantize_1d(x)
+    c1, s1, g1 = O.quantize_1d_smooth(x, np.ones(512, np.float32))
+    assert np.array_equal(c0, c1) and np.array_equal(s0, s1) and g0 == g1
+    rng = np.random.default_rng(3)
+    j = rng.integers(-6, 7, 512)
+    xs = O.bf16_to_f64(x) * np.exp2(j)[None, :]          # exact in float32 and in BF16 (8-bit mantissas kept)
+    xb = (xs.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    assert np.array_equal(O.bf16_to_f64(xb), xs)
+    c2, s2, g2 = O.quantize_1d_smooth(x, np.exp2(j).astype(np.float32))
+    c3, s3, g3 = O.quantize_1d(xb)
+    assert np.array_equal(c2, c3) and np.array_equal(s2, s3) and g2 == g3
+    c4, s4, g4 = O.quantize_1d_smooth(x, np.full(512, 8.0, np.float32))
+    assert np.array_equal(c4, c0) and np.array_equal(s4, s0) and g4 == g0 * 8
+    with pytest.raises(ValueError):
+        O.quantize_1d_smooth(x, np.zeros(512, np.float32))
