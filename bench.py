@@ -328,6 +328,15 @@ class Quant:
         j = i % self.RW
         self.nv.quantize_weight_2d(self.w[j], out=self.qw[j])
 
+    def quantize_smooth(self, i):
+        """The same activations with per-channel pre-scaling folded in."""
+        j = i % self.R
+        if not hasattr(self, "smooth"):
+            import torch
+            g = np.random.default_rng(1)
+            self.smooth = torch.from_numpy(np.exp2(g.uniform(-3.0, 3.0, self.k)).astype(np.float32)).to(self.a[0].device)
+        self.nv.quantize_act_smooth(self.a[j], self.smooth, out=self.qa[j])
+
     def result(self, i):
         return self.qa[i % self.R].codes
 
@@ -704,6 +713,14 @@ def run_ours(args):
         line["weight_quantize"] = {"workload": f"bf16 [{wl.wn},{wl.k}] N(0,0.02) -> nvfp4, 16x16 blocks",
                                    "gbs": w_gbs, "frac_hbm": w_gbs / peaks["hbm_gbs"], "avg_ms": w_avg * 1e3,
                                    "algorithmic_bytes": wl.wqbytes, "kernels": "amax_kernel + quant2d_kernel"}
+        wl.quantize_smooth(0)
+        time.sleep(REST_S)
+        s_avg = graph_seconds(torch, cs, wl.quantize_smooth, wl.R, kiters)
+        s_bytes = wl.qbytes + 4 * wl.k
+        line["smooth_quantize"] = {"workload": f"the same activations x * s[column], s log-uniform in [1/8, 8]",
+                                   "gbs": s_bytes / s_avg / 1e9, "frac_hbm": s_bytes / s_avg / 1e9 / peaks["hbm_gbs"],
+                                   "avg_ms": s_avg * 1e3, "algorithmic_bytes": s_bytes,
+                                   "kernels": "quant1d_fused_kernel (pre-scaled form)"}
     if type(wl) is Prefill:
         one_phase, two_phase = wl.next_layer_steps(nv, torch)
         time.sleep(REST_S)

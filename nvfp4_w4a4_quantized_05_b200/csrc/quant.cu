@@ -602,6 +602,14 @@ struct DstCursor {   // where a task's codes and scale words go (32-bit byte off
     __device__ __forceinline__ bool valid() const { return row + m.base < m.rlast; }
 };
 
+// Factors of the pre-scaled form in shared memory: per 1024-column segment,
+// 16-byte unit u (columns 4 u .. 4 u + 3) at unit (u & ~7) | ((u & 7) ^ ((u >> 3) & 7)),
+// so that lane l's eight units 8 l .. 8 l + 7 (its 32 columns) fall in eight
+// different bank groups for every 8-lane phase of a 16-byte load.
+__device__ __forceinline__ float4 smooth_unit(const float* seg_base, int lane, int i) {
+    return reinterpret_cast<const float4*>(seg_base)[8 * lane + (i ^ (lane & 7))];
+}
+
 // Eight BF16 values, each times its column factor (x' = x s, one IEEE product),
 // then times r -> eight packed E2M1 codes.
 __device__ __forceinline__ uint32_t quant8_smooth(const uint4& v, const float4& s0, const float4& s1, uint64_t rr) {
@@ -658,9 +666,10 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
 #pragma unroll
     for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4*>(sb + lc.ld_off[i]);
     float b0, b1;
-    const float4* sv = nullptr;   // pre-scaled form: the factors of this lane's 32 columns
-    if constexpr (SMOOTH) sv = reinterpret_cast<const float4*>(ssm + t.seg * kTaskVals + 32 * lc.lane);
+    float4 sv[8];   // pre-scaled form: the factors of this lane's 32 columns
     if constexpr (SMOOTH) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sv[i] = smooth_unit(ssm + t.seg * kTaskVals, lc.lane, i);
         b0 = fmaxf(absmax8_smooth(u[0], sv[0], sv[1]), absmax8_smooth(u[1], sv[2], sv[3]));
         b1 = fmaxf(absmax8_smooth(u[2], sv[4], sv[5]), absmax8_smooth(u[3], sv[6], sv[7]));
     } else {
@@ -926,7 +935,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
     if constexpr (SMOOTH) {
         // the factors, zero past k up to the last task's end (k <= kMaxSmoothK)
         const int kt = a.nseg * kTaskVals;
-        for (int i = tid; i < kt; i += kFThreads) s_smooth[i] = i < a.k ? a.smooth[i] : 0.0f;
+        for (int i = tid; i < kt; i += kFThreads) {
+            const int seg = i / kTaskVals, u = (i % kTaskVals) >> 2;
+            const int pu = (u & ~7) | ((u & 7) ^ ((u >> 3) & 7));
+            s_smooth[seg * kTaskVals + pu * 4 + (i & 3)] = i < a.k ? a.smooth[i] : 0.0f;
+        }
     }
     fence_mbar_init();
     __syncthreads();
@@ -986,11 +999,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
             }
             const char* sb = r.slot(s);
             if constexpr (SMOOTH) {
-                const float4* sv = reinterpret_cast<const float4*>(s_smooth + seg_now * kTaskVals + 32 * lane);
+                const float* sb2 = s_smooth + seg_now * kTaskVals;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    accf = fmaxf(accf, absmax8_smooth(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q]), sv[2 * q],
-                                                      sv[2 * q + 1]));
+                    accf = fmaxf(accf, absmax8_smooth(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q]),
+                                                      smooth_unit(sb2, lane, 2 * q), smooth_unit(sb2, lane, 2 * q + 1)));
             } else {
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
