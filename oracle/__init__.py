@@ -62,6 +62,11 @@ def lib():
             "orc_gemm_f64_rows": (None, [_f64p, _f64p, _i64p, _i64, _i64, _i64, _f64p]),
             "orc_gemm_exact_i64": (None, [_u8p, _u8p, _u8p, _u8p, _i64, _i64, _i64, _i64p]),
             "orc_single_scale_fp4": (None, [_u16p, _i64, _f64p]),
+            "orc_mx_scale_cols": (_i64, [_i64]),
+            "orc_e8m0_block_scale": (ctypes.c_uint8, [ctypes.c_double]),
+            "orc_e8m0_decode": (ctypes.c_double, [ctypes.c_uint8]),
+            "orc_quantize_1d_mx": (ctypes.c_int, [_u16p, _i64, _i64, _i64, _u8p, _u8p]),
+            "orc_dequantize_mx": (None, [_u8p, _u8p, _i64, _i64, _f64p]),
             "orc_num_threads": (ctypes.c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -239,6 +244,43 @@ def dequantize_grouped(codes, sf, g, offsets) -> np.ndarray:
         if b > a:
             out[a:b] = dequantize(codes[a:b], sf, float(g[e]), sf_row0=row0, k=k)
         row0 += scale_rows(b - a)
+    return out
+
+
+# ---- MXFP4 ----------------------------------------------------------------------
+
+def mx_scale_cols(k: int) -> int:
+    return int(lib().orc_mx_scale_cols(k))
+
+
+def e8m0_block_scale(bamax: float) -> int:
+    """E8M0 byte of a 32-value block with maximum magnitude bamax."""
+    return int(lib().orc_e8m0_block_scale(float(bamax)))
+
+
+def e8m0_decode(b: int) -> float:
+    return float(lib().orc_e8m0_decode(b))
+
+
+def quantize_1d_mx(x_bf16: np.ndarray):
+    """MXFP4: 32-value blocks with E8M0 scales, no tensor scale.  Returns
+    (codes [R, K/2] u8, scales (flat, tile layout, k/32 columns rounded to 4) u8)."""
+    x = _bf16(x_bf16)
+    rows, k = x.shape
+    codes = np.zeros((rows, k // 2), np.uint8)
+    sf = np.zeros(scale_rows(rows) * mx_scale_cols(k), np.uint8)
+    rc = lib().orc_quantize_1d_mx(x, rows, k, k, codes, sf)
+    if rc != 0:
+        raise ValueError(f"orc_quantize_1d_mx failed ({rc})")
+    return codes, sf
+
+
+def dequantize_mx(codes: np.ndarray, sf: np.ndarray, k: int | None = None) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    rows = codes.shape[0]
+    k = codes.shape[1] * 2 if k is None else k
+    out = np.empty((rows, k), np.float64)
+    lib().orc_dequantize_mx(codes, np.ascontiguousarray(sf, dtype=np.uint8), rows, k, out)
     return out
 
 

@@ -403,3 +403,66 @@ void orc_single_scale_fp4(const uint16_t* x, int64_t n, double* x_hat) {
         x_hat[i] = orc_e2m1_decode(code) * (double)s;
     }
 }
+
+/* ------------------------------------------------------------------------ */
+/* MXFP4, the other four-bit format of the same tensor cores.  "NVFP4
+ * Explained: NVIDIA's 4-Bit Format for Faster AI Inference", "Why Blocks of
+ * 16 Improve Accuracy" and "Why the Block Scale Uses FP8 E4M3"; "What is
+ * NVFP4?", "NVFP4 versus MXFP4": the same E2M1 elements, one E8M0 scale --
+ * a bare power of two, 2^(byte - 127) -- shared by 32 values, and no
+ * tensor-wide scale.  How the power is chosen is not on the pages.  Reading
+ * used here: the smallest 2^e with 6 * 2^e >= block amax, so that the block
+ * maximum fits the E2M1 range without saturating (NVFP4's block scale puts
+ * it exactly on 6), with e clamped to [-127, 127]; a block of zeros takes
+ * byte 0.  code = E2M1_RNE(x / 2^e), sign kept.  Scale bytes use the same
+ * 128 x 4 tiles, one scale column per 32 values.                            */
+
+int64_t orc_mx_scale_cols(int64_t k) { return (k / 32 + 3) / 4 * 4; }
+
+uint8_t orc_e8m0_block_scale(double bamax) {
+    int e = -127;
+    while (e < 127 && 6.0 * ldexp(1.0, e) < bamax) ++e;   /* smallest e that holds the block */
+    return (uint8_t)(e + 127);
+}
+
+double orc_e8m0_decode(uint8_t b) { return ldexp(1.0, (int)b - 127); }   /* 0xFF (NaN) never produced */
+
+int orc_quantize_1d_mx(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
+                       uint8_t* codes, uint8_t* sf) {
+    if (rows < 0 || k <= 0 || k % 32 != 0 || ld < k) return 1;
+    if (check_finite_rows(x, 0, rows, k, ld)) return 2;
+    int64_t scale_cols = orc_mx_scale_cols(k);
+    memset(sf, 0, (size_t)(orc_scale_rows(rows) * scale_cols));
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t b = 0; b < k / 32; ++b) {
+            double xv[32];
+            double bamax = 0.0;
+            for (int i = 0; i < 32; ++i) {
+                xv[i] = (double)orc_bf16_to_f32(x[r * ld + b * 32 + i]);
+                if (fabs(xv[i]) > bamax) bamax = fabs(xv[i]);
+            }
+            uint8_t s = orc_e8m0_block_scale(bamax);
+            double scale = orc_e8m0_decode(s);
+            sf[orc_sf_offset(r, b, scale_cols)] = s;
+            uint8_t c[32];
+            /* x / 2^e is exact in binary64; its binary32 rounding only touches
+             * magnitudes far below 0.25, which encode to (signed) zero anyway */
+            for (int i = 0; i < 32; ++i) c[i] = orc_e2m1_encode((float)(xv[i] / scale));
+            for (int i = 0; i < 16; ++i)
+                codes[r * (k / 2) + b * 16 + i] = (uint8_t)(c[2 * i] | (c[2 * i + 1] << 4));
+        }
+    }
+    return 0;
+}
+
+void orc_dequantize_mx(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t k, double* out) {
+    int64_t scale_cols = orc_mx_scale_cols(k);
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < k; ++j) {
+            uint8_t byte = codes[r * (k / 2) + j / 2];
+            uint8_t code = (j % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            out[r * k + j] = orc_e2m1_decode(code) * orc_e8m0_decode(sf[orc_sf_offset(r, j / 32, scale_cols)]);
+        }
+}

@@ -105,6 +105,17 @@ void orc_gemm_exact_i64(const uint8_t* a_codes, const uint8_t* a_sf,
 /* ---- single-scale FP4 baseline: one scale amax/6, no block scales -------- */
 void orc_single_scale_fp4(const uint16_t* x, int64_t n, double* x_hat);
 
+/* ---- MXFP4: E2M1 elements, one E8M0 power-of-two scale per 32 values, no
+ * tensor scale; scale = smallest 2^e with 6 * 2^e >= block amax (reading),
+ * e in [-127, 127].  k % 32 == 0.  Scales in the 128 x 4 tile layout with
+ * orc_mx_scale_cols(k) = k/32 rounded up to 4 columns.                      */
+int64_t orc_mx_scale_cols(int64_t k);
+uint8_t orc_e8m0_block_scale(double bamax);
+double  orc_e8m0_decode(uint8_t b);
+int orc_quantize_1d_mx(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
+                       uint8_t* codes, uint8_t* sf);
+void orc_dequantize_mx(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t k, double* out);
+
 int orc_num_threads(void);
 
 #ifdef __cplusplus
