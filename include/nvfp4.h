@@ -272,6 +272,45 @@ nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scale
                                   const float* b_global, void* c, int64_t n, int64_t k,
                                   int64_t total_rows, void* workspace, void* stream);
 
+/* ---- MXFP4: the other four-bit format of the same tensor cores --------------
+ * "What is NVFP4? 4-bit AI inference on NVIDIA Blackwell explained", "NVFP4
+ * versus MXFP4"; "NVFP4 Explained", "Why Blocks of 16 Improve Accuracy" and
+ * "Why the Block Scale Uses FP8 E4M3": the same E2M1 elements and nibble
+ * packing, one E8M0 scale (a power of two, 2^(byte - 127)) per 32 values
+ * along k, and no tensor-wide scale.  Scale bytes use the 128 x 4 tile layout
+ * of the NVFP4 scales with one column per 32 values; pad bytes are 0. */
+
+/* Bytes of the tiled E8M0 scale buffer of a [rows, k] MXFP4 tensor:
+ * ceil(rows / 128) * 128 * ceil(k / 128) * 4. */
+size_t mxfp4_scale_bytes(int64_t rows, int64_t k);
+
+/* mxfp4_quantize_act -- quantize a BF16 [rows, k] tensor (row stride ld
+ * elements) to MXFP4.  The pages do not say how the power of two is chosen;
+ * here it is the smallest 2^e with 6 * 2^e >= the block's largest magnitude
+ * (the block maximum never saturates), e clamped to [-127, 127]; a block of
+ * zeros takes byte 0.  code = E2M1 round-to-nearest-even of x / 2^e, sign kept.
+ * Activations and weights use the same call (blocks run along k).
+ *   codes  device, nvfp4_codes_bytes(rows, k) bytes.
+ *   scales device, mxfp4_scale_bytes(rows, k) bytes; every byte written.
+ * k % 32 == 0 (else NVFP4_ERR_UNSUPPORTED_SHAPE); x, codes, scales 16-byte
+ * aligned and ld % 8 == 0 (else NVFP4_ERR_MISALIGNED).  rows == 0 returns
+ * NVFP4_OK at once (pointers may be NULL).  One pass, one launch; no
+ * workspace.  The launch waits for the previous work on stream.  NaN/Inf
+ * inputs are outside the contract. */
+nvfp4_status_t mxfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_t ld,
+                                  uint8_t* codes, uint8_t* scales, void* stream);
+
+/* mxfp4_gemm -- C[m, n] = bf16_rn(sum_k (qa * 2^ea)(qw * 2^ew)) for MXFP4
+ * operands from mxfp4_quantize_act: A [m, k], B [n, k] (both K-major), C BF16
+ * with row stride ldc.  The same tensor-core kernels and tiling as nvfp4_gemm
+ * (the block-scaled MMA with UE8M0 scales, 32-element blocks), FP32
+ * accumulation.  Arguments, limits, errors and workspace as nvfp4_gemm
+ * (nvfp4_workspace_bytes(NVFP4_OP_GEMM, m, n, k, 0); NULL computes every tile
+ * whole), without the global scales. */
+nvfp4_status_t mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                          const uint8_t* b_scales, void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
+                          void* workspace, void* stream);
+
 /* ---- diagnostics ------------------------------------------------------------ */
 
 /* Synchronizes stream, then returns NVFP4_ERR_TIMEOUT if any kernel of this

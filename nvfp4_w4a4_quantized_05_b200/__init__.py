@@ -28,6 +28,7 @@ __all__ = [
     "nvfp4_probe_bounded_wait", "nvfp4_status_string", "nvfp4_version",
     "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
     "gemm_emit_scale", "quantize_act_scaled", "quantize_act_smooth",
+    "mxfp4_scale_bytes", "mxfp4_quantize_act", "mxfp4_gemm", "MXFP4Tensor", "quantize_mx", "gemm_mx",
     "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM", "OP_GEMM_EMIT_SCALE",
 ]
 
@@ -65,6 +66,9 @@ _SIGNATURES = {
     "nvfp4_quantize_act_scaled": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_act_smooth": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "mxfp4_scale_bytes": (_sz, [_i64, _i64]),
+    "mxfp4_quantize_act": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
+    "mxfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
     "nvfp4_get_last_device_error": (_i32, [_vp]),
     "nvfp4_set_wait_limit_ns": (_u64, [_u64]),
     "nvfp4_probe_cvt": (_i32, [_vp, _vp, _vp, _i64, _vp]),
@@ -180,6 +184,18 @@ def nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_code
                        total_rows, workspace=None, stream=0) -> int:
     return lib().nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_codes, b_scales,
                                     b_global, c, n, k, total_rows, workspace, stream)
+
+
+def mxfp4_scale_bytes(rows: int, k: int) -> int:
+    return int(lib().mxfp4_scale_bytes(rows, k))
+
+
+def mxfp4_quantize_act(x, rows, k, ld, codes, scales, stream=0) -> int:
+    return lib().mxfp4_quantize_act(x, rows, k, ld, codes, scales, stream)
+
+
+def mxfp4_gemm(a_codes, a_scales, b_codes, b_scales, c, ldc, m, n, k, workspace=None, stream=0) -> int:
+    return lib().mxfp4_gemm(a_codes, a_scales, b_codes, b_scales, c, ldc, m, n, k, workspace, stream)
 
 
 def nvfp4_get_last_device_error(stream=0) -> int:
@@ -395,6 +411,52 @@ def quantize_act_scaled(x, global_scale, out: Optional[NVFP4Tensor] = None) -> N
         out.global_scale = global_scale
         return out
     return NVFP4Tensor(codes, scales, global_scale, rows, k)
+
+
+@dataclass
+class MXFP4Tensor:
+    """An MXFP4-quantized [rows, k] tensor on the device (no global scale)."""
+    codes: "object"            # uint8 [rows, k/2]
+    scales: "object"           # uint8 E8M0, tiled scale layout, one column per 32 values
+    rows: int
+    k: int
+
+
+def quantize_mx(x, out: Optional[MXFP4Tensor] = None) -> MXFP4Tensor:
+    """MXFP4 quantization (E8M0 scale per 32 values along k) of a BF16
+    [rows, k] CUDA tensor; activations and weights alike."""
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along k")
+    rows, k = x.shape
+    dev = x.device
+    sbytes = mxfp4_scale_bytes(rows, k)
+    if out is not None:
+        if out.rows != rows or out.k != k or out.scales.numel() < sbytes:
+            raise ValueError("out does not match the input shape")
+        codes, scales = out.codes, out.scales
+    else:
+        codes = torch.empty((rows, k // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty(sbytes, dtype=torch.uint8, device=dev)
+    st = mxfp4_quantize_act(_ptr(x), rows, k, x.stride(0), _ptr(codes), _ptr(scales), _stream_ptr(torch, dev))
+    _check(st, "mxfp4_quantize_act")
+    return out if out is not None else MXFP4Tensor(codes, scales, rows, k)
+
+
+def gemm_mx(a: MXFP4Tensor, b: MXFP4Tensor, out=None):
+    """C[m, n] = A * B^T of two MXFP4 tensors, BF16 output."""
+    import torch
+    if a.k != b.k:
+        raise ValueError("k mismatch")
+    dev = a.codes.device
+    c = out if out is not None else torch.empty((a.rows, b.rows), dtype=torch.bfloat16, device=dev)
+    ws = _gemm_workspace(torch, dev, a.rows, b.rows, a.k)
+    st = mxfp4_gemm(_ptr(a.codes), _ptr(a.scales), _ptr(b.codes), _ptr(b.scales), _ptr(c), c.stride(0), a.rows,
+                    b.rows, a.k, _ptr(ws), _stream_ptr(torch, dev))
+    _check(st, "mxfp4_gemm")
+    return c
 
 
 def grouped_gemm(a: NVFP4Tensor, b_codes, b_scales, b_global, n: int, out=None):

@@ -107,6 +107,11 @@ extern "C" size_t nvfp4_scale_bytes(int64_t rows, int64_t k) {
     return (size_t)(round_up(rows, 128) * round_up(k / 16, 4));
 }
 
+extern "C" size_t mxfp4_scale_bytes(int64_t rows, int64_t k) {
+    if (rows < 0 || k < 0) return 0;
+    return (size_t)(round_up(rows, 128) * round_up(k / 32, 4));
+}
+
 extern "C" size_t nvfp4_grouped_scale_bytes(int64_t total_rows, int num_groups, int64_t k) {
     if (total_rows < 0 || num_groups < 1 || k < 0) return 0;
     return (size_t)(((total_rows + 127 * (int64_t)num_groups) / 128) * 128 * round_up(k / 16, 4));

@@ -222,13 +222,21 @@ struct Cfg {
 };
 
 // EMIT (plain form only): also fold max |C| and write C's global scale.
-template <class C, bool GROUPED, bool EMIT = false>
+// MX (plain form only): MXFP4 operands -- one UE8M0 scale per 32 elements, so a
+// k-tile of 256 holds two 512-byte scale chunks per 128-row block instead of
+// four, k-step j reads chunk j / 2 at byte pair 2 (j % 2), and there is no
+// global scale (C = bf16(acc)).
+template <class C, bool GROUPED, bool EMIT = false, bool MX = false>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
     constexpr int BN = C::BN, STAGES = C::STAGES, ACC = C::ACC, NSFB = C::NSFB;
     constexpr int CW = BN >= 32 ? 32 : 16;                   // epilogue column chunk
     constexpr uint32_t IDESC = idesc_mxf4nvf4(128, BN);
+    constexpr uint32_t IDESC_MX0 = idesc_mxf4_e8m0(128, BN, 0), IDESC_MX2 = idesc_mxf4_e8m0(128, BN, 2);
+    constexpr int SF_KT = MX ? 1024 : 2048;      // scale bytes of one k-tile per 128-row block
+    constexpr int NCH = MX ? 2 : 4;              // 512-byte scale chunks per k-tile
+    static_assert(!(MX && (GROUPED || EMIT)), "MXFP4: plain form only");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -327,18 +335,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                         break;
                     }
                     const int nat = min(4, p.num_ks - kt * 4);
+                    const uint32_t nch = MX ? (uint32_t)(nat + 1) / 2 : (uint32_t)nat;   // scale chunks used
                     uint8_t* sA = smem + stage * C::STAGE_BYTES;
                     uint8_t* sB = sA + C::A_BYTES;
                     uint8_t* sSFA = sB + C::B_BYTES;
                     uint8_t* sSFB = sSFA + C::SFA_BYTES;
                     uint64_t* bar = &tail->full[stage];
-                    mbar_arrive_expect_tx(bar, C::A_BYTES + C::B_BYTES + (uint32_t)nat * 512u * (1u + (uint32_t)nsfb));
+                    mbar_arrive_expect_tx(bar, C::A_BYTES + C::B_BYTES + nch * 512u * (1u + (uint32_t)nsfb));
                     tma_load_2d(sA, &tmA, bar, kt * 128, ti.a_row0);
                     tma_load_2d(sB, &tmB, bar, kt * 128, ti.b_row0);
-                    bulk_load(sSFA, sfa_src + (int64_t)kt * 2048, (uint32_t)nat * 512u, bar);
+                    bulk_load(sSFA, sfa_src + (int64_t)kt * SF_KT, nch * 512u, bar);
                     for (int rb = 0; rb < nsfb; ++rb)
-                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * 2048,
-                                  (uint32_t)nat * 512u, bar);
+                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * SF_KT,
+                                  nch * 512u, bar);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -376,9 +385,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t sA = smem_u32(smem + stage * C::STAGE_BYTES);
                     const uint32_t sB = sA + C::A_BYTES;
                     const uint32_t sf = tmem + C::SF_BASE + sb * C::SF_STRIDE;
-                    for (int j = 0; j < nat; ++j)
-                        mma_mxf4nvf4(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32), IDESC,
-                                     sf + j * 4, sf + sfb_off + j * 4 * NSFB, (kt > 0 || j > 0) ? 1u : 0u);
+                    for (int j = 0; j < nat; ++j) {
+                        if constexpr (MX)
+                            mma_mxf4nvf4<true>(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
+                                               (j & 1) ? IDESC_MX2 : IDESC_MX0, sf + (j >> 1) * 4, sf + sfb_off + (j >> 1) * 4 * NSFB,
+                                               (kt > 0 || j > 0) ? 1u : 0u);
+                        else
+                            mma_mxf4nvf4(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
+                                         IDESC, sf + j * 4, sf + sfb_off + j * 4 * NSFB, (kt > 0 || j > 0) ? 1u : 0u);
+                    }
                     tc_commit(&tail->empty[stage]);
                     tc_commit(&tail->sf_empty[sb]);
                     if (++stage == STAGES) {
@@ -409,8 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // one k-tile of scales in tensor-memory column order: A k-step j at 4j,
                 // B k-step j, 128-row block rb at 16 + 4 * NSFB * j + 4 * rb
                 uint32_t w[C::SF_COLS];
+                if constexpr (MX) {   // chunks 2 and 3 are unused
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                    for (int i = 0; i < (int)C::SF_COLS; ++i) w[i] = 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < NCH; ++j) {
                     const uint4 v = ld_shared_v4(sSFA + j * 512 + lane * 16);
                     w[4 * j + 0] = v.x;
                     w[4 * j + 1] = v.y;
@@ -418,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     w[4 * j + 3] = v.w;
                 }
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < NCH; ++j)
 #pragma unroll
                     for (int rb = 0; rb < NSFB; ++rb) {
                         const uint4 v = ld_shared_v4(sSFB + rb * 2048 + j * 512 + lane * 16);
@@ -469,7 +488,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
-            const float alpha = __fmul_rn(p.ga[ti.group], p.gb[ti.group]);
+            const float alpha = MX ? 1.0f : __fmul_rn(p.ga[ti.group], p.gb[ti.group]);
             const bool a_ok = rloc < ti.a_rows;
             const bool use_tma = !GROUPED || q * 32 + 32 <= ti.a_rows;
 #pragma unroll 1
@@ -724,12 +743,17 @@ __device__ __forceinline__ PairTile pair_tile(const GemmArgs& p, const TAIL* tai
     return pt;
 }
 
-template <class P, bool GROUPED, bool EMIT = false>
+// MX: MXFP4 operands, as in gemm_kernel (plain form only).
+template <class P, bool GROUPED, bool EMIT = false, bool MX = false>
 __global__ void __launch_bounds__(P::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
     constexpr int BN = P::BN, BH = P::BH, STAGES = P::STAGES, NBC = P::NBC;
     constexpr uint32_t IDESC = idesc_mxf4nvf4(256, BN);
+    constexpr uint32_t IDESC_MX0 = idesc_mxf4_e8m0(256, BN, 0), IDESC_MX2 = idesc_mxf4_e8m0(256, BN, 2);
+    constexpr int SF_KT = MX ? 1024 : 2048;      // scale bytes of one k-tile per 128-row block
+    constexpr int NCH = MX ? 2 : 4;              // 512-byte scale chunks per k-tile
+    static_assert(!(MX && (GROUPED || EMIT)), "MXFP4: plain form only");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi_smem = smem + STAGES * P::STAGE_BYTES;
@@ -846,12 +870,13 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                     tma_load_2d_pair(sA, &tmA, full0, kt * 128, a_row);
                     tma_load_2d_pair(sB, &tmB, full0, kt * 128, g0);
                     uint64_t* sbar = &tail->sfl[stage];
-                    const uint32_t sbytes = (uint32_t)nat * 512u * ((sfa_ok ? 1u : 0u) + (uint32_t)nsfb);
+                    const uint32_t nch = MX ? (uint32_t)(nat + 1) / 2 : (uint32_t)nat;   // scale chunks used
+                    const uint32_t sbytes = nch * 512u * ((sfa_ok ? 1u : 0u) + (uint32_t)nsfb);
                     mbar_arrive_expect_tx(sbar, sbytes);
-                    if (sfa_ok) bulk_load(sSFA, sfa_src + (int64_t)kt * 2048, (uint32_t)nat * 512u, sbar);
+                    if (sfa_ok) bulk_load(sSFA, sfa_src + (int64_t)kt * SF_KT, nch * 512u, sbar);
                     for (int rb = 0; rb < nsfb; ++rb)
-                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * 2048,
-                                  (uint32_t)nat * 512u, sbar);
+                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * SF_KT,
+                                  nch * 512u, sbar);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -889,9 +914,16 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                     const uint32_t sA = smem_u32(smem + stage * P::STAGE_BYTES);
                     const uint32_t sB = sA + P::A_BYTES;
                     const uint32_t sf = tmem + P::SF_BASE + sb * P::SF_STRIDE;
-                    for (int j = 0; j < nat; ++j)
-                        mma_mxf4nvf4_pair(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
-                                          IDESC, sf + j * 4, sf + 16 + j * NBC, (kt > w.kb || j > 0) ? 1u : 0u);
+                    for (int j = 0; j < nat; ++j) {
+                        if constexpr (MX)
+                            mma_mxf4nvf4_pair<true>(d_tmem, sdesc_kmajor_sw128(sA + j * 32),
+                                                    sdesc_kmajor_sw128(sB + j * 32), (j & 1) ? IDESC_MX2 : IDESC_MX0,
+                                                    sf + (j >> 1) * 4, sf + 16 + (j >> 1) * NBC,
+                                                    (kt > w.kb || j > 0) ? 1u : 0u);
+                        else
+                            mma_mxf4nvf4_pair(d_tmem, sdesc_kmajor_sw128(sA + j * 32), sdesc_kmajor_sw128(sB + j * 32),
+                                              IDESC, sf + j * 4, sf + 16 + j * NBC, (kt > w.kb || j > 0) ? 1u : 0u);
+                    }
                     tc_commit_pair(&tail->empty[stage], 0x3);
                     tc_commit_pair(&tail->sf_free[sb], 0x3);
                     if (++stage == STAGES) {
@@ -934,8 +966,12 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                 // one k-tile of scales, in tensor-memory column order: A k-step j at
                 // 4j, B k-step j at 16 + NBC * j (column c = tile rows 32c..32c+31)
                 uint32_t w[P::SF_COLS];
+                if constexpr (MX) {   // chunks 2 and 3 are unused
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                    for (int i = 0; i < (int)P::SF_COLS; ++i) w[i] = 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < NCH; ++j) {
                     const uint4 v = ld_shared_v4(sSFA + j * 512 + lane * 16);
                     w[4 * j + 0] = v.x;
                     w[4 * j + 1] = v.y;
@@ -943,7 +979,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
                     w[4 * j + 3] = v.w;
                 }
 #pragma unroll
-                for (int j = 0; j < 4; ++j)
+                for (int j = 0; j < NCH; ++j)
 #pragma unroll
                     for (int c = 0; c < NBC; ++c) {
                         // tile row 32c + lane of B: its 4 scales of k-step j
@@ -1040,7 +1076,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
             const int a_rows = pt.a_rows;
             const int b_cols = min(BN, p.rows_b - n0);
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + ab * BN;
-            const float alpha = __fmul_rn(p.ga[pt.group], p.gb[pt.group]);
+            const float alpha = MX ? 1.0f : __fmul_rn(p.ga[pt.group], p.gb[pt.group]);
             // One 32-column chunk (16 BF16 pairs per lane) through a staging box to C.
             auto store_chunk = [&](int ch, const uint32_t* w16) {
                 if (ch * 32 >= b_cols || q * 32 >= a_rows) return;   // uniform per warp
@@ -1218,10 +1254,10 @@ bool make_codes_map(CUtensorMap* map, const void* base, int64_t rows, int64_t ro
     return r == CUDA_SUCCESS;
 }
 
-template <class C, bool GROUPED, bool EMIT = false>
+template <class C, bool GROUPED, bool EMIT = false, bool MX = false>
 nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                       int grid, cudaStream_t s) {
-    auto kern = gemm_kernel<C, GROUPED, EMIT>;
+    auto kern = gemm_kernel<C, GROUPED, EMIT, MX>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -1324,10 +1360,10 @@ size_t sk_workspace_bytes(int clusters) {
     return kSkFlagsBytes + (size_t)clusters * 2 * 128 * PairUse::BN * sizeof(float);
 }
 
-template <bool GROUPED = false, bool EMIT = false>
+template <bool GROUPED = false, bool EMIT = false, bool MX = false>
 nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                            int clusters, cudaStream_t s) {
-    auto kern = gemm_pair_kernel<PairUse, GROUPED, EMIT>;
+    auto kern = gemm_pair_kernel<PairUse, GROUPED, EMIT, MX>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [&] {
@@ -1386,10 +1422,12 @@ __global__ void set_one_kernel(float* g) { g[0] = 1.0f; }
 
 // The dense GEMM.  c_amax / c_gscale (optional): also fold max |C| and write
 // the global scale of C for the next quantizer (see nvfp4_gemm_emit_scale).
+// mx: MXFP4 operands (E8M0 scales per 32 elements, no global scales; the
+// global-scale pointers are ignored and c_amax must be NULL).
 nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                          const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c, int64_t ldc,
                          int64_t m, int64_t n, int64_t k, void* workspace, uint32_t* c_amax, float* c_gscale,
-                         void* stream) {
+                         void* stream, bool mx = false) {
     if (m < 0 || n <= 0 || k <= 0 || ldc < n) return NVFP4_ERR_INVALID_ARGUMENT;
     if (k % 64 != 0 || m >= ((int64_t)1 << 31) || n >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -1401,15 +1439,21 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
         }
         return NVFP4_OK;
     }
-    if (!a_codes || !a_scales || !a_global || !b_codes || !b_scales || !b_global || !c)
+    if (mx) {
+        a_global = b_global = nullptr;
+        if (c_amax) return NVFP4_ERR_INVALID_ARGUMENT;
+    } else if (!a_global || !b_global) {
         return NVFP4_ERR_INVALID_ARGUMENT;
+    }
+    if (!a_codes || !a_scales || !b_codes || !b_scales || !c) return NVFP4_ERR_INVALID_ARGUMENT;
     if (!ptr_ok(a_codes) || !ptr_ok(a_scales) || !ptr_ok(b_codes) || !ptr_ok(b_scales) || !ptr_ok(c) ||
         (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(b_global) & 3u) || ldc % 8 != 0)
         return NVFP4_ERR_MISALIGNED;
     if (reinterpret_cast<uintptr_t>(workspace) & 15u) return NVFP4_ERR_MISALIGNED;
     const int sms = num_sms();
     if (sms <= 0) return NVFP4_ERR_NO_DEVICE;
-    const int64_t sf_rb_stride = 128 * (k / 16);
+    // scale bytes per 128-row block: 128 rows x (k/16 or k/32 rounded up to 4) columns
+    const int64_t sf_rb_stride = mx ? 128 * round_up(k / 32, 4) : 128 * (k / 16);
     GemmArgs p = {};
     p.c_amax = c_amax;
     p.c_gscale = c_gscale;
@@ -1440,6 +1484,7 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
         p.tiles_m = 1;
         p.tiles_n = (int)((n + CfgDecW::BN - 1) / CfgDecW::BN);
         const int grid = (int)std::min<int64_t>((int64_t)p.tiles_n, sms);
+        if (mx) return launch<CfgDecW, false, false, true>(ta, tb, tc, p, grid, s);
         return c_amax ? launch<CfgDecW, false, true>(ta, tb, tc, p, grid, s) : launch<CfgDecW, false>(ta, tb, tc, p, grid, s);
     }
     PairPlan pl;
@@ -1463,6 +1508,7 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
         p.sk_units = sk ? pl.sk_units : 0;
         p.sk_flags = sk ? reinterpret_cast<uint32_t*>(workspace) : nullptr;
         p.partial = sk ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + kSkFlagsBytes) : nullptr;
+        if (mx) return launch_pair<false, false, true>(ta, tb, tc, p, pl.clusters, s);
         return c_amax ? launch_pair<false, true>(ta, tb, tc, p, pl.clusters, s)
                       : launch_pair<false>(ta, tb, tc, p, pl.clusters, s);
     }
@@ -1482,6 +1528,7 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
     const int grid = (int)std::min<int64_t>(tiles, sms);
+    if (mx) return launch<CfgWide, false, false, true>(ta, tb, tc, p, grid, s);
     return c_amax ? launch<CfgWide, false, true>(ta, tb, tc, p, grid, s) : launch<CfgWide, false>(ta, tb, tc, p, grid, s);
 }
 }  // namespace
@@ -1492,6 +1539,13 @@ extern "C" nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sc
                                      int64_t ldc, int64_t m, int64_t n, int64_t k, void* workspace, void* stream) {
     return gemm_impl(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k, workspace, nullptr,
                      nullptr, stream);
+}
+
+extern "C" nvfp4_status_t mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const uint8_t* b_codes,
+                                     const uint8_t* b_scales, void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
+                                     void* workspace, void* stream) {
+    return gemm_impl(a_codes, a_scales, nullptr, b_codes, b_scales, nullptr, c, ldc, m, n, k, workspace, nullptr,
+                     nullptr, stream, true);
 }
 
 extern "C" nvfp4_status_t nvfp4_gemm_emit_scale(const uint8_t* a_codes, const uint8_t* a_scales,

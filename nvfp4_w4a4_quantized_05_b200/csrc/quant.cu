@@ -206,6 +206,34 @@ __device__ __forceinline__ void quantize_task(const uint4& v0, const uint4& v1, 
         *reinterpret_cast<uint32_t*>(scales + sf_tile_offset(srow, scol, scale_cols)) = word;
 }
 
+// MXFP4 form of the task: lanes 2i and 2i+1 hold the 32-value block i of
+// the 512 values (16 each).  Its E8M0 byte is e + 127 for the smallest e with
+// 6 * 2^e >= the block maximum, read off the maximum's FP32 bits: for
+// m * 2^E (1 <= m < 2), e = E - 2 when m <= 1.5, else E - 1; e is clamped to
+// -127 (byte 0), which also covers zero and subnormal maxima.  The codes are
+// E2M1(x * 2^-e): 2^-e is a normal FP32 power of two, so each product is x / 2^e
+// rounded only where it falls far below the smallest E2M1 step.  Lanes 8j
+// store the scale word of blocks 4j..4j+3 (scale columns seg * 16 + 4j + i).
+__device__ __forceinline__ void quantize_task_mx(const uint4& v0, const uint4& v1, bool row_ok, int seg, int lane,
+                                                 int k, int scale_cols, uint8_t* code_row, uint8_t* scales, int srow) {
+    const uint32_t h = absmax_bits(bmax_abs(absmax8_packed(v0), absmax8_packed(v1)));
+    const uint32_t fb = max(h, __shfl_xor_sync(kFull, h, 1)) << 16;   // block maximum, FP32 bits
+    const int eb = max(0, (int)(fb >> 23) - 2 + ((fb & 0x7FFFFFu) > 0x400000u ? 1 : 0));
+    const int col = seg * 512 + lane * 16;
+    if (row_ok && col < k) {
+        const uint64_t rr = pack_rr(__uint_as_float((uint32_t)(254 - eb) << 23));   // 2^-e
+        uint2 q;
+        q.x = quant8(v0, rr);
+        q.y = quant8(v1, rr);
+        *reinterpret_cast<uint2*>(code_row + col / 2) = q;
+    }
+    const uint32_t p = (uint32_t)eb | (__shfl_down_sync(kFull, (uint32_t)eb, 2) << 8);
+    const uint32_t word = p | (__shfl_down_sync(kFull, p, 4) << 16);
+    const int scol = seg * 16 + (lane >> 1);
+    if ((lane & 7) == 0 && scol < scale_cols)
+        *reinterpret_cast<uint32_t*>(scales + sf_tile_offset(srow, scol, scale_cols)) = word;
+}
+
 // Exclusive prefix over groups of round128(group rows), by one CTA.
 __device__ void write_pad_rows(const Groups& gr, int num_groups, int32_t* pad_rows) {
     __shared__ int part[kThreads];
@@ -357,6 +385,8 @@ __device__ __forceinline__ void load_block16(const Quant1dArgs& a, int r0, int n
     }
 }
 
+// MX: the MXFP4 task (one tensor, no global scale; gscale unused).
+template <bool MX = false>
 __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
     const int e = blockIdx.y;
     int r0, r1;
@@ -389,19 +419,26 @@ __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
 
     pdl_wait();   // g (and the group scale offsets) come from amax_kernel
     const int srow0 = a.pad_rows ? a.pad_rows[e] : 0;
-    const float g = a.gscale[e];
     __shared__ uint64_t rtab[128];
-    fill_rtab(rtab, g, threadIdx.x);
-    const BlockQ c = make_blockq(g);
-    __syncthreads();
+    BlockQ c{};
+    if constexpr (!MX) {
+        const float g = a.gscale[e];
+        fill_rtab(rtab, g, threadIdx.x);
+        c = make_blockq(g);
+        __syncthreads();
+    }
 
     while (tp[0].row < prows) {
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
             const TaskPos t = tp[u];
             if (t.row >= prows) break;   // uniform across the warp
-            quantize_task(v[u][0], v[u][1], t.row < nrows, t.seg, lane, a.k, a.scale_cols,
-                          a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row, c, rtab);
+            if constexpr (MX)
+                quantize_task_mx(v[u][0], v[u][1], t.row < nrows, t.seg, lane, a.k, a.scale_cols,
+                                 a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row);
+            else
+                quantize_task(v[u][0], v[u][1], t.row < nrows, t.seg, lane, a.k, a.scale_cols,
+                              a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row, c, rtab);
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
@@ -1338,7 +1375,7 @@ extern "C" nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_
     const int qx = clamp_grid((per_group + kWarps * kQuantUnroll - 1) / (kWarps * kQuantUnroll),
                               (int64_t)num_sms() * 4 / groups);
     void* args[] = {&q};
-    return cuda_status(launch_pdl(reinterpret_cast<const void*>(&quant1d_kernel), dim3(qx, groups), dim3(kThreads),
+    return cuda_status(launch_pdl(reinterpret_cast<const void*>(&quant1d_kernel<false>), dim3(qx, groups), dim3(kThreads),
                                   args, s));
 }
 
@@ -1433,7 +1470,37 @@ extern "C" nvfp4_status_t nvfp4_quantize_act_scaled(const void* x, int64_t rows,
     // A plain launch: x may come from the previous kernel on the stream, whose
     // end this kernel must not overlap (its first loads precede its
     // griddepcontrol.wait, which returns at once without the launch attribute).
-    quant1d_kernel<<<dim3(qx, 1), kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(q);
+    quant1d_kernel<false><<<dim3(qx, 1), kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(q);
+    return cuda_status(cudaGetLastError());
+}
+
+extern "C" nvfp4_status_t mxfp4_quantize_act(const void* x, int64_t rows, int64_t k, int64_t ld, uint8_t* codes,
+                                             uint8_t* scales, void* stream) {
+    if (rows < 0 || k <= 0 || ld < k) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (rows == 0) return NVFP4_OK;   // nothing to read or write (the pointers may be NULL)
+    if (!x || !codes || !scales) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 32 != 0) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    const int64_t nseg = (k + 511) / 512;
+    if (rows * (k / 8) >= (int64_t)1 << 40 || round_up(rows, 128) * nseg >= ((int64_t)1 << 31) ||
+        rows >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || ld % 8 != 0) return NVFP4_ERR_MISALIGNED;
+    if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
+    Quant1dArgs q;
+    q.x = reinterpret_cast<const uint16_t*>(x);
+    q.ld = ld;
+    q.k = (int)k;
+    q.nseg = (int)nseg;
+    q.scale_cols = (int)(round_up(k / 32, 4));
+    q.groups.offsets = nullptr;
+    q.groups.rows = (int)rows;
+    q.pad_rows = nullptr;
+    q.gscale = nullptr;
+    q.codes = codes;
+    q.scales = scales;
+    const int64_t tasks = round_up(rows, 128) * q.nseg;
+    const int qx = clamp_grid((tasks + kWarps * kQuantUnroll - 1) / (kWarps * kQuantUnroll), (int64_t)num_sms() * 4);
+    quant1d_kernel<true><<<dim3(qx, 1), kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(q);
     return cuda_status(cudaGetLastError());
 }
 
