@@ -50,6 +50,13 @@ def quant_bytes(rows: int, k: int, groups: int = 1) -> int:
     return 2 * n + n // 2 + n // 16 + 4 * groups
 
 
+def mx_quant_bytes(rows: int, k: int) -> int:
+    """Algorithmic bytes of one MXFP4 quantizer call: read BF16 once, write
+    packed codes and one E8M0 scale per 32 values."""
+    n = rows * k
+    return 2 * n + n // 2 + n // 32
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -263,6 +270,29 @@ class Prefill:
             self.nv.quantize_act_scaled(self.c[j], gs[j], out=qc[j])
         return one_phase, two_phase
 
+    def mx_steps(self, nv, torch, w_host):
+        """The same workload in MXFP4: the activations quantized per call, the
+        weights quantized once (R rotating copies of each)."""
+        dev = self.a[0].device
+        wdev = to_device(torch, w_host, dev)
+        w0 = nv.quantize_mx(wdev)
+        del wdev
+        mw = [w0] + [nv.MXFP4Tensor(w0.codes.clone(), w0.scales.clone(), w0.rows, w0.k) for _ in range(self.R - 1)]
+        ma = [nv.quantize_mx(a) for a in self.a]
+
+        def quantize(i):
+            j = i % self.R
+            self.nv.quantize_mx(self.a[j], out=ma[j])
+
+        def gemm(i):
+            j = i % self.R
+            self.nv.gemm_mx(ma[j], mw[j], out=self.c[j])
+
+        def step(i):
+            quantize(i)
+            gemm(i)
+        return quantize, gemm, step
+
     def gemm_label(self):
         if self.m <= 64:
             return "gemm_kernel (tcgen05 mxf4nvf4; 64 token rows x 192 weight rows per tile)"
@@ -336,6 +366,13 @@ class Quant:
             g = np.random.default_rng(1)
             self.smooth = torch.from_numpy(np.exp2(g.uniform(-3.0, 3.0, self.k)).astype(np.float32)).to(self.a[0].device)
         self.nv.quantize_act_smooth(self.a[j], self.smooth, out=self.qa[j])
+
+    def quantize_mx(self, i):
+        """The same activations quantized to MXFP4 (one pass, E8M0 per 32)."""
+        j = i % self.R
+        if not hasattr(self, "mx"):
+            self.mx = [self.nv.quantize_mx(a) for a in self.a]
+        self.nv.quantize_mx(self.a[j], out=self.mx[j])
 
     def result(self, i):
         return self.qa[i % self.R].codes
@@ -721,6 +758,33 @@ def run_ours(args):
                                    "gbs": s_bytes / s_avg / 1e9, "frac_hbm": s_bytes / s_avg / 1e9 / peaks["hbm_gbs"],
                                    "avg_ms": s_avg * 1e3, "algorithmic_bytes": s_bytes,
                                    "kernels": "quant1d_fused_kernel (pre-scaled form)"}
+    if hasattr(wl, "quantize_mx"):
+        wl.quantize_mx(0)
+        time.sleep(REST_S)
+        x_avg = graph_seconds(torch, cs, wl.quantize_mx, wl.R, kiters)
+        x_bytes = mx_quant_bytes(wl.rows, wl.k)
+        line["mx_quantize"] = {"workload": "the same activations -> mxfp4 (E8M0 scale per 32 values, no tensor scale)",
+                               "gbs": x_bytes / x_avg / 1e9, "frac_hbm": x_bytes / x_avg / 1e9 / peaks["hbm_gbs"],
+                               "avg_ms": x_avg * 1e3, "algorithmic_bytes": x_bytes,
+                               "kernels": "quant1d_kernel (MXFP4 form, one pass)"}
+    if isinstance(wl, Prefill):
+        import workloads as W
+        w_host = W.prefill(0, wl.m, wl.n, wl.k)[1] if type(wl) is Prefill else W.decode(wl.m)[1]
+        mq, mg, ms = wl.mx_steps(nv, torch, w_host)
+        del w_host
+        time.sleep(REST_S)
+        xq = graph_seconds(torch, cs, mq, wl.R, kiters)
+        time.sleep(REST_S)
+        xg = graph_seconds(torch, cs, mg, wl.R, kiters)
+        time.sleep(REST_S)
+        xs = graph_seconds(torch, cs, ms, wl.R, kiters)
+        xq_bytes = mx_quant_bytes(wl.m, wl.k)
+        line["mxfp4"] = {
+            "what": "the same shapes in MXFP4: activations quantized per call (E8M0 per 32), weights pre-quantized",
+            "quantize_ms": xq * 1e3, "quantize_gbs": xq_bytes / xq / 1e9,
+            "gemm_ms": xg * 1e3, "gemm_tflops": wl.flops / xg / 1e12,
+            "gemm_frac_fp4_peak": wl.flops / xg / 1e12 / fp4_peak, "step_ms": xs * 1e3,
+            "kernels": "quant1d_kernel (MXFP4 form) + " + wl.gemm_label().replace("mxf4nvf4", "mxf4nvf4 block32")}
     if type(wl) is Prefill:
         one_phase, two_phase = wl.next_layer_steps(nv, torch)
         time.sleep(REST_S)
