@@ -307,6 +307,13 @@ def gemm_f64_rows(a_hat: np.ndarray, w_hat: np.ndarray, rows) -> np.ndarray:
     return c
 
 
+def gemm_w4a16_f64(a_bf16: np.ndarray, w_codes, w_sf, w_g: float) -> np.ndarray:
+    """W4A16: BF16 activations (exact in binary64) times the reconstructed NVFP4
+    weights, C = A * W_hat^T in binary64 ("W4A8 vs NVFP4 quantization on GPUs",
+    weight-only quantization: only the weights are four-bit)."""
+    return gemm_f64(bf16_to_f64(a_bf16), dequantize(w_codes, w_sf, w_g))
+
+
 def gemm_exact_i64(a_codes, a_sf, w_codes, w_sf, k: int) -> np.ndarray:
     """sum_k (qa*sfa)(qw*sfw) * 2^20 as exact int64 (global scales excluded)."""
     a_codes = np.ascontiguousarray(a_codes, dtype=np.uint8)
