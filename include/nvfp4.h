@@ -311,6 +311,27 @@ nvfp4_status_t mxfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
                           const uint8_t* b_scales, void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
                           void* workspace, void* stream);
 
+/* ---- W4A16: BF16 activations x NVFP4 weights, for decode-sized m --------------
+ * The weight-only alternative that "W4A8 vs NVFP4 quantization on GPUs"
+ * ("Batch size can change the winner", "Dequantization can erase a four-bit
+ * win") weighs against W4A4 at small batch: the same NVFP4 weight stream, the
+ * activations kept in BF16, the weights dequantized to BF16 inside the kernel
+ * (E2M1 x E4M3, exact) and multiplied on the BF16 tensor cores.
+ *
+ * w4a16_gemm -- C[m, n] = bf16_rn(b_global * sum_k a[m][k] * (qw[n][k] * sfw)),
+ * FP32 accumulation.
+ *   a        device BF16 [m, k], row stride lda elements (lda >= k, lda % 8 == 0).
+ *   b_codes, b_scales, b_global: NVFP4 weights [n, k] as for nvfp4_gemm (1D or
+ *            2D scales), global scale device FP32 [1].
+ *   c        device BF16 [m, n], row stride ldc (ldc >= n, ldc % 8 == 0).
+ * 0 <= m <= 64 and k % 64 == 0 (else NVFP4_ERR_UNSUPPORTED_SHAPE); a, b_codes,
+ * b_scales, c 16-byte aligned (else NVFP4_ERR_MISALIGNED).  m == 0 returns
+ * NVFP4_OK at once (pointers may be NULL).  One launch, no workspace; bounded
+ * waits as nvfp4_gemm. */
+nvfp4_status_t w4a16_gemm(const void* a, int64_t lda, const uint8_t* b_codes, const uint8_t* b_scales,
+                          const float* b_global, void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
+                          void* stream);
+
 /* ---- diagnostics ------------------------------------------------------------ */
 
 /* Synchronizes stream, then returns NVFP4_ERR_TIMEOUT if any kernel of this

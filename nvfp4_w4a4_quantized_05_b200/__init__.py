@@ -29,6 +29,7 @@ __all__ = [
     "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
     "gemm_emit_scale", "quantize_act_scaled", "quantize_act_smooth",
     "mxfp4_scale_bytes", "mxfp4_quantize_act", "mxfp4_gemm", "MXFP4Tensor", "quantize_mx", "gemm_mx",
+    "w4a16_gemm", "gemm_w4a16",
     "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM", "OP_GEMM_EMIT_SCALE",
 ]
 
@@ -69,6 +70,7 @@ _SIGNATURES = {
     "mxfp4_scale_bytes": (_sz, [_i64, _i64]),
     "mxfp4_quantize_act": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "mxfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
+    "w4a16_gemm": (_i32, [_vp, _i64, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp]),
     "nvfp4_get_last_device_error": (_i32, [_vp]),
     "nvfp4_set_wait_limit_ns": (_u64, [_u64]),
     "nvfp4_probe_cvt": (_i32, [_vp, _vp, _vp, _i64, _vp]),
@@ -196,6 +198,10 @@ def mxfp4_quantize_act(x, rows, k, ld, codes, scales, stream=0) -> int:
 
 def mxfp4_gemm(a_codes, a_scales, b_codes, b_scales, c, ldc, m, n, k, workspace=None, stream=0) -> int:
     return lib().mxfp4_gemm(a_codes, a_scales, b_codes, b_scales, c, ldc, m, n, k, workspace, stream)
+
+
+def w4a16_gemm(a, lda, b_codes, b_scales, b_global, c, ldc, m, n, k, stream=0) -> int:
+    return lib().w4a16_gemm(a, lda, b_codes, b_scales, b_global, c, ldc, m, n, k, stream)
 
 
 def nvfp4_get_last_device_error(stream=0) -> int:
@@ -456,6 +462,25 @@ def gemm_mx(a: MXFP4Tensor, b: MXFP4Tensor, out=None):
     st = mxfp4_gemm(_ptr(a.codes), _ptr(a.scales), _ptr(b.codes), _ptr(b.scales), _ptr(c), c.stride(0), a.rows,
                     b.rows, a.k, _ptr(ws), _stream_ptr(torch, dev))
     _check(st, "mxfp4_gemm")
+    return c
+
+
+def gemm_w4a16(a, b: NVFP4Tensor, out=None):
+    """C[m, n] = A * dequant(B)^T with A a BF16 [m, k] CUDA tensor (m <= 64)
+    and B NVFP4 weights; BF16 output."""
+    import torch
+    if a.dtype != torch.bfloat16 or a.dim() != 2 or not a.is_cuda:
+        raise TypeError("a must be a 2-D bfloat16 CUDA tensor")
+    if a.stride(1) != 1:
+        raise ValueError("a must have unit stride along k")
+    m, k = a.shape
+    if k != b.k:
+        raise ValueError("k mismatch")
+    dev = a.device
+    c = out if out is not None else torch.empty((m, b.rows), dtype=torch.bfloat16, device=dev)
+    st = w4a16_gemm(_ptr(a), a.stride(0), _ptr(b.codes), _ptr(b.scales), _ptr(b.global_scale), _ptr(c), c.stride(0),
+                    m, b.rows, k, _stream_ptr(torch, dev))
+    _check(st, "w4a16_gemm")
     return c
 
 

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libnvfp4.so")
 STAMP = LIB + ".srchash"
-SOURCES = ["api.cu", "quant.cu", "gemm.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm.cu", "w4a16.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
