@@ -797,6 +797,18 @@ def run_ours(args):
             "note": "one phase: GEMM, then the one-launch quantizer (amax pass + quantize pass over C); two phase: "
                     "GEMM emitting C's global scale from its epilogue, then the quantize pass alone"}
     if isinstance(wl, Decode):
+        def w16(i):
+            j = i % wl.R
+            nv.gemm_w4a16(wl.a[j], wl.w[j], out=wl.c[j])
+        time.sleep(REST_S)
+        t16 = graph_seconds(torch, cs, w16, wl.R, kiters)
+        line["w4a16"] = {
+            "what": "the same decode GEMM as W4A16: activations kept in BF16, the same NVFP4 weights dequantized "
+                    "to BF16 in the kernel, BF16 tensor-core MMAs (no activation quantization)",
+            "gemm_ms": t16 * 1e3, "weight_stream_gbs": wl.wbytes / t16 / 1e9,
+            "frac_hbm": wl.wbytes / t16 / 1e9 / peaks["hbm_gbs"],
+            "w4a4_gemm_ms": g_avg * 1e3, "w4a4_step_ms": line["ms_per_step"],
+            "kernels": "w4a16_kernel (tcgen05 kind::f16, 64 token rows x 192 weight rows per tile)"}
         line["weight_stream"] = {"gbs": wl.wbytes / g_avg / 1e9, "frac_hbm": wl.wbytes / g_avg / 1e9 / peaks["hbm_gbs"],
                                  "bytes": wl.wbytes}
     line["e2e"] = e2e

@@ -10,13 +10,15 @@
 //                per step, E2M1 x E4M3 -> BF16 (exact: at most 6 significant
 //                bits, magnitudes 2^-10 .. 2688), written in the MMA's
 //                128-byte-swizzled K-major layout.  Warps 0 and 1 also drain
-//                the accumulator (tensor-memory lanes 0..63 = the tokens).
+//                the accumulator.
 //   warp 12      TMA producer: activation slices [64 tokens x 64] (BF16) and
 //                raw weight tiles [192 rows x 256 values] (FP4 codes, 128-byte
 //                swizzle) with their scale chunks (bulk copies).
-//   warp 13      MMA issuer (tcgen05.mma kind::f16, BF16 x BF16 -> FP32, M =
-//                128 token rows of which 64 are loaded, N = 192, K = 16) and
-//                tensor-memory owner.
+//   warp 13      MMA issuer (tcgen05.mma kind::f16, BF16 x BF16 -> FP32, M = 64
+//                token rows, N = 192 weight rows, K = 16) and tensor-memory
+//                owner.  With M = 64 the accumulator rows 16 q .. 16 q + 15 sit
+//                in tensor-memory lanes 32 q .. 32 q + 15, so dequantizing warps
+//                0..3 (one per lane quarter) drain it.
 // Every wait is bounded; on expiry the kernel sets the library's error word
 // and every role leaves its loop.
 #include <cuda.h>
@@ -33,7 +35,7 @@
 namespace nvfp4 {
 namespace {
 
-constexpr int kW16Tokens = 64;               // token rows loaded (the MMA's M is 128)
+constexpr int kW16Tokens = 64;               // token rows: the MMA's M
 constexpr int kW16BN = 192;                  // weight rows per tile
 constexpr int kW16DqWarps = 12;
 constexpr int kW16Threads = 32 * (kW16DqWarps + 2);
@@ -46,7 +48,7 @@ constexpr uint32_t kW16RBytes = kW16BN * 128;            // 192 rows x 256 FP4
 constexpr uint32_t kW16SfBytes = 2 * 2048;               // <= 2 row blocks x 4 chunks
 constexpr uint32_t kW16TmemCols = 256;
 constexpr uint32_t kW16IDesc =                           // kind::f16: F32 D, BF16 A and B, K-major
-    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kW16BN >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+    (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kW16BN >> 3) << 17) | ((uint32_t)(kW16Tokens >> 4) << 24);
 static_assert(kW16DqWarps * 32 == 2 * kW16BN, "one 32-value item per dequantizing thread per slice");
 
 struct W16Tail {
@@ -142,8 +144,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
     w4a16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmW, const W16Args p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    // layout: activation slices (the MMA reads 128 rows from each: the next 8 KB
-    // belong to the following buffer), dequantized slices, raw tiles, scales
+    // layout: activation slices, dequantized slices, raw tiles, scales
     uint8_t* sA = smem;
     uint8_t* sD = sA + kW16AStages * kW16ABytes;
     uint8_t* sR = sD + kW16DStages * kW16DBytes;
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             mbar_init(&tail->d_empty[s], 1);
         }
         mbar_init(&tail->acc_full, 1);
-        mbar_init(&tail->acc_empty, 2);
+        mbar_init(&tail->acc_empty, 4);
         tail->abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -265,7 +266,7 @@ __global__ void __launch_bounds__(kW16Threads, 1)
             if (!ok) w16_abort(tail, p.err);
         }
     } else {
-        // ---------------- dequantization (and, warps 0..1, the epilogue) ----------------
+        // ---------------- dequantization (and, warps 0..3, the epilogue) ----------------
         // Item of thread i per slice: weight row r = i % 192 of the tile, values
         // 32 h .. 32 h + 31 of the 64-wide slice (h = i / 192): one 16-byte
         // chunk of the raw tile, four 16-byte units of the dequantized slice.
@@ -328,14 +329,14 @@ __global__ void __launch_bounds__(kW16Threads, 1)
                     dph ^= 1u;
                 }
             }
-            if (warp < 2 && ok) {
-                // epilogue: tensor-memory lanes 32 warp + lane are token rows
+            if (warp < 4 && ok) {
+                // epilogue: lanes 32 warp .. 32 warp + 15 hold token rows 16 warp ..
                 if (!mbar_wait(&tail->acc_full, (uint32_t)it & 1u, limit) || tail->abort_flag) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const int tok = warp * 32 + lane;
+                const int tok = lane < 16 ? warp * 16 + lane : p.m;   // lanes 16..31: no row
                 const float gw = p.gb[0];
                 const int ncols = min(kW16BN, p.n - n0);
                 const uint32_t tq = tmem + ((uint32_t)(warp * 32) << 16);
