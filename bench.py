@@ -808,6 +808,7 @@ def run_ours(args):
             "gemm_ms": t16 * 1e3, "weight_stream_gbs": wl.wbytes / t16 / 1e9,
             "frac_hbm": wl.wbytes / t16 / 1e9 / peaks["hbm_gbs"],
             "w4a4_gemm_ms": g_avg * 1e3, "w4a4_step_ms": line["ms_per_step"],
+            "traffic": load_traffic("w4a16_decode"),
             "kernels": "w4a16_kernel (tcgen05 kind::f16, 64 token rows x 192 weight rows per tile)"}
         line["weight_stream"] = {"gbs": wl.wbytes / g_avg / 1e9, "frac_hbm": wl.wbytes / g_avg / 1e9 / peaks["hbm_gbs"],
                                  "bytes": wl.wbytes}
