@@ -86,9 +86,9 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
     return d;
 }
-__device__ __forceinline__ uint32_t or_sign(uint32_t v, uint32_t s) {   // v | (s & 0x80008000)
+__device__ __forceinline__ uint32_t or_byte_signs(uint32_t v, uint32_t s) {   // v | (s & 0x80808080)
     uint32_t d;
-    asm("lop3.b32 %0, %1, %2, 0x80008000, 0xF8;" : "=r"(d) : "r"(v), "r"(s));
+    asm("lop3.b32 %0, %1, %2, 0x80808080, 0xF8;" : "=r"(d) : "r"(v), "r"(s));
     return d;
 }
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
@@ -100,19 +100,23 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
 // Eight E2M1 codes (value e in bits 4e..4e+3) -> eight BF16 values times the
 // BF16 pair s2, as four packed pairs.  The magnitudes come from two byte tables
 // by prmt: BF16 high bytes 00 3F 3F 3F 40 40 40 40 and low bytes 00 00 80 C0
-// 00 40 80 C0 for 0, 0.5, 1, 1.5, 2, 3, 4, 6; the code's sign bit becomes the
-// BF16 sign bit.  Every product is exact.
+// 00 40 80 C0 for 0, 0.5, 1, 1.5, 2, 3, 4, 6.  The sign bits go into the high
+// bytes before they are interleaved with the low bytes: the sign of value 2i
+// is the top bit of byte i of w << 4, that of value 2i + 1 the top bit of byte
+// i of w, so one prmt gathers four of them onto the top bits of a word whose
+// bytes line up with a high-byte table result.  Every product is exact.
 __device__ __forceinline__ void dequant8(uint32_t w, uint32_t s2, uint32_t* out) {
     constexpr uint32_t kHi0 = 0x3F3F3F00u, kHi1 = 0x40404040u, kLo0 = 0xC0800000u, kLo1 = 0xC0804000u;
     const uint32_t mag = w & 0x77777777u;
     const uint32_t mag_hi = mag >> 16;
-    const uint32_t lo_a = prmt(kLo0, kLo1, mag), hi_a = prmt(kHi0, kHi1, mag);
-    const uint32_t lo_b = prmt(kLo0, kLo1, mag_hi), hi_b = prmt(kHi0, kHi1, mag_hi);
-    const uint32_t w4 = w << 4;   // the sign of code 2i at the top bit of byte i
-    out[0] = mul_bf16x2(or_sign(prmt(lo_a, hi_a, 0x5140), prmt(w4, w, 0x4000)), s2);
-    out[1] = mul_bf16x2(or_sign(prmt(lo_a, hi_a, 0x7362), prmt(w4, w, 0x5010)), s2);
-    out[2] = mul_bf16x2(or_sign(prmt(lo_b, hi_b, 0x5140), prmt(w4, w, 0x6020)), s2);
-    out[3] = mul_bf16x2(or_sign(prmt(lo_b, hi_b, 0x7362), prmt(w4, w, 0x7030)), s2);
+    const uint32_t w4 = w << 4;
+    const uint32_t lo_a = prmt(kLo0, kLo1, mag), lo_b = prmt(kLo0, kLo1, mag_hi);
+    const uint32_t hi_a = or_byte_signs(prmt(kHi0, kHi1, mag), prmt(w4, w, 0x5140));      // values 0..3
+    const uint32_t hi_b = or_byte_signs(prmt(kHi0, kHi1, mag_hi), prmt(w4, w, 0x7362));   // values 4..7
+    out[0] = mul_bf16x2(prmt(lo_a, hi_a, 0x5140), s2);
+    out[1] = mul_bf16x2(prmt(lo_a, hi_a, 0x7362), s2);
+    out[2] = mul_bf16x2(prmt(lo_b, hi_b, 0x5140), s2);
+    out[3] = mul_bf16x2(prmt(lo_b, hi_b, 0x7362), s2);
 }
 
 // Two E4M3 scale bytes (low byte first) -> FP32 values (exact).
