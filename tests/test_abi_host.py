@@ -18,14 +18,16 @@ def _declared_symbols():
         if fn.endswith(".h"):
             src = open(os.path.join(ROOT, "include", fn)).read()
             src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-            names += re.findall(r"\b(nvfp4_[a-z0-9_]+)\s*\(", src)
+            names += re.findall(r"^\s*(?:nvfp4_status_t|size_t|uint64_t|int|const char\s*\*)\s+([a-z][a-z0-9_]*)\s*\(",
+                                src, re.M)
     return sorted(set(names))
 
 
 def test_library_exports_every_declared_symbol():
     L = nv.lib()
     declared = _declared_symbols()
-    assert len(declared) >= 15
+    assert len(declared) >= 23
+    assert {"mxfp4_quantize_act", "mxfp4_gemm", "mxfp4_scale_bytes", "w4a16_gemm"} <= set(declared)
     missing = [n for n in declared if not hasattr(L, n)]
     assert not missing, missing
     assert set(declared) <= set(nv.__all__)
@@ -45,6 +47,8 @@ def test_size_helpers(rows, k):
     pr = (rows + 127) // 128 * 128
     pc = (k // 16 + 3) // 4 * 4
     assert nv.nvfp4_scale_bytes(rows, k) == pr * pc
+    if k % 32 == 0:
+        assert nv.mxfp4_scale_bytes(rows, k) == pr * ((k // 32 + 3) // 4 * 4)
 
 
 def test_grouped_scale_bound_covers_any_split():
@@ -75,3 +79,13 @@ def test_argument_errors_are_reported_before_launch():
     assert nv.nvfp4_gemm(8, 16, 16, 16, 16, 16, 16, 64, 16, 64, 128, None, 0) == 3   # misaligned
     assert nv.nvfp4_grouped_gemm(16, 16, 16, 16, 300, 16, 16, 16, 16, 64, 128, 10, None, 0) == 2
     assert nv.nvfp4_probe_cvt(0, 0, 0, 10, 0) == 1
+    # MXFP4 and W4A16 entry points
+    assert nv.mxfp4_quantize_act(0, 16, 256, 256, 16, 16, 0) == 1            # null input
+    assert nv.mxfp4_quantize_act(16, 16, 48, 48, 16, 16, 0) == 2             # k % 32
+    assert nv.mxfp4_quantize_act(16, 16, 256, 256, 8, 16, 0) == 3            # misaligned codes
+    assert nv.mxfp4_gemm(16, 16, 16, 16, 16, 64, 16, 64, 96, None, 0) == 2   # k % 64
+    assert nv.mxfp4_gemm(0, 16, 16, 16, 16, 64, 16, 64, 128, None, 0) == 1
+    assert nv.w4a16_gemm(16, 128, 16, 16, 16, 16, 64, 65, 64, 128, 0) == 2   # m above 64
+    assert nv.w4a16_gemm(16, 96, 16, 16, 16, 16, 64, 8, 64, 96, 0) == 2     # k % 64
+    assert nv.w4a16_gemm(0, 128, 16, 16, 16, 16, 64, 8, 64, 128, 0) == 1    # null activations
+    assert nv.w4a16_gemm(8, 128, 16, 16, 16, 16, 64, 8, 64, 128, 0) == 3    # misaligned activations
