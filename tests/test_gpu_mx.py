@@ -149,3 +149,33 @@ def test_mx_decode_workload():
     _sync()
     ref = O.gemm_f64(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
     assert_gemm_close(to_host_f64(c), ref, "mx decode")
+
+
+def test_mx_strided_input_zero_tensor_and_empty_gemm():
+    import torch
+    # a [300, 1088] view of a wider buffer (row stride 1152 elements)
+    xb = W.laplace_outliers_bf16((300, 1152), 0, 820, outlier_frac=0.01)
+    x = bf16_to_device(xb)[:, :1088]
+    q = nv.quantize_mx(x)
+    _sync()
+    oc, osf = O.quantize_1d_mx(np.ascontiguousarray(xb[:, :1088]))
+    assert np.array_equal(q.codes.cpu().numpy(), oc) and np.array_equal(q.scales.cpu().numpy(), osf)
+    # all-zero tensor: zero codes, zero scale bytes
+    z = nv.quantize_mx(torch.zeros((130, 256), dtype=torch.bfloat16, device="cuda"))
+    _sync()
+    assert not z.codes.any() and not z.scales.any()
+    # empty GEMM and a GEMM into a strided output
+    w = W.gaussian_bf16((96, 256), 0, 821, 0.02)
+    wc, wsf = O.quantize_1d_mx(w)
+    tw = _mx_from_host(wc, wsf)
+    ta0 = nv.MXFP4Tensor(torch.empty((0, 128), dtype=torch.uint8, device="cuda"),
+                         torch.empty(0, dtype=torch.uint8, device="cuda"), 0, 256)
+    c0 = nv.gemm_mx(ta0, tw)
+    a = W.gaussian_bf16((40, 256), 0, 822, 1.0)
+    ac, asf = O.quantize_1d_mx(a)
+    out = torch.full((40, 104), 7.0, dtype=torch.bfloat16, device="cuda")
+    nv.gemm_mx(_mx_from_host(ac, asf), tw, out=out[:, :96])
+    _sync()
+    assert c0.shape == (0, 96)
+    assert_gemm_close(to_host_f64(out[:, :96]), O.gemm_f64(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf)), "mx strided")
+    assert torch.all(out[:, 96:] == 7.0)

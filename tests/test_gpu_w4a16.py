@@ -64,3 +64,14 @@ def test_w4a16_decode_workload(m):
     _sync()
     assert np.array_equal(tw.codes.cpu().numpy(), wc)
     assert_gemm_close(to_host_f64(c), O.gemm_w4a16_f64(a, wc, wsf, gw), f"w4a16 decode m={m}")
+
+
+def test_w4a16_strided_activations():
+    """Activations as a [48, 512] view of a [48, 640] buffer (row stride 640)."""
+    m, n, k = 48, 400, 512
+    a_full = W.gaussian_bf16((m, 640), 0, 980, 1.0, outlier_frac=0.01)
+    wc, wsf, gw = O.quantize_1d(W.gaussian_bf16((n, k), 0, 981, 0.02))
+    c = nv.gemm_w4a16(bf16_to_device(a_full)[:, :k], nvfp4_from_host(wc, wsf, gw))
+    _sync()
+    ref = O.gemm_w4a16_f64(np.ascontiguousarray(a_full[:, :k]), wc, wsf, gw)
+    assert_gemm_close(to_host_f64(c), ref, "w4a16 strided activations")
