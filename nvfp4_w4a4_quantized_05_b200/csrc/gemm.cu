@@ -1258,12 +1258,8 @@ template <class C, bool GROUPED, bool EMIT = false, bool MX = false>
 nvfp4_status_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                       int grid, cudaStream_t s) {
     auto kern = gemm_kernel<C, GROUPED, EMIT, MX>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::SMEM);
-    });
-    if (attr_err != cudaSuccess) return NVFP4_ERR_CUDA;
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!smem_attr_on_device(reinterpret_cast<const void*>(kern), (int)C::SMEM, attr_done)) return NVFP4_ERR_CUDA;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -1364,12 +1360,9 @@ template <bool GROUPED = false, bool EMIT = false, bool MX = false>
 nvfp4_status_t launch_pair(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tc, const GemmArgs& args,
                            int clusters, cudaStream_t s) {
     auto kern = gemm_pair_kernel<PairUse, GROUPED, EMIT, MX>;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [&] {
-        attr_err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPairSmem<GROUPED>);
-    });
-    if (attr_err != cudaSuccess) return NVFP4_ERR_CUDA;
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!smem_attr_on_device(reinterpret_cast<const void*>(kern), (int)kPairSmem<GROUPED>, attr_done))
+        return NVFP4_ERR_CUDA;
     cudaLaunchAttribute attr[2];
     cudaLaunchConfig_t cfg = pair_config<GROUPED>(clusters, s, attr);
     return cuda_status(cudaLaunchKernelEx(&cfg, kern, ta, tb, tc, args));

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <atomic>
 #include <cstdint>
 
 #include "../../include/nvfp4.h"
@@ -25,6 +26,19 @@ size_t gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 // nvfp4_gemm_emit_scale's workspace: its output-amax words first, then the
 // plain GEMM's workspace.
 constexpr int64_t kEmitScaleWsBytes = 256;
+
+// Raises a kernel's dynamic shared-memory limit to `bytes` on the current
+// device, once per device (the attribute belongs to the device's context);
+// `done` holds one bit per device.  False if the runtime refuses it.
+inline bool smem_attr_on_device(const void* kernel, int bytes, std::atomic<unsigned long long>& done) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const unsigned long long bit = 1ull << dev;
+    if (done.load(std::memory_order_acquire) & bit) return true;
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) return false;
+    done.fetch_or(bit, std::memory_order_acq_rel);
+    return true;
+}
 
 // Current limit of the bounded waits, in ns.
 uint64_t wait_limit_ns();

@@ -27,7 +27,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <mutex>
 
 #include "internal.h"
 #include "ptx.cuh"
@@ -436,12 +435,9 @@ extern "C" nvfp4_status_t w4a16_gemm(const void* a, int64_t lda, const uint8_t* 
     p.wait_limit_ns = wait_limit_ns();
     p.err = device_error_word();
     if (!p.err) return NVFP4_ERR_CUDA;
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-        attr_err = cudaFuncSetAttribute(w4a16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kW16Smem);
-    });
-    if (attr_err != cudaSuccess) return NVFP4_ERR_CUDA;
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!smem_attr_on_device(reinterpret_cast<const void*>(&w4a16_kernel), (int)kW16Smem, attr_done))
+        return NVFP4_ERR_CUDA;
     const int grid = std::min(p.tiles, sms);
     w4a16_kernel<<<grid, kW16Threads, kW16Smem, reinterpret_cast<cudaStream_t>(stream)>>>(ta, tw, p);
     return cuda_status(cudaGetLastError());
