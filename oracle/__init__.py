@@ -11,7 +11,12 @@ Parity pins (tests/test_oracle_*.py): E2M1 magnitudes from the pages; encoders
 against brute-force nearest search; exactly representable round trips with
 the global scale of Figure 1 of "Accelerating large language models with NVFP4
 quantization"; the 4.5 bits/value storage rule; the outlier-error claim; the
-GEMM against an exact integer sum and a library matmul.  The scale-tile
+GEMM against an exact integer sum and a library matmul; the given-scale and
+pre-scaled quantizers against the plain one on exactly scaled inputs; the
+MXFP4 scale choice as a property over every BF16 magnitude, its round trip,
+nearest codes and 4.25 bits/value, and NVFP4's lower error on outliers; the
+W4A16 product against one-hot rows, the W4A4 product and a library matmul
+(tests/test_oracle_mx.py, tests/test_oracle_w4a16.py).  The scale-tile
 layout is not on the pages: its parity is pinned only through the GPU GEMM
 (tensor cores read it), so on the CPU it is "parity unpinned".
 """

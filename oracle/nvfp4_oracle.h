@@ -33,8 +33,15 @@
  *   scales stored in 128-row x 4-column tiles of 512 bytes (tensor-core
  *   block-scale layout), pad bytes zero.
  *
+ * Also: the quantize steps with g given (two-phase form); the quantizer of
+ * x * s[column] (per-column pre-scaling, one binary32 product); MXFP4 --
+ * "What is NVFP4?", "NVFP4 versus MXFP4": E2M1 codes, one E8M0 power-of-two
+ * scale per 32 values, no tensor scale, the power read as the smallest 2^e
+ * with 6 * 2^e >= block amax.
+ *
  * Every float operation is a single IEEE-754 binary32 operation rounded to
- * nearest even (built with -ffp-contract=off, no fast-math).
+ * nearest even (built with -ffp-contract=off, no fast-math); the MXFP4
+ * scaling x / 2^e is done in binary64, where it is exact.
  */
 #ifndef NVFP4_ORACLE_H
 #define NVFP4_ORACLE_H
