@@ -13,6 +13,10 @@ the global scale of Figure 1 of "Accelerating large language models with NVFP4
 quantization"; the 4.5 bits/value storage rule; the outlier-error claim; the
 GEMM against an exact integer sum and a library matmul; the given-scale and
 pre-scaled quantizers against the plain one on exactly scaled inputs; the
+block quantizer at tiny global scales, where 1 / d overflows binary32
+(exact constructions whose codes are known: the round trip at g = 2^-123 and
+blocks of v * 2^-130 at a rounded subnormal g); the single-scale baseline on
+worked examples (its scale amax / 6 and its ties to the even code); the
 MXFP4 scale choice as a property over every BF16 magnitude, its round trip,
 nearest codes and 4.25 bits/value, and NVFP4's lower error on outliers; the
 W4A16 product against one-hot rows, the W4A4 product and a library matmul

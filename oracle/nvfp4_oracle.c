@@ -12,7 +12,6 @@
  */
 #include "nvfp4_oracle.h"
 
-#include <float.h>
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
@@ -131,14 +130,35 @@ float orc_global_scale(float amax) {
 }
 
 /* One scale block: values xv[0..n), sharing block amax bamax.  Writes n codes
- * (unpacked, one per byte) and returns the E4M3 scale byte.                  */
+ * (unpacked, one per byte) and returns the E4M3 scale byte.
+ *
+ * Each code is the E2M1 value nearest x / d, d = decode(sf) * g, the divisor
+ * that the reconstruction fp4 x block_scale x global_scale implies ("NVFP4
+ * Explained", "How NVFP4 Represents a Value").  The quotient is formed as
+ * x * r with r = 1 / d, each rounded to binary32's 24-bit significand.  When
+ * 1 / d is too large for binary32 (d at or below 2^-128, so g below about
+ * 2^-119), the same two roundings are done one exponent range lower: d and x
+ * are first multiplied by 2^64, which leaves the quotient unchanged and is
+ * exact for d (d * 2^64 is a normal number).  x * 2^64 or the product can
+ * overflow only where x / d is far above 6, which saturates to 6 either way;
+ * with g from the tensor's own amax, x is below 2^-100 there and nothing
+ * overflows. */
 static uint8_t quantize_block(const float* xv, int n, float bamax, float g, uint8_t* code_out) {
+    const float two64 = 18446744073709551616.0f;   /* 2^64 */
     float k6 = 6.0f * g;
     uint8_t sf = orc_e4m3_encode(bamax / k6);
     float d = (float)orc_e4m3_decode(sf) * g;      /* decoded block scale times g */
-    float r = (d == 0.0f) ? 0.0f : 1.0f / d;
-    if (r > FLT_MAX) r = FLT_MAX;                   /* 1/d overflows only when g is subnormal */
-    for (int i = 0; i < n; ++i) code_out[i] = orc_e2m1_encode(xv[i] * r);
+    if (d == 0.0f) {                                /* zero block scale: every magnitude is 0 */
+        for (int i = 0; i < n; ++i) code_out[i] = orc_e2m1_encode(xv[i] * 0.0f);
+        return sf;
+    }
+    float r = 1.0f / d;
+    if (isinf(r)) {
+        float r64 = 1.0f / (d * two64);            /* r / 2^64 */
+        for (int i = 0; i < n; ++i) code_out[i] = orc_e2m1_encode((xv[i] * two64) * r64);
+    } else {
+        for (int i = 0; i < n; ++i) code_out[i] = orc_e2m1_encode(xv[i] * r);
+    }
     return sf;
 }
 

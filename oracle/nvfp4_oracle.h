@@ -27,8 +27,11 @@
  * Readings where the pages are silent (each listed in the design notes):
  *   g  = amax / (6 * 448) as a decode multiplier (1.0 when amax == 0);
  *   sf = E4M3_RNE_satfinite(block_amax / (6 * g));
- *   d  = decode(sf) * g;  r = (d == 0) ? 0 : min(1 / d, FLT_MAX);
- *   code = E2M1_RNE_satfinite(x * r), sign bit kept (also for zero);
+ *   d  = decode(sf) * g;  r = 1 / d (0 when d == 0);
+ *   code = E2M1_RNE_satfinite(x * r), sign bit kept (also for zero); r and
+ *   x * r are rounded to binary32's 24-bit significand without binary32's
+ *   exponent ceiling: where 1 / d overflows, d and x are scaled by 2^64
+ *   first, so the code stays the one nearest x / d;
  *   element 2i in bits 3:0 of byte i, element 2i+1 in bits 7:4;
  *   scales stored in 128-row x 4-column tiles of 512 bytes (tensor-core
  *   block-scale layout), pad bytes zero.

@@ -252,3 +252,101 @@ def test_smooth_quantizer_pins():
     assert np.array_equal(c4, c0) and np.array_equal(s4, s0) and g4 == g0 * 8
     with pytest.raises(ValueError):
         O.quantize_1d_smooth(x, np.zeros(512, np.float32))
+
+
+def _overflow_blocks(sf, g, rows, k):
+    """Blocks whose 1 / (decode(sf) g) overflows binary32."""
+    sfb = np.array([[sf[O.sf_offset(r, b, k)] for b in range(k // 16)] for r in range(rows)])
+    d = (np.array([O.e4m3_decode(c) for c in range(256)], np.float32)[sfb] * np.float32(g)).astype(np.float32)
+    with np.errstate(divide="ignore", over="ignore"):
+        return np.isinf(np.float32(1) / d[d != 0]).sum()
+
+
+@pytest.mark.parametrize("block_rows", [1, 16])
+def test_exact_round_trip_at_a_tiny_global_scale(block_rows):
+    """The exact construction at g = 2^-123 (Figure 1's 2^-8 moved down by
+    2^-115; every value stays exact in BF16, down to its smallest subnormal
+    2^-133).  Blocks with a block scale at or below 2^-5 have d <= 2^-128,
+    where 1 / d overflows binary32; their codes must still be the ones the
+    tensor was built from, because x / d is exactly a grid value ("NVFP4
+    Explained", "How NVFP4 Represents a Value").  Capping 1 / d at FLT_MAX
+    instead would shrink those codes by up to 2^4."""
+    g_tiny = 2.0 ** -123
+    rng = np.random.default_rng(5 + block_rows)
+    rows, k = (160, 96) if block_rows == 1 else (48, 96)
+    xb, x, want_codes, want_s = _build_exact(rng, rows, k, g_tiny, block_rows=block_rows)
+    if block_rows == 1:
+        codes, sf, g = O.quantize_1d(xb)
+    else:
+        codes, sf, g = O.quantize_2d(xb)
+    assert g == g_tiny
+    assert _overflow_blocks(sf, g, rows, k) > 0, "the construction must reach the overflow branch"
+    assert np.array_equal(_unpack(codes), want_codes)
+    for r in range(rows):
+        for b in range(k // 16):
+            assert sf[O.sf_offset(r, b, k)] == want_s[r // block_rows, b]
+    assert np.array_equal(O.dequantize(codes, sf, g), x)
+    if block_rows == 1:
+        c2, s2 = O.quantize_1d_given_g(xb, g_tiny)
+        assert np.array_equal(c2, codes) and np.array_equal(s2, sf)
+
+
+def test_codes_known_by_construction_at_a_rounded_subnormal_global_scale():
+    """x = v D with D = 2^-130 and v on the E2M1 grid; blocks peak at 6 D, 3 D
+    or 1.5 D.  Worked by hand: g = RN(6 D / 2688) = 1170 * 2^-149 (a rounded
+    subnormal), 6 g = 7020 * 2^-149 exactly, so the block-scale quotients are
+    448.1 (saturates to 448, byte 0x7E), 224.05 (-> 224, byte 0x76) and
+    112.03 (-> 112, byte 0x6E); d = 524160, 262080 and 131040 times 2^-149,
+    all below 2^-128.  x / d is then v, 2 v and 4 v times (1 + 2.4e-4), whose
+    nearest codes are v, 2 v and 4 v."""
+    D = 2.0 ** -130
+    rng = np.random.default_rng(9)
+    rows, k = 24, 96
+    peaks = {6.0: (1, 0x7E), 3.0: (2, 0x76), 1.5: (4, 0x6E)}
+    mag = np.zeros((rows, k))
+    want_mag = np.zeros((rows, k))
+    want_s = np.zeros((rows, k // 16), np.uint8)
+    for r in range(rows):
+        for b in range(k // 16):
+            peak = [6.0, 3.0, 1.5][(r + b) % 3]
+            mult, byte = peaks[peak]
+            allowed = GRID[GRID <= peak]
+            vals = rng.choice(allowed, 16)
+            vals[rng.integers(16)] = peak
+            mag[r, b * 16:(b + 1) * 16] = vals
+            want_mag[r, b * 16:(b + 1) * 16] = vals * mult
+            want_s[r, b] = byte
+    mag[0, :16] = 6.0                                      # the tensor amax is 6 D
+    want_mag[0, :16] = 6.0
+    want_s[0, 0] = 0x7E
+    sign = rng.integers(0, 2, size=(rows, k))
+    x = mag * D * np.where(sign == 1, -1.0, 1.0)
+    xb = W.to_bf16_bits(x.astype(np.float32))
+    assert np.array_equal(W.bf16_bits_to_f32(xb).astype(np.float64), x)
+    codes, sf, g = O.quantize_1d(xb)
+    assert np.float32(g).view(np.uint32) == 1170             # 1170 * 2^-149
+    assert _overflow_blocks(sf, g, rows, k) == rows * k // 16
+    want_codes = np.searchsorted(GRID, want_mag) | (sign << 3)
+    want_codes = np.where(mag == 0, sign << 3, want_codes)   # a signed zero keeps its sign bit
+    assert np.array_equal(_unpack(codes), want_codes)
+    for r in range(rows):
+        for b in range(k // 16):
+            assert sf[O.sf_offset(r, b, k)] == want_s[r, b]
+
+
+def test_single_scale_baseline_worked_examples():
+    """One scale amax / 6 for the whole tensor, codes rounded to the nearest
+    E2M1 value with ties to the even code ("NVFP4 Explained", "Why Blocks of 16
+    Improve Accuracy": one scale over many values lets the outlier set it).
+    [0.5, 1, 60]: scale 10, quotients 0.05, 0.1, 6 -> 0, 0, 6 -> [0, 0, 60].
+    amax 6 (scale 1) with every tie of the grid: 0.25 -> 0, 0.75 -> 1,
+    1.25 -> 1, 1.75 -> 2, 2.5 -> 2, 3.5 -> 4, 5 -> 4; the sign is kept."""
+    x = np.array([0.5, 1.0, 60.0], np.float32)
+    assert np.array_equal(O.single_scale_fp4(W.to_bf16_bits(x)), [0.0, 0.0, 60.0])
+    t = np.array([6, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, -5, -1.75, 0.5], np.float32)
+    want = [6, 0, 1, 1, 2, 2, 4, 4, -4, -2, 0.5]
+    assert np.array_equal(O.single_scale_fp4(W.to_bf16_bits(t)), want)
+    # amax 12 (scale 2): every value is halved before rounding, then doubled back
+    assert np.array_equal(O.single_scale_fp4(W.to_bf16_bits(np.array([12, 1.5, -2.5, 7], np.float32))),
+                          [12, 2, -2, 8])
+    assert not O.single_scale_fp4(np.zeros(4, np.uint16)).any()
