@@ -8,8 +8,13 @@
 //   g    = amax / (6 * 448)  (1 if amax == 0)   FP32 global decode scale
 //   per 16-element block (1D) or 16x16 tile (2D), kernel 2:
 //     sf   = e4m3_rn_satfinite(block_amax / (6 g))
-//     d    = float(sf) * g ;  r = d == 0 ? 0 : min(1 / d, FLT_MAX)
+//     d    = float(sf) * g ;  r = d == 0 ? 0 : 1 / d
 //     code = e2m1_rn_satfinite(x * r)
+// r and x * r are rounded to binary32's 24-bit significand without binary32's
+// exponent ceiling, so each code is the one nearest x / d (the divisor that
+// the reconstruction fp4 x block_scale x global_scale implies) even where
+// 1 / d overflows: for a global scale below 2^-64 the kernels keep r / 2^32
+// and multiply each product back by 2^32, both steps exact (see block_recip).
 // Every step rounds as one IEEE binary32 operation to nearest even would
 // (compiled with -fmad=false), and the roundings to E4M3 / E2M1 are the
 // hardware cvt.rn.satfinite instructions, so the codes and scale bytes are
@@ -84,35 +89,58 @@ __device__ __forceinline__ uint32_t absmax_bits(uint32_t packed) {
     return max(m & 0xFFFFu, m >> 16);
 }
 
-// (lo, hi) BF16 pair times (r, r): two IEEE round-to-nearest products.
-__device__ __forceinline__ void mul_bf16x2(uint32_t w, uint64_t rr, float& lo, float& hi) {
-    uint64_t x, y;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w << 16), "r"(w & 0xFFFF0000u));
-    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(rr));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(y));
-}
 __device__ __forceinline__ uint64_t pack_rr(float r) {
     uint64_t rr;
     asm("mov.b64 %0, {%1, %1};" : "=l"(rr) : "f"(r));
     return rr;
 }
 
+// Global scales below this take the tiny form of r (block_recip).
+constexpr float kTinyG = 0x1p-64f;
+
+// r for a block with d = float(sf) g: RN(1 / d), 0 when d == 0.  With a tiny
+// global scale (g < 2^-64) it returns RN(1 / (d 2^32)) = RN(1 / d) / 2^32
+// instead, and the caller multiplies each product x * r by 2^32:
+//   - g >= 2^-64: d >= 2^-9 g >= 2^-73 (or 0), so 1 / d <= 2^73 never
+//     overflows and plain binary32 is the reading;
+//   - g < 2^-64: d < 448 * 2^-64, so d 2^32 is exact and normal (d >= 2^-149)
+//     and 1 / (d 2^32) lies in [2^23, 2^117], where binary32 rounds it as an
+//     unbounded exponent range would; RN(x * r / 2^32) * 2^32 equals that
+//     range's RN(x * r) whenever x * r >= 2^-94, and below that both give a
+//     signed zero code; a product that overflows is far above 6 and saturates
+//     to 6, as x / d would.
+__device__ __forceinline__ float block_recip(float d, bool tiny) {
+    if (d == 0.0f) return 0.0f;
+    return __frcp_rn(tiny ? __fmul_rn(d, 0x1p32f) : d);
+}
+
+// (lo, hi) BF16 pair times (r, r): two IEEE round-to-nearest products (TINY:
+// r holds r / 2^32 and both products are then multiplied by 2^32, exactly).
+template <bool TINY = false>
+__device__ __forceinline__ void mul_bf16x2(uint32_t w, uint64_t rr, float& lo, float& hi) {
+    uint64_t x, y;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(y) : "l"(x), "l"(rr));
+    if constexpr (TINY) asm("mul.rn.f32x2 %0, %0, %1;" : "+l"(y) : "l"(pack_rr(0x1p32f)));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(y));
+}
+
 // Eight BF16 values times r -> eight packed E2M1 codes.
+template <bool TINY = false>
 __device__ __forceinline__ uint32_t quant8(const uint4& v, uint64_t rr) {
     float x[8];
-    mul_bf16x2(v.x, rr, x[0], x[1]);
-    mul_bf16x2(v.y, rr, x[2], x[3]);
-    mul_bf16x2(v.z, rr, x[4], x[5]);
-    mul_bf16x2(v.w, rr, x[6], x[7]);
+    mul_bf16x2<TINY>(v.x, rr, x[0], x[1]);
+    mul_bf16x2<TINY>(v.y, rr, x[2], x[3]);
+    mul_bf16x2<TINY>(v.z, rr, x[4], x[5]);
+    mul_bf16x2<TINY>(v.w, rr, x[6], x[7]);
     return cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
 }
 
 // Block scale byte and element multiplier from the block amax (exact IEEE steps;
 // used by the 16 x 16 weight quantizer, where it runs once per 256 values).
-__device__ __forceinline__ uint32_t block_scale(float bamax, float g, float k6, float& r) {
+__device__ __forceinline__ uint32_t block_scale(float bamax, float g, float k6, bool tiny, float& r) {
     const uint32_t sf = cvt_e4m3(__fdiv_rn(bamax, k6));
-    const float d = __fmul_rn(e4m3_to_f32(sf), g);
-    r = (d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX);
+    r = block_recip(__fmul_rn(e4m3_to_f32(sf), g), tiny);
     return sf;
 }
 
@@ -163,15 +191,12 @@ __device__ __forceinline__ uint32_t block_sf2(float b0, float b1, const BlockQ& 
     return cvt_e4m3x2(__fdiv_rn(b1, c.k6), __fdiv_rn(b0, c.k6));
 }
 
-// rtab[sf] = (r, r) for a block with scale byte sf: d = float(sf) * g,
-// r = d == 0 ? 0 : min(1 / d, FLT_MAX), stored as the FP32 pair that the paired
-// multiplies take.  128 entries (bytes 0..127; 127 is never produced by the
-// saturating conversion).  Threads 0..127 fill it.
+// rtab[sf] = (r, r) for a block with scale byte sf: r = block_recip(float(sf) * g)
+// (r / 2^32 for a tiny g), stored as the FP32 pair that the paired multiplies
+// take.  128 entries (bytes 0..127; 127 is never produced by the saturating
+// conversion).  Threads 0..127 fill it.
 __device__ __forceinline__ void fill_rtab(uint64_t* rtab, float g, int tid) {
-    if (tid < 128) {
-        const float d = __fmul_rn(e4m3_to_f32((uint32_t)tid), g);
-        rtab[tid] = pack_rr((d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX));
-    }
+    if (tid < 128) rtab[tid] = pack_rr(block_recip(__fmul_rn(e4m3_to_f32((uint32_t)tid), g), g < kTinyG));
 }
 
 __device__ __forceinline__ int64_t sf_tile_offset(int srow, int scol, int scale_cols) {
@@ -188,15 +213,20 @@ __device__ __forceinline__ int64_t sf_tile_offset(int srow, int scol, int scale_
 // side by side without branches between them.
 __device__ __forceinline__ void quantize_task(const uint4& v0, const uint4& v1, bool row_ok, int seg, int lane,
                                               int k, int scale_cols, uint8_t* code_row, uint8_t* scales, int srow,
-                                              const BlockQ& c, const uint64_t* rtab, bool valid = true) {
+                                              const BlockQ& c, const uint64_t* rtab, bool tiny, bool valid = true) {
     const uint32_t am = absmax_bits(bmax_abs(absmax8_packed(v0), absmax8_packed(v1)));
     const uint32_t sf = block_sf(__uint_as_float(am << 16), c);
     const int col = seg * 512 + lane * 16;
     if (valid && row_ok && col < k) {
         const uint64_t rr = rtab[sf];
         uint2 q;
-        q.x = quant8(v0, rr);
-        q.y = quant8(v1, rr);
+        if (tiny) {   // uniform across the grid row: one global scale
+            q.x = quant8<true>(v0, rr);
+            q.y = quant8<true>(v1, rr);
+        } else {
+            q.x = quant8(v0, rr);
+            q.y = quant8(v1, rr);
+        }
         *reinterpret_cast<uint2*>(code_row + col / 2) = q;
     }
     const uint32_t p = sf | (__shfl_down_sync(kFull, sf, 1) << 8);
@@ -421,10 +451,12 @@ __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
     const int srow0 = a.pad_rows ? a.pad_rows[e] : 0;
     __shared__ uint64_t rtab[128];
     BlockQ c{};
+    bool tiny = false;
     if constexpr (!MX) {
         const float g = a.gscale[e];
         fill_rtab(rtab, g, threadIdx.x);
         c = make_blockq(g);
+        tiny = g < kTinyG;
         __syncthreads();
     }
 
@@ -438,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
                                  a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row);
             else
                 quantize_task(v[u][0], v[u][1], t.row < nrows, t.seg, lane, a.k, a.scale_cols,
-                              a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row, c, rtab);
+                              a.codes + (int64_t)(r0 + t.row) * kbytes, a.scales, srow0 + t.row, c, rtab, tiny);
         }
 #pragma unroll
         for (int u = 0; u < kQuantUnroll; ++u) {
@@ -648,9 +680,11 @@ __device__ __forceinline__ float4 smooth_unit(const float* seg_base, int lane, i
 }
 
 // Eight BF16 values, each times its column factor (x' = x s, one IEEE product),
-// then times r -> eight packed E2M1 codes.
+// then times r -> eight packed E2M1 codes (TINY: r / 2^32, then times 2^32).
+template <bool TINY>
 __device__ __forceinline__ uint32_t quant8_smooth(const uint4& v, const float4& s0, const float4& s1, uint64_t rr) {
     const float r = __uint_as_float((uint32_t)rr);
+    const float up = TINY ? 0x1p32f : 1.0f;
     float x[8];
     x[0] = __fmul_rn(__fmul_rn(__uint_as_float(v.x << 16), s0.x), r);
     x[1] = __fmul_rn(__fmul_rn(__uint_as_float(v.x & 0xFFFF0000u), s0.y), r);
@@ -660,6 +694,10 @@ __device__ __forceinline__ uint32_t quant8_smooth(const uint4& v, const float4& 
     x[5] = __fmul_rn(__fmul_rn(__uint_as_float(v.z & 0xFFFF0000u), s1.y), r);
     x[6] = __fmul_rn(__fmul_rn(__uint_as_float(v.w << 16), s1.z), r);
     x[7] = __fmul_rn(__fmul_rn(__uint_as_float(v.w & 0xFFFF0000u), s1.w), r);
+    if constexpr (TINY) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) x[i] = __fmul_rn(x[i], up);
+    }
     return cvt_e2m1x8(x[0], x[1], x[2], x[3], x[4], x[5], x[6], x[7]);
 }
 // max |x s| over the eight values of a unit.
@@ -674,28 +712,30 @@ __device__ __forceinline__ float absmax8_smooth(const uint4& v, const float4& s0
     return fmaxf(m, fabsf(__fmul_rn(__uint_as_float(v.w & 0xFFFF0000u), s1.w)));
 }
 
-// Per-group quantizer constants: the global scale g and the bracket constants.
+// Per-group quantizer constants: the global scale g, the bracket constants and
+// whether g takes the tiny form of r.
 struct GroupQ {
     float g;
+    bool tiny;
     BlockQ c;
 };
 __device__ __forceinline__ GroupQ make_groupq(uint32_t amax_fbits) {   // FP32 bits of the amax
     GroupQ q;
     const float amax = __uint_as_float(amax_fbits);
     q.g = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, kGlobalDen);
+    q.tiny = q.g < kTinyG;
     q.c = make_blockq(q.g);
     return q;
 }
-// (r, r) for scale byte sf, d = float(sf) g, r = d == 0 ? 0 : min(1 / d, FLT_MAX):
-// the same value the table of the one-tensor form holds.
-__device__ __forceinline__ uint64_t block_rr(uint32_t sf, float g) {
-    const float d = __fmul_rn(e4m3_to_f32(sf), g);
-    return pack_rr((d == 0.0f) ? 0.0f : fminf(__frcp_rn(d), FLT_MAX));
+// (r, r) for scale byte sf: the same value the table of the one-tensor form holds.
+__device__ __forceinline__ uint64_t block_rr(uint32_t sf, const GroupQ& q) {
+    return pack_rr(block_recip(__fmul_rn(e4m3_to_f32(sf), q.g), q.tiny));
 }
 
 // Quantize the task held in slot sb.  FULL: the whole task is inside the
 // tensor.  One tensor: r from the per-CTA table; grouped: r computed per block.
-template <bool FULL, bool GROUPED, bool SMOOTH>
+// TINY: the group's g takes the tiny form of r (block_recip).
+template <bool FULL, bool GROUPED, bool SMOOTH, bool TINY>
 __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
                                               const LaneC& lc, const GroupQ& gq, const uint64_t* rtab,
                                               const float* ssm) {
@@ -721,23 +761,23 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
     const uint32_t pair = block_sf2(b0, b1, gq.c);   // scale bytes of blocks 2 lane, 2 lane + 1
     uint64_t rr0, rr1;
     if constexpr (GROUPED) {
-        rr0 = block_rr(pair & 0xFFu, gq.g);
-        rr1 = block_rr(pair >> 8, gq.g);
+        rr0 = block_rr(pair & 0xFFu, gq);
+        rr1 = block_rr(pair >> 8, gq);
     } else {
         rr0 = rtab[pair & 0xFFu];
         rr1 = rtab[pair >> 8];
     }
     uint4 q;
     if constexpr (SMOOTH) {
-        q.x = quant8_smooth(u[0], sv[0], sv[1], rr0);
-        q.y = quant8_smooth(u[1], sv[2], sv[3], rr0);
-        q.z = quant8_smooth(u[2], sv[4], sv[5], rr1);
-        q.w = quant8_smooth(u[3], sv[6], sv[7], rr1);
+        q.x = quant8_smooth<TINY>(u[0], sv[0], sv[1], rr0);
+        q.y = quant8_smooth<TINY>(u[1], sv[2], sv[3], rr0);
+        q.z = quant8_smooth<TINY>(u[2], sv[4], sv[5], rr1);
+        q.w = quant8_smooth<TINY>(u[3], sv[6], sv[7], rr1);
     } else {
-        q.x = quant8(u[0], rr0);
-        q.y = quant8(u[1], rr0);
-        q.z = quant8(u[2], rr1);
-        q.w = quant8(u[3], rr1);
+        q.x = quant8<TINY>(u[0], rr0);
+        q.y = quant8<TINY>(u[1], rr0);
+        q.z = quant8<TINY>(u[2], rr1);
+        q.w = quant8<TINY>(u[3], rr1);
     }
     const uint32_t word = __byte_perm(pair, __shfl_down_sync(kFull, pair, 1), 0x5410);
     const bool even = (lc.lane & 1) == 0;
@@ -757,10 +797,15 @@ template <bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void quantize_any(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
                                              const LaneC& lc, const GroupQ& gq, const uint64_t* rtab,
                                              const float* ssm) {
-    if (t.valid() && t.seg < a.full_segs)
-        quantize_slot<true, GROUPED, SMOOTH>(a, sb, t, lc, gq, rtab, ssm);
-    else
-        quantize_slot<false, GROUPED, SMOOTH>(a, sb, t, lc, gq, rtab, ssm);
+    const bool full = t.valid() && t.seg < a.full_segs;
+    if (gq.tiny) {   // warp-uniform (one g per group): a global scale below 2^-64
+        if (full) quantize_slot<true, GROUPED, SMOOTH, true>(a, sb, t, lc, gq, rtab, ssm);
+        else quantize_slot<false, GROUPED, SMOOTH, true>(a, sb, t, lc, gq, rtab, ssm);
+    } else if (full) {
+        quantize_slot<true, GROUPED, SMOOTH, false>(a, sb, t, lc, gq, rtab, ssm);
+    } else {
+        quantize_slot<false, GROUPED, SMOOTH, false>(a, sb, t, lc, gq, rtab, ssm);
+    }
 }
 
 // Grid barrier (and, for one tensor, the amax reduction) in one: CTA c
@@ -1125,6 +1170,7 @@ __global__ void __launch_bounds__(kThreads) quant2d_kernel(Quant2dArgs a) {
     pdl_wait();
     const float g = a.gscale[0];
     const float k6 = __fmul_rn(6.0f, g);
+    const bool tiny = g < kTinyG;
     const int ntasks = (round128(a.n) / 16) * a.nseg;
     const int lane = threadIdx.x & 31;
     const int wstride = gridDim.x * kWarps;
@@ -1144,13 +1190,17 @@ __global__ void __launch_bounds__(kThreads) quant2d_kernel(Quant2dArgs a) {
         uint32_t am = absmax_bits(pm);
         am = max(am, __shfl_xor_sync(kFull, am, 1));
         float r;
-        const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, r);
+        const uint32_t sf = block_scale(__uint_as_float(am << 16), g, k6, tiny, r);
         const uint64_t rr = pack_rr(r);
         if (valid) {
+            uint8_t* dst = a.codes + (int64_t)(tr * 16) * kbytes + col / 2;
+            if (tiny) {   // uniform: one global scale
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                *reinterpret_cast<uint32_t*>(a.codes + (int64_t)(tr * 16 + i) * kbytes + col / 2) =
-                    quant8(v[i], rr);
+                for (int i = 0; i < 16; ++i) *reinterpret_cast<uint32_t*>(dst + i * kbytes) = quant8<true>(v[i], rr);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) *reinterpret_cast<uint32_t*>(dst + i * kbytes) = quant8(v[i], rr);
+            }
             if (a.compact && (lane & 1) == 0) a.compact[(int64_t)tr * (a.k / 16) + col / 16] = (uint8_t)sf;
         }
         const uint32_t s1 = __shfl_down_sync(kFull, sf, 2);
@@ -1529,14 +1579,20 @@ namespace {
 // Device address of g_static_quant_scratch on the current device.  Host code
 // must not pass the symbol itself to a kernel: on the host it names a
 // host-side stand-in, not device memory.  Looked up once per device, with
-// that device current.
+// that device current, and kept for the life of the device's primary context
+// (the address does not survive a cudaDeviceReset, after which this library
+// cannot be used on that device).  A failed lookup is also cleared from the
+// runtime's last-error slot, so that no later, unrelated call reports it.
 void* static_scratch() {
     int d = -1;
     if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return nullptr;
     std::lock_guard<std::mutex> lk(g_static_mu);
     if (!g_static_ptr[d]) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_static_quant_scratch) != cudaSuccess || !p) return nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_quant_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return nullptr;
+        }
         g_static_ptr[d] = p;
     }
     return g_static_ptr[d];

@@ -115,6 +115,76 @@ def test_quantize_act_edge_values(case):
     _assert_same_1d(xb)
 
 
+
+# ---- tiny global scales (1 / d beyond binary32) -----------------------------------------
+
+def _tiny_bf16(shape, stream, scale_pow):
+    """N(0,1) values times 2^scale_pow, rounded to BF16 (subnormal BF16 values
+    included for the smallest scales)."""
+    x = W.bf16_bits_to_f32(W.gaussian_bf16(shape, 0, stream, 1.0, outlier_frac=0.01))
+    return W.to_bf16_bits((x * np.float32(2.0 ** scale_pow)).astype(np.float32))
+
+
+@pytest.mark.parametrize("scale_pow", [-60, -110, -118, -124, -128])
+@pytest.mark.parametrize("shape", [(160, 96), (160, 1088), (70, 2048)])
+def test_quantize_act_tiny_global_scale(shape, scale_pow):
+    """Tensors whose amax puts g below 2^-64 (the kernels' tiny form of r)
+    and, from 2^-118 down, d = decode(sf) g below 2^-128, where 1 / d
+    overflows binary32: codes and scales equal the oracle's bit for bit.
+    k = 96 takes the two-kernel path, 1088 and 2048 the one-launch path."""
+    xb = _tiny_bf16(shape, 500 + shape[1], scale_pow)
+    _assert_same_1d(xb)
+
+
+@pytest.mark.parametrize("k", [1024, 1040])
+def test_grouped_quantize_tiny_and_normal_groups(k):
+    """Groups of very different magnitude in one call: each group takes the
+    tiny form of r or not by its own global scale (one-launch form for
+    k = 1024, two-kernel form for 1040)."""
+    sizes = [130, 64, 0, 200, 17]
+    pows = [0, -120, 0, -126, -100]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    parts = [_tiny_bf16((n, k), 600 + e, p) for e, (n, p) in enumerate(zip(sizes, pows))]
+    _assert_same_grouped(np.concatenate(parts, axis=0), off)
+
+
+def test_quantize_weight_2d_tiny_global_scale():
+    import torch
+    wb = _tiny_bf16((96, 160), 700, -122)
+    t = nv.quantize_weight_2d(bf16_to_device(wb))
+    torch.cuda.synchronize()
+    oc, osf, og = O.quantize_2d(wb)
+    assert t.global_scale.cpu().numpy()[0].view(np.uint32) == np.float32(og).view(np.uint32)
+    assert np.array_equal(t.codes.cpu().numpy(), oc)
+    assert np.array_equal(t.scales.cpu().numpy(), osf)
+
+
+@pytest.mark.parametrize("g_bits", [0x04000000, 0x00800000, 0x00001234])   # 2^-119, 2^-126, subnormal
+@pytest.mark.parametrize("scale_pow", [0, -118])
+def test_quantize_act_scaled_tiny_given_scale(g_bits, scale_pow):
+    """The given-scale pass with g below 2^-64: on a tensor of matching size,
+    and on one far too large for g, whose codes saturate at 6."""
+    import torch
+    xb = _tiny_bf16((150, 320), 710, scale_pow)
+    g = np.array([g_bits], np.uint32).view(np.float32)
+    q = nv.quantize_act_scaled(bf16_to_device(xb), torch.from_numpy(g.copy()).to(device()))
+    torch.cuda.synchronize()
+    oc, osf = O.quantize_1d_given_g(xb, g[0])
+    assert np.array_equal(q.codes.cpu().numpy(), oc)
+    assert np.array_equal(q.scales.cpu().numpy(), osf)
+
+
+def test_quantize_act_smooth_tiny_global_scale():
+    import torch
+    xb = _tiny_bf16((130, 2048), 720, -121)
+    s = (0.5 + W.uniform(0, 721, 2048)).astype(np.float32)
+    q = nv.quantize_act_smooth(bf16_to_device(xb), torch.from_numpy(s).to(device()))
+    torch.cuda.synchronize()
+    oc, osf, og = O.quantize_1d_smooth(xb, s)
+    assert q.global_scale.cpu().numpy()[0].view(np.uint32) == np.float32(og).view(np.uint32)
+    assert np.array_equal(q.codes.cpu().numpy(), oc)
+    assert np.array_equal(q.scales.cpu().numpy(), osf)
+
 @pytest.mark.parametrize("amax_bits", [0x3F80, 0x4340, 0x3B4D, 0x0B00, 0x0080, 0x0001, 0x7F7F])
 def test_block_scale_every_bf16_block_amax(amax_bits):
     """One block per positive BF16 value up to the tensor amax: each block's
