@@ -19,13 +19,19 @@
  *     block scale   = E4M3_rne_satfinite(block_amax / (6 * g));
  *     code          = E2M1_rne_satfinite(x * r), r = 1 / (block_scale * g),
  *                     r = 0 when block_scale * g == 0; the sign bit of x is
- *                     kept, also for zero codes.
+ *                     kept, also for zero codes.  r and x * r are rounded
+ *                     to binary32's 24-bit significand without binary32's
+ *                     exponent ceiling, so the code is the one nearest
+ *                     x / (block_scale * g) even where 1 / (block_scale * g)
+ *                     overflows binary32 (a global scale below ~2^-119).
  *   Storage: codes [rows, k/2] bytes, row-major, element 2i in bits 3:0 and
  *     element 2i+1 in bits 7:4 of byte i -- 4 bits per value; scales 1 byte
  *     per 16 values; 4.5 bits per value plus 4 bytes per tensor ("W4A8 vs
  *     NVFP4 quantization on GPUs", "Scale layout changes the real storage
  *     cost").
- *   Scale layout (not on the pages; the layout the tensor cores read):
+ *   Scale layout (not on the pages; the block-scale layout of the sm_100
+ *   block-scaled MMA, which the tests also check by having a library NVFP4
+ *   GEMM, cuBLASLt through torch's scaled_mm, read these bytes):
  *     rows padded to a multiple of 128, scale columns (k/16) padded to a
  *     multiple of 4, stored as 512-byte tiles of 128 rows x 4 columns, tiles
  *     ordered row-tile major, column-tile minor; inside a tile row r and
@@ -177,7 +183,9 @@ nvfp4_status_t nvfp4_quantize_act_scaled(const void* x, int64_t rows, int64_t k,
  *   most 1024 row groups; num_groups > 1024 returns
  *   NVFP4_ERR_UNSUPPORTED_SHAPE.
  *   The first call on a device looks up the array's device address with that
- *   device current; make that first call before any stream capture.
+ *   device current; make that first call before any stream capture.  The
+ *   address is kept for the life of the device's primary context (it does not
+ *   survive cudaDeviceReset).
  *   Each call first clears the array with an asynchronous memset on stream;
  *   otherwise it behaves exactly like nvfp4_quantize_act (same arguments,
  *   results, errors).
@@ -265,7 +273,18 @@ nvfp4_status_t nvfp4_gemm_emit_scale(const uint8_t* a_codes, const uint8_t* a_sc
  *   b_codes [num_experts, n, k/2]; b_scales num_experts consecutive blocks of
  *   nvfp4_scale_bytes(n, k) bytes; b_global [num_experts];
  *   c BF16 [total_rows, n] (row stride n), rows in grouped order.
- *   k % 64 == 0. */
+ *   Limits, checked before any launch:
+ *     k % 64 == 0, 1 <= num_experts <= 256, total_rows < 2^31 and
+ *     n * num_experts < 2^31, else NVFP4_ERR_UNSUPPORTED_SHAPE (the per-expert
+ *     tile table lives in the kernel's shared memory, 256 entries);
+ *     n % 8 == 0 and 16-byte aligned code, scale and output pointers, else
+ *     NVFP4_ERR_MISALIGNED (each output row must start on a 16-byte boundary
+ *     for the tensor-memory-accelerator store).
+ *   The grouped quantizer takes up to 65535 groups, so a layer of more than
+ *   256 experts quantizes its activations in one call and splits its GEMM
+ *   into calls of at most 256 experts (offsets rebased to the first row of
+ *   each call, the A pointers advanced to it).
+ *   workspace: unused (NULL accepted). */
 nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales,
                                   const float* a_global, const int32_t* offsets, int num_experts,
                                   const uint8_t* b_codes, const uint8_t* b_scales,

@@ -21,8 +21,10 @@ MXFP4 scale choice as a property over every BF16 magnitude, its round trip,
 nearest codes and 4.25 bits/value, and NVFP4's lower error on outliers; the
 W4A16 product against one-hot rows, the W4A4 product and a library matmul
 (tests/test_oracle_mx.py, tests/test_oracle_w4a16.py).  The scale-tile
-layout is not on the pages: its parity is pinned only through the GPU GEMM
-(tensor cores read it), so on the CPU it is "parity unpinned".
+layout is not on the pages: on the CPU only its bijection onto the padded
+buffer is checked; on the GPU a library block-scaled NVFP4 GEMM (cuBLASLt
+through torch's scaled_mm) reads scale bytes equal to the oracle's and must
+give the oracle's product (tests/test_gpu_gemm.py).
 """
 import ctypes
 import os

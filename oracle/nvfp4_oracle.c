@@ -110,7 +110,8 @@ void orc_e4m3_encode_array(const float* v, uint8_t* out, int64_t n) {
 /* Scale layout: 128-row x 4-column tiles of 512 bytes, tiles ordered with
  * the scale-column tile fastest.  Inside a tile, row r and column c sit at
  * (r % 32) * 16 + ((r % 128) / 32) * 4 + (c % 4).  This is the block-scale
- * layout the Blackwell tensor cores read; the pages do not describe it.     */
+ * layout of the Blackwell block-scaled MMA (checked on the GPU by a library
+ * NVFP4 GEMM reading these bytes); the pages do not describe it.            */
 
 int64_t orc_scale_rows(int64_t rows) { return (rows + 127) / 128 * 128; }
 int64_t orc_scale_cols(int64_t k) { return (k / 16 + 3) / 4 * 4; }

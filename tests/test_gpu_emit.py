@@ -9,7 +9,7 @@ import pytest
 import oracle as O
 import workloads as W
 import nvfp4_w4a4_quantized_05_b200 as nv
-from gpu_util import nvfp4_from_host
+from gpu_util import assert_gemm_close, gemm_refs, nvfp4_from_host, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -20,11 +20,15 @@ def _sync():
     nv.check_device_error()
 
 
-def _operands(m, n, k, seed, scale=1.0):
+def _operands(m, n, k, seed, scale=1.0, with_ref=False):
     a = W.gaussian_bf16((m, k), seed, 600 + m, scale, outlier_frac=0.01)
     w = W.gaussian_bf16((n, k), seed, 601 + n, 0.02)
+    qa = O.quantize_1d(a)
     qw = O.quantize_2d(w) if n % 16 == 0 else O.quantize_1d(w)
-    return nvfp4_from_host(*O.quantize_1d(a)), nvfp4_from_host(*qw)
+    ops = (nvfp4_from_host(*qa), nvfp4_from_host(*qw))
+    if with_ref:
+        return ops + (gemm_refs(O.dequantize(*qa), O.dequantize(*qw)),)
+    return ops
 
 
 def _expected_g(c):
@@ -43,11 +47,12 @@ def _expected_g(c):
 ])
 def test_emit_scale_and_two_phase_quantization(m, n, k):
     import torch
-    ta, tw = _operands(m, n, k, 7)
+    ta, tw, (ref, absref) = _operands(m, n, k, 7, with_ref=True)
     c_ref = nv.gemm(ta, tw)
     c, g = nv.gemm_emit_scale(ta, tw)
     _sync()
     assert torch.equal(c, c_ref)                      # the same output bits
+    assert_gemm_close(to_host_f64(c), ref, absref, k, f"emit {m}x{n}x{k}")
     g_exp, bits = _expected_g(c)
     assert g.cpu().numpy().view(np.uint32)[0] == np.array([g_exp]).view(np.uint32)[0]
     q2 = nv.quantize_act_scaled(c, g)                 # one read of C

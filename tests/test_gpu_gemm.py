@@ -1,15 +1,17 @@
 """GPU GEMM parity: the tcgen05 block-scaled GEMM against the binary64 oracle
 GEMM over the reconstructed operands, within the stated tolerance
-(relative Frobenius <= 2e-3, max |error| <= 1e-2 x row max |ref|).  Small
-cases compare every output; the full-size prefill / decode / MoE workloads
-compare sampled rows the oracle computes one by one."""
+(relative Frobenius <= 2e-3, max |error| <= 1e-2 x row max |ref|) and,
+element by element, within one BF16 ulp plus the FP32 summation bound
+(gpu_util.assert_gemm_close).  Small cases compare every output; the
+full-size prefill / decode / MoE workloads compare sampled rows the oracle
+computes one by one.  Every operand of a reference is the oracle's."""
 import numpy as np
 import pytest
 
 import oracle as O
 import workloads as W
 import nvfp4_w4a4_quantized_05_b200 as nv
-from gpu_util import assert_gemm_close, bf16_to_device, nvfp4_from_host, to_host_f64
+from gpu_util import assert_gemm_close, bf16_to_device, gemm_refs, nvfp4_from_host, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -37,9 +39,9 @@ def test_tiny_workload_end_to_end():
     ac, asf, ga = O.quantize_1d(a)
     wc, wsf, gw = O.quantize_2d(w)
     assert np.array_equal(ta.codes.cpu().numpy(), ac) and np.array_equal(tw.codes.cpu().numpy(), wc)
-    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
     got = to_host_f64(c)
-    assert_gemm_close(got, ref, "tiny")
+    assert_gemm_close(got, ref, absref, 256, "tiny")
     # the exact integer sum, scaled, rounds to within one BF16 step of the output
     exact = O.gemm_exact_i64(ac, asf, wc, wsf, 256).astype(np.float64) * 2.0 ** -20 * float(np.float32(ga) * np.float32(gw))
     assert np.all(np.abs(got - exact) <= 2.0 ** -7 * np.abs(exact) + 1e-30)
@@ -69,8 +71,8 @@ def test_gemm_matches_oracle(m, n, k):
     (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 0)
     c = nv.gemm(nvfp4_from_host(ac, asf, ga), nvfp4_from_host(wc, wsf, gw))
     _sync()
-    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
-    assert_gemm_close(to_host_f64(c), ref, f"{m}x{n}x{k}")
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    assert_gemm_close(to_host_f64(c), ref, absref, k, f"{m}x{n}x{k}")
 
 
 def test_gemm_output_row_stride():
@@ -79,8 +81,8 @@ def test_gemm_output_row_stride():
     out = torch.full((150, 136), 7.0, dtype=torch.bfloat16, device="cuda")
     nv.gemm(nvfp4_from_host(ac, asf, ga), nvfp4_from_host(wc, wsf, gw), out=out[:, :96])
     _sync()
-    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
-    assert_gemm_close(to_host_f64(out[:, :96]), ref, "strided")
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    assert_gemm_close(to_host_f64(out[:, :96]), ref, absref, 128, "strided")
     assert torch.all(out[:, 96:] == 7.0)                  # nothing written past n
 
 
@@ -95,7 +97,7 @@ def test_stream_k_workspace_reuse_and_without_workspace():
     assert nv.nvfp4_workspace_bytes(nv.OP_GEMM, 64, n, k, 0) == 0          # decode tiles: none
     (ac, asf, ga), (wc, wsf, gw) = _oracle_operands(m, n, k, 3)
     ta, tw = nvfp4_from_host(ac, asf, ga), nvfp4_from_host(wc, wsf, gw)
-    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
     ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
     for it in range(3):
@@ -107,7 +109,7 @@ def test_stream_k_workspace_reuse_and_without_workspace():
             assert st == 0
             _sync()
             assert int(ws[:32768].to(torch.int64).sum()) == 0
-            assert_gemm_close(to_host_f64(c), ref, f"stream-K call {it}, workspace {ws_ptr is not None}")
+            assert_gemm_close(to_host_f64(c), ref, absref, k, f"stream-K call {it}, workspace {ws_ptr is not None}")
     # a misaligned workspace is refused before anything runs
     assert nv.nvfp4_gemm(ta.codes.data_ptr(), ta.scales.data_ptr(), ta.global_scale.data_ptr(),
                          tw.codes.data_ptr(), tw.scales.data_ptr(), tw.global_scale.data_ptr(), c.data_ptr(),
@@ -121,17 +123,20 @@ def prefill_case():
 
 
 def test_prefill_workload_sampled_rows(prefill_case):
+    """Quantize on the GPU, check both operands against the oracle's bit for
+    bit, then the GEMM on sampled rows against the oracle's operands."""
     a, w, (ac, asf, ga), (wc, wsf, gw) = prefill_case
     ta = nv.quantize_act(bf16_to_device(a))
     tw = nv.quantize_weight_2d(bf16_to_device(w))
     c = nv.gemm(ta, tw)
     _sync()
+    assert np.array_equal(ta.codes.cpu().numpy(), ac) and np.array_equal(ta.scales.cpu().numpy(), asf)
+    assert np.array_equal(tw.codes.cpu().numpy(), wc) and np.array_equal(tw.scales.cpu().numpy(), wsf)
+    assert ta.global_scale.item() == float(np.float32(ga)) and tw.global_scale.item() == float(np.float32(gw))
     rows = np.unique(np.concatenate([np.arange(0, 4096, 128), np.arange(127, 4096, 128)[::4], [1, 2049, 4095]]))
-    ah = O.dequantize(ac, asf, ga)[rows]
-    wh = O.dequantize(wc, wsf, gw)
-    ref = O.gemm_f64(ah, wh)
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga)[rows], O.dequantize(wc, wsf, gw))
     got = to_host_f64(c[rows.tolist()])
-    assert_gemm_close(got, ref, "prefill")
+    assert_gemm_close(got, ref, absref, 4096, "prefill")
 
 
 @pytest.fixture(scope="module")
@@ -150,8 +155,8 @@ def test_decode_workload_full(m, decode_weights):
     c = nv.gemm(ta, nvfp4_from_host(wc, wsf, gw))
     _sync()
     assert np.array_equal(ta.codes.cpu().numpy(), ac)
-    ref = O.gemm_f64(O.dequantize(ac, asf, ga), wh)
-    assert_gemm_close(to_host_f64(c), ref, f"decode m={m}")
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), wh)
+    assert_gemm_close(to_host_f64(c), ref, absref, 5120, f"decode m={m}")
 
 
 @pytest.mark.parametrize("sizes,k,n", [
@@ -181,11 +186,15 @@ def test_grouped_gemm_ragged_experts(sizes, k, n):
     for e in range(E):
         r0, r1 = off[e], off[e + 1]
         if r1 > r0:
-            ref = O.gemm_f64(ah[r0:r1], O.dequantize(wq[e][0], wq[e][1], wq[e][2]))
-            assert_gemm_close(got[r0:r1], ref, f"expert {e}")
+            ref, absref = gemm_refs(ah[r0:r1], O.dequantize(wq[e][0], wq[e][1], wq[e][2]))
+            assert_gemm_close(got[r0:r1], ref, absref, k, f"expert {e}")
 
 
 def test_moe_workload_sampled_rows():
+    """The MoE workload end to end on the GPU: grouped activation
+    quantization and each expert's 2D weight quantization are checked against
+    the oracle's bit for bit, then the grouped GEMM on sampled rows of every
+    expert against the binary64 product of the oracle's operands."""
     import torch
     a, off, w = W.moe(0)
     E, N, K = w.shape
@@ -199,8 +208,15 @@ def test_moe_workload_sampled_rows():
     _sync()
     ac, asf, ga = O.quantize_1d_grouped(a, off)
     assert np.array_equal(ta.codes.cpu().numpy(), ac)
-    wc_all, wsf_all, gw_all = b_codes.cpu().numpy(), b_scales.cpu().numpy(), b_global.cpu().numpy()
+    assert np.array_equal(ta.scales.cpu().numpy()[:asf.size], asf)
+    assert np.array_equal(ta.global_scale.cpu().numpy().view(np.uint32), np.asarray(ga, np.float32).view(np.uint32))
+    wq = [O.quantize_2d(np.ascontiguousarray(w[e])) for e in range(E)]
     sbytes = nv.nvfp4_scale_bytes(N, K)
+    dev_codes, dev_scales, dev_g = b_codes.cpu().numpy(), b_scales.cpu().numpy(), b_global.cpu().numpy()
+    for e in range(E):
+        assert np.array_equal(dev_codes[e], wq[e][0]), f"expert {e} weight codes"
+        assert np.array_equal(dev_scales[e * sbytes:(e + 1) * sbytes], wq[e][1]), f"expert {e} weight scales"
+        assert dev_g[e] == np.float32(wq[e][2]), f"expert {e} weight global scale"
     row0 = 0
     got = to_host_f64(c)
     for e in range(E):
@@ -209,6 +225,37 @@ def test_moe_workload_sampled_rows():
         if n_e:
             sel = np.unique([r0, r0 + n_e // 2, r1 - 1, min(r1 - 1, r0 + 127), min(r1 - 1, r0 + 128)])
             a_hat = O.dequantize(ac[r0:r1], asf, float(ga[e]), sf_row0=row0, k=K)[sel - r0]
-            w_hat = O.dequantize(wc_all[e], wsf_all[e * sbytes:(e + 1) * sbytes], float(gw_all[e]))
-            assert_gemm_close(got[sel], O.gemm_f64(a_hat, w_hat), f"moe expert {e}")
+            w_hat = O.dequantize(*wq[e])
+            ref, absref = gemm_refs(a_hat, w_hat)
+            assert_gemm_close(got[sel], ref, absref, K, f"moe expert {e}")
         row0 += O.scale_rows(n_e)
+
+
+@pytest.mark.parametrize("m,n,k", [(384, 256, 1024), (200, 272, 320)])
+def test_scale_layout_read_by_library_block_scaled_gemm(m, n, k):
+    """The scale bytes the quantizers write, unmodified, read by another
+    block-scaled NVFP4 GEMM on this GPU (torch's scaled_mm: E2M1 operands,
+    E4M3 scales per 16 values, 32 x 4 x 4 swizzled scale layout): its output
+    must be the oracle's product of the block-scaled operands (no global
+    scales) to the GEMM tolerance.  A layout this library only agreed with
+    itself on would fail here.  Several 128 x 4 scale tiles along both rows
+    and columns; the second shape has padded rows and columns."""
+    import torch
+    import torch.nn.functional as F
+    a = W.gaussian_bf16((m, k), 0, 1300 + m, 1.0, outlier_frac=0.01)
+    w = W.gaussian_bf16((n, k), 0, 1301 + n, 0.02)
+    ta = nv.quantize_act(bf16_to_device(a))
+    tw = nv.quantize_weight_2d(bf16_to_device(w))
+    _sync()
+    ac, asf, _ = O.quantize_1d(a)
+    wc, wsf, _ = O.quantize_2d(w)
+    assert np.array_equal(ta.codes.cpu().numpy(), ac) and np.array_equal(ta.scales.cpu().numpy(), asf)
+    assert np.array_equal(tw.codes.cpu().numpy(), wc) and np.array_equal(tw.scales.cpu().numpy(), wsf)
+    c = F.scaled_mm(ta.codes.view(torch.float4_e2m1fn_x2), tw.codes.view(torch.float4_e2m1fn_x2).t(),
+                    ta.scales.view(torch.float8_e4m3fn), F.ScalingType.BlockWise1x16,
+                    tw.scales.view(torch.float8_e4m3fn), F.ScalingType.BlockWise1x16,
+                    swizzle_a=F.SwizzleType.SWIZZLE_32_4_4, swizzle_b=F.SwizzleType.SWIZZLE_32_4_4,
+                    output_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref, absref = gemm_refs(O.dequantize(ac, asf, 1.0), O.dequantize(wc, wsf, 1.0))
+    assert_gemm_close(to_host_f64(c), ref, absref, k, f"library GEMM on our scale bytes {m}x{n}x{k}")

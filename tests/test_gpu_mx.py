@@ -10,7 +10,7 @@ import pytest
 import oracle as O
 import workloads as W
 import nvfp4_w4a4_quantized_05_b200 as nv
-from gpu_util import assert_gemm_close, bf16_to_device, to_host_f64, u8_to_device
+from gpu_util import assert_gemm_close, bf16_to_device, gemm_refs, to_host_f64, u8_to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -98,8 +98,8 @@ def test_mx_gemm_matches_oracle(m, n, k):
     wc, wsf = O.quantize_1d_mx(w)
     c = nv.gemm_mx(_mx_from_host(ac, asf), _mx_from_host(wc, wsf))
     _sync()
-    ref = O.gemm_f64(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
-    assert_gemm_close(to_host_f64(c), ref, f"mx {m}x{n}x{k}")
+    ref, absref = gemm_refs(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
+    assert_gemm_close(to_host_f64(c), ref, absref, k, f"mx {m}x{n}x{k}")
 
 
 def test_mx_gemm_stream_k_workspace_and_none():
@@ -110,7 +110,7 @@ def test_mx_gemm_stream_k_workspace_and_none():
     ac, asf = O.quantize_1d_mx(a)
     wc, wsf = O.quantize_1d_mx(w)
     ta, tw = _mx_from_host(ac, asf), _mx_from_host(wc, wsf)
-    ref = O.gemm_f64(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
+    ref, absref = gemm_refs(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
     ws = torch.zeros(nv.nvfp4_workspace_bytes(nv.OP_GEMM, m, n, k, 0), dtype=torch.uint8, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
     for ws_ptr in (ws.data_ptr(), None, ws.data_ptr()):
@@ -120,7 +120,7 @@ def test_mx_gemm_stream_k_workspace_and_none():
         assert st == 0
         _sync()
         assert int(ws[:32768].to(torch.int64).sum()) == 0
-        assert_gemm_close(to_host_f64(c), ref, f"mx stream-K, workspace {ws_ptr is not None}")
+        assert_gemm_close(to_host_f64(c), ref, absref, k, f"mx stream-K, workspace {ws_ptr is not None}")
 
 
 def test_mx_prefill_workload_end_to_end():
@@ -136,8 +136,8 @@ def test_mx_prefill_workload_end_to_end():
     assert np.array_equal(ta.codes.cpu().numpy(), ac) and np.array_equal(ta.scales.cpu().numpy(), asf)
     assert np.array_equal(tw.codes.cpu().numpy(), wc) and np.array_equal(tw.scales.cpu().numpy(), wsf)
     rows = np.unique(np.concatenate([np.arange(0, 4096, 128), np.arange(127, 4096, 128)[::4], [1, 2049, 4095]]))
-    ref = O.gemm_f64(O.dequantize_mx(ac, asf)[rows], O.dequantize_mx(wc, wsf))
-    assert_gemm_close(to_host_f64(c[rows.tolist()]), ref, "mx prefill")
+    ref, absref = gemm_refs(O.dequantize_mx(ac, asf)[rows], O.dequantize_mx(wc, wsf))
+    assert_gemm_close(to_host_f64(c[rows.tolist()]), ref, absref, 4096, "mx prefill")
 
 
 def test_mx_decode_workload():
@@ -147,8 +147,8 @@ def test_mx_decode_workload():
     wc, wsf = O.quantize_1d_mx(w)
     c = nv.gemm_mx(nv.quantize_mx(bf16_to_device(a)), nv.quantize_mx(bf16_to_device(w)))
     _sync()
-    ref = O.gemm_f64(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
-    assert_gemm_close(to_host_f64(c), ref, "mx decode")
+    ref, absref = gemm_refs(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
+    assert_gemm_close(to_host_f64(c), ref, absref, 5120, "mx decode")
 
 
 def test_mx_strided_input_zero_tensor_and_empty_gemm():
@@ -177,5 +177,6 @@ def test_mx_strided_input_zero_tensor_and_empty_gemm():
     nv.gemm_mx(_mx_from_host(ac, asf), tw, out=out[:, :96])
     _sync()
     assert c0.shape == (0, 96)
-    assert_gemm_close(to_host_f64(out[:, :96]), O.gemm_f64(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf)), "mx strided")
+    ref, absref = gemm_refs(O.dequantize_mx(ac, asf), O.dequantize_mx(wc, wsf))
+    assert_gemm_close(to_host_f64(out[:, :96]), ref, absref, 256, "mx strided")
     assert torch.all(out[:, 96:] == 7.0)

@@ -8,7 +8,7 @@ import pytest
 import oracle as O
 import workloads as W
 import nvfp4_w4a4_quantized_05_b200 as nv
-from gpu_util import assert_gemm_close, bf16_to_device, to_host_f64
+from gpu_util import assert_gemm_close, bf16_to_device, gemm_refs, to_host_f64
 
 pytestmark = pytest.mark.gpu
 
@@ -74,5 +74,5 @@ def test_smooth_gemm_end_to_end():
     nv.check_device_error()
     ac, asf, ga = O.quantize_1d_smooth(xb, s)
     wc, wsf, gw = O.quantize_2d(wsb)
-    ref = O.gemm_f64(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
-    assert_gemm_close(to_host_f64(c), ref, "smooth")
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(wc, wsf, gw))
+    assert_gemm_close(to_host_f64(c), ref, absref, k, "smooth")

@@ -9,7 +9,14 @@ import pytest
 import oracle as O
 import workloads as W
 import nvfp4_w4a4_quantized_05_b200 as nv
-from gpu_util import assert_gemm_close, bf16_to_device, nvfp4_from_host, to_host_f64
+from gpu_util import assert_gemm_close, bf16_to_device, gemm_refs, nvfp4_from_host, to_host_f64
+
+
+def _refs(a_bits, wc, wsf, gw):
+    """The oracle's W4A16 product and the product of the operands' magnitudes."""
+    ref = O.gemm_w4a16_f64(a_bits, wc, wsf, gw)
+    _, absref = gemm_refs(O.bf16_to_f64(a_bits), O.dequantize(wc, wsf, gw))
+    return ref, absref
 
 pytestmark = pytest.mark.gpu
 
@@ -34,8 +41,8 @@ def test_w4a16_matches_oracle(m, n, k, two_d):
     wc, wsf, gw = O.quantize_2d(w) if two_d else O.quantize_1d(w)
     c = nv.gemm_w4a16(bf16_to_device(a), nvfp4_from_host(wc, wsf, gw))
     _sync()
-    ref = O.gemm_w4a16_f64(a, wc, wsf, gw)
-    assert_gemm_close(to_host_f64(c), ref, f"w4a16 {m}x{n}x{k}")
+    ref, absref = _refs(a, wc, wsf, gw)
+    assert_gemm_close(to_host_f64(c), ref, absref, k, f"w4a16 {m}x{n}x{k}")
 
 
 def test_w4a16_output_stride_and_limits():
@@ -47,7 +54,7 @@ def test_w4a16_output_stride_and_limits():
     out = torch.full((m, 136), 7.0, dtype=torch.bfloat16, device="cuda")
     nv.gemm_w4a16(bf16_to_device(a), tw, out=out[:, :96])
     _sync()
-    assert_gemm_close(to_host_f64(out[:, :96]), O.gemm_w4a16_f64(a, wc, wsf, gw), "w4a16 strided")
+    assert_gemm_close(to_host_f64(out[:, :96]), *_refs(a, wc, wsf, gw), k, "w4a16 strided")
     assert torch.all(out[:, 96:] == 7.0)
     with pytest.raises(nv.Nvfp4Error):                     # m above the decode tile
         nv.gemm_w4a16(bf16_to_device(W.gaussian_bf16((65, k), 0, 972, 1.0)), tw)
@@ -63,7 +70,7 @@ def test_w4a16_decode_workload(m):
     c = nv.gemm_w4a16(bf16_to_device(a), tw)
     _sync()
     assert np.array_equal(tw.codes.cpu().numpy(), wc)
-    assert_gemm_close(to_host_f64(c), O.gemm_w4a16_f64(a, wc, wsf, gw), f"w4a16 decode m={m}")
+    assert_gemm_close(to_host_f64(c), *_refs(a, wc, wsf, gw), 5120, f"w4a16 decode m={m}")
 
 
 def test_w4a16_strided_activations():
@@ -73,5 +80,5 @@ def test_w4a16_strided_activations():
     wc, wsf, gw = O.quantize_1d(W.gaussian_bf16((n, k), 0, 981, 0.02))
     c = nv.gemm_w4a16(bf16_to_device(a_full)[:, :k], nvfp4_from_host(wc, wsf, gw))
     _sync()
-    ref = O.gemm_w4a16_f64(np.ascontiguousarray(a_full[:, :k]), wc, wsf, gw)
-    assert_gemm_close(to_host_f64(c), ref, "w4a16 strided activations")
+    ref, absref = _refs(np.ascontiguousarray(a_full[:, :k]), wc, wsf, gw)
+    assert_gemm_close(to_host_f64(c), ref, absref, k, "w4a16 strided activations")
