@@ -500,6 +500,31 @@ def grouped_gemm(a: NVFP4Tensor, b_codes, b_scales, b_global, n: int, out=None):
     return c
 
 
+def _reset_workspaces(device_index: int) -> None:
+    """Re-initialise every workspace this module keeps for one device.  A
+    bounded wait that ran out leaves a workspace out of step (a grid barrier
+    that gave up leaves some CTAs' generation words behind the others', a
+    stream-K hand-off may leave a flag set), and every later call on it would
+    wait in vain again.  All work on the device is finished first, so no
+    kernel still uses one; each is then zeroed, as nvfp4_workspace_init
+    would."""
+    import torch
+    mine = [ws for key, ws in _ws_cache.items() if key[0] == device_index]
+    if not mine:
+        return
+    with torch.cuda.device(device_index):
+        torch.cuda.synchronize()
+        for ws in mine:
+            ws.zero_()
+        torch.cuda.synchronize()
+
+
 def check_device_error(stream: int = 0) -> None:
-    """Raise if a kernel of the library reported a bounded wait that ran out."""
-    _check(nvfp4_get_last_device_error(stream), "device")
+    """Raise if a kernel of the library reported a bounded wait that ran out
+    on the current device.  Before raising, the workspaces this module cached
+    for that device are re-initialised, so the next call starts clean."""
+    st = nvfp4_get_last_device_error(stream)
+    if st == 5:
+        import torch
+        _reset_workspaces(torch.cuda.current_device())
+    _check(st, "device")

@@ -78,6 +78,35 @@ def test_static_scratch_matches_workspace_entry_point_groups():
     _run_both(bf16_to_device(xb), torch.from_numpy(off).to(device()), len(sizes))
 
 
+@pytest.mark.parametrize("k", [48, 80])
+def test_static_scratch_two_kernel_path(k):
+    """k % 64 != 0 takes the two-kernel path, whose scratch words (the CTA
+    counter, the per-group amaxes and the groups' first scale rows) sit
+    elsewhere in the array than the one-launch path's: one tensor and row
+    groups, two calls in a row each."""
+    import torch
+    xb = W.gaussian_bf16((333, k), 0, 902 + k, 1.0, outlier_frac=0.01)
+    _run_both(bf16_to_device(xb), None, 0)
+    sizes = [7, 0, 200, 129, 1]
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    xg = W.gaussian_bf16((int(off[-1]), k), 0, 903 + k, 1.0, outlier_frac=0.01)
+    _run_both(bf16_to_device(xg), torch.from_numpy(off).to(device()), len(sizes))
+
+
+@pytest.mark.parametrize("k", [128, 80])
+def test_static_scratch_at_its_group_limit(k):
+    """Exactly 1024 row groups, the most the fixed array holds (sizes 0..9,
+    runs of empty groups), on the one-launch (k = 128) and the two-kernel
+    (k = 80) path."""
+    import torch
+    rng = np.random.default_rng(k)
+    sizes = rng.integers(0, 10, 1024)
+    sizes[100:140] = 0
+    off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
+    xb = W.gaussian_bf16((int(off[-1]), k), 0, 904 + k, 1.0, outlier_frac=0.01)
+    _run_both(bf16_to_device(xb), torch.from_numpy(off).to(device()), 1024)
+
+
 def test_static_scratch_rejects_more_groups_than_it_holds():
     import torch
     groups = 1025
