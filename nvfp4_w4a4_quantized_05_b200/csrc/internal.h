@@ -51,17 +51,25 @@ inline nvfp4_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? NVF
 
 // Workspace layout of the quantizers (bytes); G = number of row groups:
 //   [0, 128 * kMaxFusedCtas)  one-launch path: the word of CTA c at 128 c,
-//                  generation << 32 | BF16 amax bits (uint64; one per 128-byte
-//                  line, so that pollers spread over the L2 slices).  At a
-//                  fixed place, so that every call on the workspace, with or
-//                  without groups, steps the same generation count.
+//                  generation << 32 (uint64, one per 128-byte line): the
+//                  generation of the CTA's last call.  At a fixed place, so
+//                  that every call on the workspace, with or without groups,
+//                  steps the same generation count.
+//   [B, B + 128)   one-launch path, grid barrier (B = quant_ws_bar_off()):
+//                  word 0 counts CTA arrivals (uint32, one per CTA per call,
+//                  never reset: all CTAs of call gen have arrived when it
+//                  reads gen * grid size); words 1 and 2 hold the tensor
+//                  amax of calls with even and odd generation (FP32 bits,
+//                  folded with atomicMax; each call zeroes the other one for
+//                  the next call).
 //   [T, T + 4)     two-kernel path: CTA completion counter (uint32), T = quant_ws_two_off()
 //   [T + 16, T + 16 + 4G)  two-kernel path: per-group amax as FP32 bit patterns (uint32)
 //   [pad_off, +4(G+1))     per-group first scale row (int32), written each call
 //   [gword_off, +8G)       one-launch grouped path: per-group generation << 32 | amax bits (uint64)
 constexpr int kMaxFusedCtas = 256;
 constexpr int kPartStrideWords = 16;   // uint64 words: 128 bytes
-constexpr int64_t quant_ws_two_off() { return 128 * (int64_t)kMaxFusedCtas; }
+constexpr int64_t quant_ws_bar_off() { return 128 * (int64_t)kMaxFusedCtas; }
+constexpr int64_t quant_ws_two_off() { return quant_ws_bar_off() + 128; }
 constexpr int64_t quant_ws_pad_off(int groups) { return round_up(quant_ws_two_off() + 16 + 4 * (int64_t)groups, 16); }
 constexpr int64_t quant_ws_gword_off(int groups) {
     return round_up(quant_ws_pad_off(groups) + 4 * ((int64_t)groups + 1), 128);

@@ -505,6 +505,7 @@ constexpr int kTaskVals = 1024;                  // values per warp task
 constexpr int kTaskBytes = kTaskVals * 2;
 constexpr int kStage = 3;                        // task slots per warp
 
+constexpr int kTmTasks = 4;                      // tasks a warp can park in tensor memory (64 columns)
 constexpr int kMaxFusedGroups = 1024;            // row groups the one-launch form takes
 constexpr int kMaxSmoothK = 6144;                // k of the pre-scaled form (its factors sit in shared memory)
 
@@ -519,8 +520,10 @@ struct FusedArgs {
     float* gscale;    // [groups]
     uint8_t* codes;
     uint8_t* scales;
-    uint64_t* part;   // per-CTA generation << 32 | amax words, kPartStrideWords apart
+    uint64_t* part;   // per-CTA generation << 32 words, kPartStrideWords apart
+    uint32_t* bar;    // grid barrier: arrival counter, amax words of even and odd generations
     uint64_t* gword;  // grouped: per-group generation << 32 | amax words
+    int tm_tasks;     // tasks per warp parked in tensor memory (0: none allocated)
     const int32_t* offsets;   // grouped: [groups + 1]; nullptr for one tensor
     int groups;
     const float* smooth;      // pre-scaled form: per-column factors [k]; nullptr otherwise
@@ -732,16 +735,14 @@ __device__ __forceinline__ uint64_t block_rr(uint32_t sf, const GroupQ& q) {
     return pack_rr(block_recip(__fmul_rn(e4m3_to_f32(sf), q.g), q.tiny));
 }
 
-// Quantize the task held in slot sb.  FULL: the whole task is inside the
-// tensor.  One tensor: r from the per-CTA table; grouped: r computed per block.
-// TINY: the group's g takes the tiny form of r (block_recip).
+// Quantize one task whose values the lane holds in u (its 32 values, units
+// 4 lane .. 4 lane + 3 of the task).  FULL: the whole task is inside the
+// tensor.  One tensor: r from the per-CTA table; grouped: r computed per
+// block.  TINY: the group's g takes the tiny form of r (block_recip).
 template <bool FULL, bool GROUPED, bool SMOOTH, bool TINY>
-__device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
+__device__ __forceinline__ void quantize_vals(const FusedArgs& a, const uint4 (&u)[4], const DstCursor<GROUPED>& t,
                                               const LaneC& lc, const GroupQ& gq, const uint64_t* rtab,
                                               const float* ssm) {
-    uint4 u[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4*>(sb + lc.ld_off[i]);
     float b0, b1;
     float4 sv[8];   // pre-scaled form: the factors of this lane's 32 columns
     if constexpr (SMOOTH) {
@@ -794,49 +795,60 @@ __device__ __forceinline__ void quantize_slot(const FusedArgs& a, const char* sb
     }
 }
 template <bool GROUPED, bool SMOOTH>
-__device__ __forceinline__ void quantize_any(const FusedArgs& a, const char* sb, const DstCursor<GROUPED>& t,
+__device__ __forceinline__ void quantize_any(const FusedArgs& a, const uint4 (&u)[4], const DstCursor<GROUPED>& t,
                                              const LaneC& lc, const GroupQ& gq, const uint64_t* rtab,
                                              const float* ssm) {
     const bool full = t.valid() && t.seg < a.full_segs;
     if (gq.tiny) {   // warp-uniform (one g per group): a global scale below 2^-64
-        if (full) quantize_slot<true, GROUPED, SMOOTH, true>(a, sb, t, lc, gq, rtab, ssm);
-        else quantize_slot<false, GROUPED, SMOOTH, true>(a, sb, t, lc, gq, rtab, ssm);
+        if (full) quantize_vals<true, GROUPED, SMOOTH, true>(a, u, t, lc, gq, rtab, ssm);
+        else quantize_vals<false, GROUPED, SMOOTH, true>(a, u, t, lc, gq, rtab, ssm);
     } else if (full) {
-        quantize_slot<true, GROUPED, SMOOTH, false>(a, sb, t, lc, gq, rtab, ssm);
+        quantize_vals<true, GROUPED, SMOOTH, false>(a, u, t, lc, gq, rtab, ssm);
     } else {
-        quantize_slot<false, GROUPED, SMOOTH, false>(a, sb, t, lc, gq, rtab, ssm);
+        quantize_vals<false, GROUPED, SMOOTH, false>(a, u, t, lc, gq, rtab, ssm);
     }
 }
-
-// Grid barrier (and, for one tensor, the amax reduction) in one: CTA c
-// publishes its word (part + kPartStrideWords c, one per 128-byte line) =
-// gen << 32 | (the FP32 bits of its amax; 0 in the grouped form), so a reader that
-// sees this call's generation also sees the amax.  gen is one more (mod 2^32)
-// than the generation of the CTA's own word from the previous call (0 in a
-// fresh workspace), the same for every CTA.  Warp 0 of each CTA polls all G
-// words until every one carries gen; false if that wait ran out (error word set).
-__device__ __forceinline__ bool grid_amax(const uint64_t* part, int G, uint32_t gen, uint64_t limit, unsigned* err,
-                                          int lane, uint32_t& amax_bits) {
-    const uint64_t t0 = globaltimer_ns();
-    while (true) {
-        bool mine = true;
-        uint32_t mx = 0;
-        for (int i = lane; i < G; i += 32) {
-            const uint64_t w = ld_relaxed_gpu_u64(part + kPartStrideWords * i);
-            mine = mine && (uint32_t)(w >> 32) == gen;
-            mx = max(mx, (uint32_t)w);
-        }
-        if (__all_sync(kFull, mine)) {
+// The lane's 32 values of the task in shared-memory slot sb.
+__device__ __forceinline__ void load_slot(const char* sb, const LaneC& lc, uint4 (&u)[4]) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(kFull, mx, o));
-            amax_bits = mx;
-            return true;
-        }
+    for (int i = 0; i < 4; ++i) u[i] = *reinterpret_cast<const uint4*>(sb + lc.ld_off[i]);
+}
+// ... and of the task parked in tensor memory at address ta (16 columns of
+// the warp's lane quarter, lane i holding lane i's values).
+__device__ __forceinline__ void load_tmem(uint32_t ta, uint4 (&u)[4]) {
+    uint32_t r[16];
+    tmem_ld_32x32b_x16(ta, r);
+    tmem_ld_wait();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) u[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+}
+
+// Grid barrier and, for one tensor, the amax reduction.  Every CTA knows the
+// call's generation gen from its own word (one more than its last call's;
+// every CTA of a call holds the same).  Arrival: fold the CTA's amax into
+// amax word gen & 1, then add one to the arrival counter with release
+// semantics; CTA 0 also zeroes the other amax word for the next call (no CTA
+// of this call uses it, and the previous call is over).  All CTAs of call
+// gen have arrived when the counter reads gen * G (mod 2^32: it never resets
+// and each call adds exactly G).  Lane 0 of warp 0 polls it with acquire
+// loads; false if that wait ran out (error word set).
+__device__ __forceinline__ void grid_arrive(uint32_t* bar, uint32_t gen, uint32_t amax_bits, bool first_cta) {
+    if (amax_bits) atomicMax(bar + 1 + (gen & 1u), amax_bits);
+    if (first_cta) st_relaxed_gpu_u32(bar + 1 + ((gen + 1u) & 1u), 0u);
+    red_release_gpu_add_u32(bar, 1u);
+}
+__device__ __forceinline__ bool grid_wait(const uint32_t* bar, uint32_t gen, int G, uint64_t limit, unsigned* err,
+                                          uint32_t& amax_bits) {
+    const uint32_t target = gen * (uint32_t)G;
+    const uint64_t t0 = globaltimer_ns();
+    while (ld_acquire_gpu_u32(bar) != target) {
         if (globaltimer_ns() - t0 > limit) {
-            if (lane == 0) atomicOr(err, 1u);
+            atomicOr(err, 1u);
             return false;
         }
     }
+    amax_bits = ld_relaxed_gpu_u32(bar + 1 + (gen & 1u));
+    return true;
 }
 
 // Grouped form: fold a warp's amax bits m of group e into the group's word.
@@ -918,48 +930,62 @@ struct Pass2Q {
     }
 };
 
-// Pass 2 of one warp with tasks tw .. tw + n - 1, the last nres = min(kStage, n)
-// of them still on chip: task n - nres + k is in slot (n - nres + k) % kStage.
-// The nl = n - nres others come back newest first -- task nl - 1, nl - 2, ...,
-// 0 -- because pass 1 read them in increasing order, so the later ones are the
-// likeliest to be still in L2 when the tensor is larger than L2.  Quantizing
-// on-chip task k frees its slot for the k-th of those, and then the q-th
-// follows the (q - kStage)-th through the same slot.
+// Pass 2 of one warp with tasks tw .. tw + n - 1.  Pass 1 left the last
+// nres = min(kStage, n) of them in the warp's shared-memory slots (task
+// n - nres + k in slot (n - nres + k) % kStage) and the first nt (at most
+// kTmTasks) in the warp's tensor-memory columns (task j at column tcol + 16 j);
+// the nl = n - nres - nt in between come back from L2, newest first -- task
+// nt + nl - 1, nt + nl - 2, ..., nt -- because pass 1 read them in increasing
+// order, so the later ones are the likeliest to be still in L2.  Order: the
+// slot tasks (each one's slot then takes the next refill), the
+// tensor-memory tasks (while the refills are in flight), the refills.
 template <bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const FusedArgs& a, const GroupTab& gt, Ring& r,
                                             const uint64_t* rtab, Pass2Q<GROUPED>& pq, uint32_t gen, int tw, int n,
-                                            const LaneC& lc, const float* ssm) {
+                                            int nt, uint32_t tcol, const LaneC& lc, const float* ssm) {
     const uint64_t pol = l2_policy_evict_first();   // last use
     const int nres = n < kStage ? n : kStage;
-    const int nl = n - nres;
+    const int nl = n - nres - nt;
     DstCursor<GROUPED> rp, lq;
     SrcCursor<GROUPED> lp;
     rp.init(a, gt, tw + n - nres);
     if (nl > 0) {
-        lq.init(a, gt, tw + nl - 1);
-        lp.init(a, gt, tw + nl - 1);
+        lq.init(a, gt, tw + nt + nl - 1);
+        lp.init(a, gt, tw + nt + nl - 1);
     }
+    uint4 u[4];
     int s = (n - nres) % kStage;
     for (int k = 0; k < nres; ++k) {
-        quantize_any<GROUPED, SMOOTH>(a, r.slot(s), rp, lc, pq.at(a, rp, gen), rtab, ssm);
-        rp.next(a, gt);
+        load_slot(r.slot(s), lc, u);
         __syncwarp();   // every lane is done reading the slot
         if (k < nl) {
             stage<GROUPED>(tmap, a, r, s, lp, pol, lc.lane);
             lp.prev(a, gt);
         }
+        quantize_any<GROUPED, SMOOTH>(a, u, rp, lc, pq.at(a, rp, gen), rtab, ssm);
+        rp.next(a, gt);
         s = (s + 1 == kStage) ? 0 : s + 1;
     }
-    // s is back at the slot of the first on-chip task, where the first refill lands.
+    if (nt > 0) {
+        DstCursor<GROUPED> tp;
+        tp.init(a, gt, tw);
+        for (int j = 0; j < nt; ++j) {
+            load_tmem(tcol + 16u * (uint32_t)j, u);
+            quantize_any<GROUPED, SMOOTH>(a, u, tp, lc, pq.at(a, tp, gen), rtab, ssm);
+            tp.next(a, gt);
+        }
+    }
+    // s is back at the slot of the first slot task, where the first refill lands.
     for (int q = 0; q < nl; ++q) {
         land(r, s, a);
-        quantize_any<GROUPED, SMOOTH>(a, r.slot(s), lq, lc, pq.at(a, lq, gen), rtab, ssm);
-        lq.prev(a, gt);
+        load_slot(r.slot(s), lc, u);
         __syncwarp();
         if (q + kStage < nl) {
             stage<GROUPED>(tmap, a, r, s, lp, pol, lc.lane);
             lp.prev(a, gt);
         }
+        quantize_any<GROUPED, SMOOTH>(a, u, lq, lc, pq.at(a, lq, gen), rtab, ssm);
+        lq.prev(a, gt);
         s = (s + 1 == kStage) ? 0 : s + 1;
     }
 }
@@ -975,7 +1001,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __shared__ int s_off[GROUPED ? kMaxFusedGroups + 1 : 1];
     __shared__ int s_blk[GROUPED ? kMaxFusedGroups + 1 : 1];
     __shared__ __align__(16) float s_smooth[SMOOTH ? kMaxSmoothK : 4];
-    __shared__ uint32_t s_amax, s_gen;
+    __shared__ uint32_t s_amax, s_gen, s_tmem;
     __shared__ int s_ok;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x;
@@ -986,6 +1012,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
     int n = t0 + cnt * (warp + 1) / kFWarps - tw;
     if (tid == 0) s_gen = (uint32_t)(ld_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x) >> 32) + 1u;
     if (tid < kStage * kFWarps) mbar_init(&sbar[tid], 1);
+    // Tensor memory (all 512 columns: 64 per warp, in the warp's own lane
+    // quarter) when some warp has more tasks than shared-memory slots.
+    if (a.tm_tasks > 0 && warp == 0) {
+        tmem_alloc(&s_tmem, 512);
+        tmem_relinquish();
+    }
     GroupTab gt;
     gt.off = s_off;
     gt.blk = s_blk;
@@ -1038,8 +1070,16 @@ __global__ void __launch_bounds__(kFThreads, 1)
     r.phase = 0;
     r.box_bytes = box_bytes;
     if (lane == 0) prefetch_tmap(&tmap);
+    // this warp's first nt tasks stay in tensor memory, at columns tcol + 16 j
+    const int nt = max(0, min(a.tm_tasks, n - kStage));
+    uint32_t tcol = 0;
+    if (a.tm_tasks > 0) {
+        tc_fence_after();
+        tcol = s_tmem + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * 16 * kTmTasks);
+    }
 
-    // ---- pass 1: amax through the slot ring; the last kStage tasks stay on chip
+    // ---- pass 1: amax through the slot ring; the first nt tasks are parked in
+    // tensor memory, the last kStage stay in their slots
     const LaneC lc = make_lanec(lane);
     uint32_t acc = 0;      // packed BF16 running max |x|
     float accf = 0.0f;     // pre-scaled form: running max |x s|
@@ -1053,7 +1093,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
 #pragma unroll
         for (int i = 0; i < kStage; ++i) {
             if (i < n) {
-                stage_cp<GROUPED>(a, r, i, sp, lc, i >= n - kStage ? pol_last : pol_keep);
+                stage_cp<GROUPED>(a, r, i, sp, lc, (i < nt || i >= n - kStage) ? pol_last : pol_keep);
                 sp.next(a, gt);
             }
             cp_async_commit();
@@ -1079,27 +1119,34 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 seg_now = lp.seg;
                 lp.next(a, gt);
             }
-            const char* sb = r.slot(s);
+            uint4 u[4];
+            load_slot(r.slot(s), lc, u);
             if constexpr (SMOOTH) {
                 const float* sb2 = s_smooth + seg_now * kTaskVals;
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
-                    accf = fmaxf(accf, absmax8_smooth(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q]),
-                                                      smooth_unit(sb2, lane, 2 * q), smooth_unit(sb2, lane, 2 * q + 1)));
+                    accf = fmaxf(accf, absmax8_smooth(u[q], smooth_unit(sb2, lane, 2 * q),
+                                                      smooth_unit(sb2, lane, 2 * q + 1)));
             } else {
 #pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    acc = bmax_abs(acc, absmax8_packed(*reinterpret_cast<const uint4*>(sb + lc.ld_off[q])));
+                for (int q = 0; q < 4; ++q) acc = bmax_abs(acc, absmax8_packed(u[q]));
+            }
+            if (i < nt) {
+                const uint32_t w[16] = {u[0].x, u[0].y, u[0].z, u[0].w, u[1].x, u[1].y, u[1].z, u[1].w,
+                                        u[2].x, u[2].y, u[2].z, u[2].w, u[3].x, u[3].y, u[3].z, u[3].w};
+                tmem_st_32x32b_x16(tcol + 16u * (uint32_t)i, w);
             }
             if (i + kStage < n) {
                 __syncwarp();   // every lane is done reading the slot
-                stage_cp<GROUPED>(a, r, s, sp, lc, i + kStage >= n - kStage ? pol_last : pol_keep);
+                stage_cp<GROUPED>(a, r, s, sp, lc,
+                                  (i + kStage < nt || i + kStage >= n - kStage) ? pol_last : pol_keep);
                 sp.next(a, gt);
             }
             cp_async_commit();
             s = (s + 1 == kStage) ? 0 : s + 1;
         }
         cp_async_wait<0>();
+        if (nt > 0) tmem_st_wait();
         __syncwarp();
         if constexpr (GROUPED) {
             if (n > 0) {
@@ -1118,24 +1165,21 @@ __global__ void __launch_bounds__(kFThreads, 1)
     }
     __syncthreads();
 
-    // ---- grid barrier: publish this CTA's word, gather everyone's
+    // ---- grid barrier: arrive with this CTA's amax, wait for everyone's
     if (tid == 0) {
         uint32_t b = 0;
         if constexpr (!GROUPED)
             for (int w = 0; w < kFWarps; ++w) b = max(b, red[w]);
+        st_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x, (uint64_t)gen << 32);   // next call: gen + 1
         // grouped: every warp's folds (ordered before this by the CTA barrier)
-        // become visible with the word
+        // are released with the arrival
         if constexpr (GROUPED) fence_acq_rel_gpu();
-        st_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x, ((uint64_t)gen << 32) | b);
-    }
-    if (warp == 0) {
+        grid_arrive(a.bar, gen, b, blockIdx.x == 0);
         uint32_t amax_bits = 0;
-        const bool got = grid_amax(a.part, G, gen, a.limit, a.err, lane, amax_bits);
-        if constexpr (GROUPED) fence_acq_rel_gpu();   // the group words after every CTA's word
-        if (lane == 0) {
-            s_ok = got ? 1 : 0;
-            s_amax = amax_bits;
-        }
+        const bool got = grid_wait(a.bar, gen, G, a.limit, a.err, amax_bits);
+        if constexpr (GROUPED) fence_acq_rel_gpu();   // the group words after every CTA's arrival
+        s_ok = got ? 1 : 0;
+        s_amax = amax_bits;
     }
     __syncthreads();
     const bool ok = s_ok != 0;
@@ -1150,7 +1194,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
             fill_rtab(rtab, pq.q.g, tid);
             __syncthreads();
         }
-        fused_pass2<GROUPED, SMOOTH>(&tmap, a, gt, r, rtab, pq, gen, tw, n, lc, s_smooth);
+        fused_pass2<GROUPED, SMOOTH>(&tmap, a, gt, r, rtab, pq, gen, tw, n, nt, tcol, lc, s_smooth);
+    }
+    if (a.tm_tasks > 0) {   // every warp's tensor-memory reads are done (tcgen05.wait::ld after each)
+        tc_fence_before();
+        __syncthreads();
+        if (warp == 0) tmem_dealloc(s_tmem, 512);
     }
     pdl_launch_dependents();
 }
@@ -1326,7 +1375,11 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     a.codes = codes;
     a.scales = scales;
     a.part = reinterpret_cast<uint64_t*>(workspace);
+    a.bar = reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_bar_off());
     a.gword = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(workspace) + quant_ws_gword_off(groups));
+    // Warps with more tasks than slots park up to kTmTasks of them in tensor
+    // memory, so that pass 2 re-reads none (or fewer) from L2.
+    a.tm_tasks = per_warp > kStage ? kTmTasks : 0;
     a.offsets = offsets;
     a.groups = grouped ? groups : 1;
     a.smooth = smooth;
