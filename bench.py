@@ -19,6 +19,17 @@ pair of CUDA events; per-kernel durations come from a copy of the same graph
 with an event between consecutive kernels.  N > 1 runs N independent
 replicas (the path needs no exchange between GPUs), one process per GPU.
 
+With the default workload on one GPU the line also carries every other
+configuration of the path, each with its own roofline, clocks and CPU
+baseline: `quant_c2` (the activation quantizer on [8192,4096] Laplace with
+outliers, plus its pre-scaled and MXFP4 forms), `weight_quant` (16x16 blocks
+on [14336,4096]), `decode` (m in {1, 8, 32, 64}: step, quantizer, GEMM with
+the weight-stream roofline, and the same GEMM as W4A16) and `moe` (grouped
+quantizer and grouped GEMM, FP4 and HBM fractions, MMA padding).  Per-kernel
+loops run at least 200 launches whatever --steps is.  `warmup` echoes the
+requested count; `warmup_calls_run` counts the untimed calls actually made
+(eager first calls and graph replays).
+
 --impl reference times the CPU oracle (plain C, binary64 GEMM) on a bounded
 sample of the same workload: rank 0 only.
 """
@@ -55,6 +66,14 @@ def mx_quant_bytes(rows: int, k: int) -> int:
     packed codes and one E8M0 scale per 32 values."""
     n = rows * k
     return 2 * n + n // 2 + n // 32
+
+
+_T_START = time.perf_counter()
+
+
+def progress(what: str) -> None:
+    """One line on stderr per section, with the seconds since start."""
+    print(f"[bench +{time.perf_counter() - _T_START:6.1f} s] {what}", file=sys.stderr, flush=True)
 
 
 def load_peaks():
@@ -120,6 +139,7 @@ class ClockSampler:
 
     def start(self):
         if self.ok:
+            self._stop.clear()
             self._thr = threading.Thread(target=self._run, daemon=True)
             self._thr.start()
             time.sleep(0.02)
@@ -309,10 +329,13 @@ class Prefill:
 class Decode(Prefill):
     name = "decode"
 
-    def __init__(self, nv, torch, dev, m=64):
+    def __init__(self, nv, torch, dev, m=64, w_host=None):
         import workloads as W
         self.m, self.n, self.k = m, 25600, 5120
-        self._build(nv, torch, dev, *W.decode(m))
+        w = w_host if w_host is not None else W.decode_weights()
+        self._build(nv, torch, dev, W.decode_activations(m), w)
+        self.abytes = quant_bytes(m, self.k) - 2 * m * self.k   # A codes, scales and g, read by the GEMM
+        self.cbytes = 2 * m * self.n
 
     def config(self):
         return {"workload": f"decode W4A4: A bf16 [{self.m},{self.k}] quantized per call x W nvfp4 "
@@ -391,7 +414,7 @@ class Moe:
         a, off, w = W.moe(0)
         E, N, K = w.shape
         self.E, self.n, self.k, self.rows = E, N, K, a.shape[0]
-        self.a_host = a
+        self.a_host, self.off_host, self.w_host = a, off, w
         a0 = to_device(torch, a, dev)
         self.off = torch.from_numpy(off).to(dev)
         wdev = to_device(torch, w.reshape(E * N, K), dev)
@@ -411,6 +434,8 @@ class Moe:
         self.c = [c0] + [torch.empty_like(c0) for _ in range(R - 1)]
         self.flops = 2.0 * self.rows * N * K
         self.qbytes = quant_bytes(self.rows, K, E)
+        # the grouped GEMM reads every expert's weights and A's codes and scales once, writes C
+        self.gemm_bytes = nbytes(b0[0], b0[1]) + quant_bytes(self.rows, K, E) - 2 * self.rows * K + nbytes(c0)
         self.launches_per_step = 2                    # one-launch grouped quantizer, grouped GEMM
 
     def quantize(self, i):
@@ -431,7 +456,17 @@ class Moe:
         return self.c[i % self.R]
 
     def gemm_label(self):
-        return "gemm_kernel<grouped> (tcgen05 mxf4nvf4; 128 x 192 tiles per expert group)"
+        return "gemm_pair_kernel<grouped> (tcgen05 mxf4nvf4, cta_group::2; 256 x 256 tiles per expert)"
+
+    def padding(self):
+        """Rows of tensor-core work per expert, as the grouped GEMM tiles them
+        (experts of >= 192 rows on average take 256-row pair tiles), against
+        the rows that hold tokens."""
+        sizes = np.diff(self.off.cpu().numpy().astype(np.int64))
+        tile = 256 if sizes.sum() >= 192 * len(sizes) else 128
+        padded = int(np.sum(-(-sizes // tile) * tile))
+        return {"token_rows": int(sizes.sum()), "mma_rows": padded, "tile_rows": tile,
+                "padding_frac": 1.0 - sizes.sum() / padded if padded else 0.0}
 
     def config(self):
         return {"workload": f"MoE grouped W4A4: {self.rows // 8} tokens top-8 of {self.E} experts, A bf16 "
@@ -510,6 +545,24 @@ def graph_seconds(torch, stream, fn, R, n):
     return e0.elapsed_time(e1) * 1e-3 / n
 
 
+def timed_loop(torch, stream, fn, R, n, sampler):
+    """(average seconds per call, clocks during the loop) of n graph-replayed
+    calls of fn, after an untimed pass over every graph and a rest."""
+    g = StepGraphs(torch, stream, fn, R, n)
+    g.warm(0)
+    time.sleep(REST_S)
+    t0 = time.perf_counter()
+    e0, e1 = g.run()
+    stream.synchronize()
+    t1 = time.perf_counter()
+    return e0.elapsed_time(e1) * 1e-3 / n, sampler.summary(t0, t1)
+
+
+# Launches per per-kernel timing loop, whatever --steps is.
+KERNEL_ITERS = 200
+NOMINAL_FP4_TFLOPS = 9000.0   # B200 dense FP4, datasheet (context beside the measured-derived peak)
+
+
 def cpu_baseline_prefill(wl, max_seconds=12.0):
     """The oracle as it stands on the host cores: dynamic quantization of the
     whole A plus the binary64 GEMM of a sample of rows (W reconstructed once,
@@ -540,6 +593,60 @@ def cpu_baseline_prefill(wl, max_seconds=12.0):
                       f"{wl.m} rows against W [{wl.n},{wl.k}] ({dt:.1f} s)"}
 
 
+def cpu_baseline_weight_quant(w_bits):
+    import oracle as O
+    t = time.perf_counter()
+    O.quantize_2d(w_bits)
+    dt = time.perf_counter() - t
+    rows, k = w_bits.shape
+    return {"value": quant_bytes(rows, k) / dt / 1e9, "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"one full 16x16-block quantization of [{rows},{k}] ({dt:.2f} s)"}
+
+
+def cpu_baseline_decode(a_bits, wh, n, k, max_rows=8):
+    """The oracle on one decode step: dynamic quantization of A, then the
+    binary64 GEMM of up to max_rows of its rows against the reconstructed W
+    (W reconstructed once, outside the timing)."""
+    import oracle as O
+    m = a_bits.shape[0]
+    rows = min(m, max_rows)
+    sel = np.linspace(0, m - 1, rows).astype(np.int64)
+    t = time.perf_counter()
+    ac, asf, ga = O.quantize_1d(a_bits)
+    O.gemm_f64_rows(O.dequantize(ac, asf, ga), wh, sel)
+    dt = time.perf_counter() - t
+    return {"value": 2.0 * rows * n * k / dt / 1e12, "unit": "TFLOP/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"dynamic quantization of A [{m},{k}] + binary64 GEMM of {rows} of {m} rows against "
+                      f"W [{n},{k}] ({dt:.2f} s)"}
+
+
+def cpu_baseline_moe(a_bits, off, w_bits, experts=4, rows_per_expert=2):
+    """The oracle on the MoE step, sampled: grouped dynamic quantization of all
+    of A, then for a few experts their weights' 2D quantization and the
+    binary64 GEMM of a few of their rows."""
+    import oracle as O
+    E, N, K = w_bits.shape
+    t = time.perf_counter()
+    ac, asf, ga = O.quantize_1d_grouped(a_bits, off)
+    flops = 0.0
+    row0 = 0
+    picked = np.linspace(0, E - 1, experts).astype(int)
+    for e in range(E):
+        r0, r1 = int(off[e]), int(off[e + 1])
+        if e in picked and r1 > r0:
+            wc, wsf, gw = O.quantize_2d(np.ascontiguousarray(w_bits[e]))
+            sel = np.linspace(0, r1 - r0 - 1, min(rows_per_expert, r1 - r0)).astype(np.int64)
+            ah = O.dequantize(ac[r0:r1], asf, float(ga[e]), sf_row0=row0, k=K)
+            O.gemm_f64_rows(ah, O.dequantize(wc, wsf, gw), sel)
+            flops += 2.0 * sel.size * N * K
+        row0 += O.scale_rows(r1 - r0)
+    dt = time.perf_counter() - t
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"grouped dynamic quantization of A [{a_bits.shape[0]},{K}] ({E} groups) + for {experts} "
+                      f"experts their 2D weight quantization and the binary64 GEMM of {rows_per_expert} rows "
+                      f"({dt:.2f} s)"}
+
+
 def cpu_baseline_quant(wl, max_seconds=12.0):
     import oracle as O
     t = time.perf_counter()
@@ -547,6 +654,136 @@ def cpu_baseline_quant(wl, max_seconds=12.0):
     dt = time.perf_counter() - t
     return {"value": wl.qbytes / dt / 1e9, "unit": "GB/s", "cores": O.num_threads(), "kind": "oracle",
             "sample": f"one full quantization of [{wl.rows},{wl.k}] ({dt:.2f} s)"}
+
+
+# ---- the other configurations, measured beside the headline -------------------------------------
+
+def _roofline(bound, kernel, achieved, peak, unit, traffic, avg_s, clocks, **extra):
+    r = {"bound": bound, "kernel": kernel, "achieved": achieved, "peak": peak, "unit": unit,
+         "frac": achieved / peak, "traffic": traffic, "avg_launch_ms": avg_s * 1e3,
+         "launches_timed": KERNEL_ITERS, "clocks": clocks}
+    r.update(extra)
+    return r
+
+
+def measure_quant_c2(nv, torch, dev, cs, sampler, peaks, with_cpu):
+    """The activation quantizer on [8192, 4096] Laplace with outliers, and the
+    16 x 16-block weight quantizer on [14336, 4096]."""
+    import workloads as W
+    hbm = peaks["hbm_gbs"]
+    wl = Quant(nv, torch, dev)
+    n = 1000
+    step_s, clk = timed_loop(torch, cs, wl.step, wl.R, n, sampler)
+    gbs = wl.qbytes / step_s / 1e9
+    q = {"workload": wl.config()["workload"], "avg_ms": step_s * 1e3, "launches_timed": n, "gbs": gbs,
+         "frac_hbm": gbs / hbm, "algorithmic_bytes": wl.qbytes,
+         "roofline": _roofline("hbm", "quant1d_fused_kernel (one cooperative launch)", gbs, hbm, "GB/s",
+                               load_traffic("quant_quant"), step_s, clk),
+         "clocks": clk,
+         "l2": f"{wl.R} rotating buffer sets of {wl.set_bytes / 1e6:.1f} MB (inputs larger than L2 between uses)"}
+    wl.quantize_smooth(0)
+    s_s, s_clk = timed_loop(torch, cs, wl.quantize_smooth, wl.R, KERNEL_ITERS, sampler)
+    s_bytes = wl.qbytes + 4 * wl.k
+    q["smooth"] = {"what": "x * s[column], s log-uniform in [1/8, 8], folded into the one-launch quantizer",
+                   "avg_ms": s_s * 1e3, "gbs": s_bytes / s_s / 1e9, "frac_hbm": s_bytes / s_s / 1e9 / hbm,
+                   "clocks": s_clk}
+    wl.quantize_mx(0)
+    x_s, x_clk = timed_loop(torch, cs, wl.quantize_mx, wl.R, KERNEL_ITERS, sampler)
+    x_bytes = mx_quant_bytes(wl.rows, wl.k)
+    q["mxfp4"] = {"what": "the same activations -> mxfp4 (E8M0 per 32 values, no tensor scale), one pass",
+                  "avg_ms": x_s * 1e3, "gbs": x_bytes / x_s / 1e9, "frac_hbm": x_bytes / x_s / 1e9 / hbm,
+                  "clocks": x_clk}
+    w_s, w_clk = timed_loop(torch, cs, wl.quantize_weight, wl.RW, KERNEL_ITERS, sampler)
+    w_gbs = wl.wqbytes / w_s / 1e9
+    wq = {"workload": f"weight quantizer: bf16 [{wl.wn},{wl.k}] N(0,0.02) -> nvfp4, 16x16 blocks",
+          "avg_ms": w_s * 1e3, "gbs": w_gbs, "frac_hbm": w_gbs / hbm, "algorithmic_bytes": wl.wqbytes,
+          "roofline": _roofline("hbm", "amax_kernel + quant2d_kernel", w_gbs, hbm, "GB/s", None, w_s, w_clk),
+          "clocks": w_clk}
+    if with_cpu:
+        q["cpu_baseline"] = cpu_baseline_quant(wl)
+        wq["cpu_baseline"] = cpu_baseline_weight_quant(W.quant_weight(0, wl.wn, wl.k))
+    del wl
+    torch.cuda.empty_cache()
+    return q, wq
+
+
+def measure_decode(nv, torch, dev, cs, sampler, peaks, with_cpu, ms=(1, 8, 32, 64)):
+    """The decode sweep: per m, the step (quantize + GEMM), each kernel alone,
+    and the same GEMM as W4A16; the GEMM's roofline is the HBM stream of the
+    weights and scales (plus A's codes and C)."""
+    import workloads as W
+    hbm = peaks["hbm_gbs"]
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    w_host = W.decode_weights()
+    wh = None
+    if with_cpu:
+        import oracle as O
+        wh = O.dequantize(*O.quantize_2d(w_host))
+    out = {"workload": "decode W4A4: A bf16 [m,5120] quantized per call x W nvfp4 [25600,5120] (2D blocks) "
+                       "-> C bf16 [m,25600]", "per_m": {}}
+    for m in ms:
+        progress(f"decode m = {m}")
+        wl = Decode(nv, torch, dev, m=m, w_host=w_host)
+        n = 1000
+        step_s, clk = timed_loop(torch, cs, wl.step, wl.R, n, sampler)
+        q_s, q_clk = timed_loop(torch, cs, lambda i: wl.quantize(i), wl.R, KERNEL_ITERS, sampler)
+        g_s, g_clk = timed_loop(torch, cs, lambda i: wl.gemm(i), wl.R, KERNEL_ITERS, sampler)
+
+        def w16(i):
+            j = i % wl.R
+            nv.gemm_w4a16(wl.a[j], wl.w[j], out=wl.c[j])
+        t16, clk16 = timed_loop(torch, cs, w16, wl.R, KERNEL_ITERS, sampler)
+        gbytes = wl.wbytes + wl.abytes + wl.cbytes
+        g_gbs = gbytes / g_s / 1e9
+        r = {"step_ms": step_s * 1e3, "steps_timed": n, "quantize_ms": q_s * 1e3, "gemm_ms": g_s * 1e3,
+             "gemm_tflops": wl.flops / g_s / 1e12, "gemm_frac_fp4": wl.flops / g_s / 1e12 / fp4_peak,
+             "weight_stream_gbs": wl.wbytes / g_s / 1e9, "weight_stream_frac_hbm": wl.wbytes / g_s / 1e9 / hbm,
+             "step_weight_stream_gbs": wl.wbytes / step_s / 1e9,
+             "roofline": _roofline("hbm", wl.gemm_label(), g_gbs, hbm, "GB/s",
+                                   load_traffic("gemm_decode") if m == 64 else None, g_s, g_clk,
+                                   algorithmic_bytes=gbytes),
+             "w4a16": {"gemm_ms": t16 * 1e3, "weight_stream_gbs": (wl.wbytes + 2 * m * wl.k) / t16 / 1e9,
+                       "frac_hbm": (wl.wbytes + 2 * m * wl.k) / t16 / 1e9 / hbm, "clocks": clk16},
+             "clocks": clk, "quantize_clocks": q_clk}
+        if with_cpu:
+            r["cpu_baseline"] = cpu_baseline_decode(wl.a_host, wh, wl.n, wl.k)
+        out["per_m"][str(m)] = r
+        del wl, w16
+        torch.cuda.empty_cache()
+    return out
+
+
+def measure_moe(nv, torch, dev, cs, sampler, peaks, with_cpu):
+    """The MoE layer: grouped quantization of the routed activations and the
+    grouped GEMM over 128 experts.  Below the FP4 ridge (about 565 flop per
+    byte against ~1000), so the GEMM's roofline is the HBM traffic of the
+    expert weights, A's codes and C; the FP4 fraction is reported beside it."""
+    hbm = peaks["hbm_gbs"]
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    wl = Moe(nv, torch, dev)
+    n = 200
+    step_s, clk = timed_loop(torch, cs, wl.step, wl.R, n, sampler)
+    q_s, q_clk = timed_loop(torch, cs, lambda i: wl.quantize(i), wl.R, KERNEL_ITERS, sampler)
+    g_s, g_clk = timed_loop(torch, cs, lambda i: wl.gemm(i), wl.R, KERNEL_ITERS, sampler)
+    tfl = wl.flops / g_s / 1e12
+    g_gbs = wl.gemm_bytes / g_s / 1e9
+    t_tensor, t_hbm = wl.flops / (fp4_peak * 1e12), wl.gemm_bytes / (hbm * 1e9)
+    out = {"workload": wl.config()["workload"], "step_ms": step_s * 1e3, "steps_timed": n,
+           "step_tflops": wl.flops / step_s / 1e12, "quantize_ms": q_s * 1e3,
+           "quantize_gbs": wl.qbytes / q_s / 1e9, "quantize_frac_hbm": wl.qbytes / q_s / 1e9 / hbm,
+           "gemm_ms": g_s * 1e3, "gemm_tflops": tfl, "gemm_frac_fp4": tfl / fp4_peak,
+           "gemm_frac_nominal_fp4": tfl / NOMINAL_FP4_TFLOPS, "gemm_gbs": g_gbs, "gemm_frac_hbm": g_gbs / hbm,
+           "roofline": (_roofline("hbm", wl.gemm_label(), g_gbs, hbm, "GB/s", load_traffic("gemm_moe"), g_s, g_clk,
+                                  algorithmic_bytes=wl.gemm_bytes, tensor_bound_ms=t_tensor * 1e3)
+                        if t_hbm >= t_tensor else
+                        _roofline("tensor", wl.gemm_label(), tfl, fp4_peak, "TFLOP/s", load_traffic("gemm_moe"),
+                                  g_s, g_clk, hbm_bound_ms=t_hbm * 1e3)),
+           "mma_padding": wl.padding(), "clocks": clk, "quantize_clocks": q_clk}
+    if with_cpu:
+        out["cpu_baseline"] = cpu_baseline_moe(wl.a_host, wl.off_host, wl.w_host)
+    del wl
+    torch.cuda.empty_cache()
+    return out
 
 
 # ---- the two arms ------------------------------------------------------------------------------
@@ -631,12 +868,14 @@ def run_ours(args):
     import nvfp4_w4a4_quantized_05_b200 as nv
     nv.lib()
     peaks = load_peaks()
+    progress(f"building the {args.workload} workload")
     wl = {"prefill": Prefill, "decode": Decode, "quant": Quant, "moe": Moe}[args.workload]
     wl = wl(nv, torch, dev, m=args.decode_m) if args.workload == "decode" else wl(nv, torch, dev)
     cs = torch.cuda.Stream(dev)
     sampler = ClockSampler(local)
     sampler.start()
 
+    progress("timed steps")
     # capture, then warm-up (eager first calls + one replay of every graph)
     steps = StepGraphs(torch, cs, wl.step, wl.R, args.steps)
     warm = steps.warm(max(3, args.warmup))
@@ -657,7 +896,7 @@ def run_ours(args):
     del steps
 
     # ---- per-kernel times: each kernel alone, back to back over the same buffer sets ----
-    kiters = max(10, min(args.steps, 200))
+    kiters = max(KERNEL_ITERS, min(args.steps, 2000))
     ktimes, kclocks = [], []
     for f in wl.kernels:
         time.sleep(REST_S)
@@ -710,7 +949,8 @@ def run_ours(args):
     else:
         value = world * wl.qbytes * args.steps / total / 1e9
         line.update({"value": value, "unit": "GB/s"})
-    line.update({"n_gpus": world, "steps": args.steps, "warmup": warm, "ms_per_step": ms,
+    line.update({"n_gpus": world, "steps": args.steps, "warmup": args.warmup, "warmup_calls_run": warm,
+                 "ms_per_step": ms,
                  "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                  "dtype": "fp4 (e2m1 x e2m1, e4m3 block scales, f32 accumulate)",
                  "data": "synthetic (seeded; see workloads/)"})
@@ -733,6 +973,8 @@ def run_ours(args):
                             "frac": g_tflops / fp4_peak, "traffic": load_traffic(f"gemm_{wl.name}"),
                             "peak_note": f"{peaks['source']} bf16 burst {peaks['bf16_tflops']} x {FP4_PER_BF16} "
                                          "(dense FP4 / BF16 nominal ratio)",
+                            "frac_of_nominal_fp4": g_tflops / NOMINAL_FP4_TFLOPS,
+                            "nominal_fp4_tflops": NOMINAL_FP4_TFLOPS,
                             "avg_launch_ms": g_avg * 1e3, "launches_timed": kiters, "clocks": kclocks[1]}
     else:
         line["roofline"] = {"bound": "hbm", "kernel": "quant1d_fused_kernel (one cooperative launch)",
@@ -816,9 +1058,29 @@ def run_ours(args):
     line["gpu_launches"] = wl.launches_per_step * args.steps
     line["clocks"] = clocks
     sampler.stop()
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    with_cpu = rank == 0 and world == 1 and not args.no_cpu_baseline
+    progress("cpu baseline")
+    if with_cpu:
         line["cpu_baseline"] = (cpu_baseline_quant(wl) if wl.name == "quant" else
-                                cpu_baseline_prefill(wl) if wl.name in ("prefill", "decode") else None)
+                                cpu_baseline_prefill(wl) if wl.name in ("prefill", "decode") else
+                                cpu_baseline_moe(wl.a_host, wl.off_host, wl.w_host))
+    if args.workload == "prefill" and not args.no_extra and world == 1:
+        # every other configuration of the path, each measured here with its
+        # own roofline, clocks and CPU baseline (one GPU: per-GPU figures)
+        del wl
+        import gc
+        gc.collect()
+        torch.cuda.empty_cache()
+        sampler.start()
+        progress("activation and weight quantizers")
+        line["quant_c2"], line["weight_quant"] = measure_quant_c2(nv, torch, dev, cs, sampler, peaks, with_cpu)
+        progress("decode sweep")
+        line["decode"] = measure_decode(nv, torch, dev, cs, sampler, peaks, with_cpu)
+        progress("moe")
+        line["moe"] = measure_moe(nv, torch, dev, cs, sampler, peaks, with_cpu)
+        progress("done")
+        sampler.stop()
+        nv.check_device_error()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -839,6 +1101,8 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="prefill: skip the other configurations (activation and weight quantizers, decode sweep, MoE)")
     args = ap.parse_args(argv)
     if args.steps is None:
         args.steps = (20 if args.impl == "reference" else

@@ -195,10 +195,16 @@ def prefill(seed: int = 0, m: int = 4096, n: int = 14336, k: int = 4096):
     return a, w
 
 
+def decode_activations(m: int, seed: int = 0, k: int = 5120):
+    return gaussian_bf16((m, k), seed, 7 + m, 1.0, outlier_frac=0.01)
+
+
+def decode_weights(seed: int = 0, n: int = 25600, k: int = 5120):
+    return gaussian_bf16((n, k), seed, 6000, 0.02)
+
+
 def decode(m: int, seed: int = 0, n: int = 25600, k: int = 5120):
-    a = gaussian_bf16((m, k), seed, 7 + m, 1.0, outlier_frac=0.01)
-    w = gaussian_bf16((n, k), seed, 6000, 0.02)
-    return a, w
+    return decode_activations(m, seed, k), decode_weights(seed, n, k)
 
 
 def moe_routing(seed: int = 0, tokens: int = 4096, experts: int = 128, top_k: int = 8):
