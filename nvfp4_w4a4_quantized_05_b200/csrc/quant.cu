@@ -199,6 +199,33 @@ __device__ __forceinline__ void fill_rtab(uint64_t* rtab, float g, int tid) {
     if (tid < 128) rtab[tid] = pack_rr(block_recip(__fmul_rn(e4m3_to_f32((uint32_t)tid), g), g < kTinyG));
 }
 
+// Exact block scales without a division, for a BF16 block amax and a normal
+// 6 g (g >= 2^-64).  Write b = m_b 2^(e_b - 127) with m_b = 1 + i / 128 and
+// 6 g = m_k 2^(e_k - 127).  Scaling by a power of two does not round, so
+// RN(b / (6 g)) = RN(m_b / m_k) 2^(e_b - e_k) whenever the quotient is a
+// normal binary32 number.  qtab[i] holds the bits of RN((1 + i / 128) / m_k)
+// minus e_k << 23, so the quotient's bits are qtab[i] + (e_b << 23).  A
+// quotient below 2^-126 (E4M3 byte 0 either way) comes out as a binary32
+// subnormal or, below that, as a negative integer, clamped to +0; so does a
+// zero or BF16-subnormal b (its exponent sum is at most 128 - e_k, e_k >= 66).
+// No quotient overflows: with g from the tensor's own amax it is at most
+// 448 (1 + 2^-23).  The threads with tid in [0, 128) fill the table.
+__device__ __forceinline__ void fill_qtab(int32_t* qtab, float k6, int tid) {
+    if ((unsigned)tid < 128u) {
+        const uint32_t kb = __float_as_uint(k6);
+        const float mk = __uint_as_float((kb & 0x807FFFFFu) | (127u << 23));
+        const float q = __fdiv_rn(__uint_as_float((127u << 23) | ((uint32_t)tid << 16)), mk);
+        qtab[tid] = (int32_t)__float_as_uint(q) - (int32_t)(kb & 0x7F800000u);
+    }
+}
+// Scale bytes sf0 | sf1 << 8 of blocks 2 lane and 2 lane + 1, whose BF16
+// amaxes are the low and high halves of m (sign bits ignored).
+__device__ __forceinline__ uint32_t block_sf2_tab(uint32_t m, const int32_t* qtab) {
+    const int32_t q0 = max(qtab[m & 0x7Fu] + (int32_t)((m << 16) & 0x7F800000u), 0);
+    const int32_t q1 = max(qtab[(m >> 16) & 0x7Fu] + (int32_t)(m & 0x7F800000u), 0);
+    return cvt_e4m3x2(__int_as_float(q1), __int_as_float(q0));
+}
+
 __device__ __forceinline__ int64_t sf_tile_offset(int srow, int scol, int scale_cols) {
     return ((int64_t)(srow >> 7) * (scale_cols >> 2) + (scol >> 2)) * 512 + (srow & 31) * 16 +
            ((srow >> 5) & 3) * 4 + (scol & 3);
@@ -735,6 +762,42 @@ __device__ __forceinline__ uint64_t block_rr(uint32_t sf, const GroupQ& q) {
     return pack_rr(block_recip(__fmul_rn(e4m3_to_f32(sf), q.g), q.tiny));
 }
 
+// A lane's 16 code bytes and, from even lanes, the scale word of its lane pair.
+template <bool FULL, bool GROUPED>
+__device__ __forceinline__ void store_task(const FusedArgs& a, const uint4& q, uint32_t pair, const DstCursor<GROUPED>& t,
+                                           const LaneC& lc) {
+    const uint32_t word = __byte_perm(pair, __shfl_down_sync(kFull, pair, 1), 0x5410);
+    const bool even = (lc.lane & 1) == 0;
+    uint8_t* dst = a.codes + t.co + 16 * lc.lane;
+    uint32_t* sw = reinterpret_cast<uint32_t*>(a.scales + t.so + lc.s_off);
+    if (FULL) {
+        *reinterpret_cast<uint4*>(dst) = q;
+        if (even) *sw = word;
+    } else {
+        // Padding rows and values past k arrived as zeros: their scale bytes
+        // are 0, as the padded scale tile wants; no codes are stored there.
+        if (t.valid() && t.seg * kTaskVals + 32 * lc.lane < a.k) *reinterpret_cast<uint4*>(dst) = q;
+        if (even && t.seg * (kTaskVals / 16) + 2 * lc.lane < a.scale_cols) *sw = word;
+    }
+}
+
+// One tensor with g >= 2^-64: the block amaxes m come from pass 1 (packed
+// BF16, block 2 lane low), the scale bytes from the quotient table.
+template <bool FULL>
+__device__ __forceinline__ void quantize_plain(const FusedArgs& a, const uint4 (&u)[4], uint32_t m,
+                                               const DstCursor<false>& t, const LaneC& lc, const uint64_t* rtab,
+                                               const int32_t* qtab) {
+    const uint32_t pair = block_sf2_tab(m, qtab);
+    const uint64_t rr0 = rtab[pair & 0xFFu];
+    const uint64_t rr1 = rtab[pair >> 8];
+    uint4 q;
+    q.x = quant8(u[0], rr0);
+    q.y = quant8(u[1], rr0);
+    q.z = quant8(u[2], rr1);
+    q.w = quant8(u[3], rr1);
+    store_task<FULL, false>(a, q, pair, t, lc);
+}
+
 // Quantize one task whose values the lane holds in u (its 32 values, units
 // 4 lane .. 4 lane + 3 of the task).  FULL: the whole task is inside the
 // tensor.  One tensor: r from the per-CTA table; grouped: r computed per
@@ -780,19 +843,7 @@ __device__ __forceinline__ void quantize_vals(const FusedArgs& a, const uint4 (&
         q.z = quant8<TINY>(u[2], rr1);
         q.w = quant8<TINY>(u[3], rr1);
     }
-    const uint32_t word = __byte_perm(pair, __shfl_down_sync(kFull, pair, 1), 0x5410);
-    const bool even = (lc.lane & 1) == 0;
-    uint8_t* dst = a.codes + t.co + 16 * lc.lane;
-    uint32_t* sw = reinterpret_cast<uint32_t*>(a.scales + t.so + lc.s_off);
-    if (FULL) {
-        *reinterpret_cast<uint4*>(dst) = q;
-        if (even) *sw = word;
-    } else {
-        // Padding rows and values past k arrived as zeros: their scale bytes
-        // are 0, as the padded scale tile wants; no codes are stored there.
-        if (t.valid() && t.seg * kTaskVals + 32 * lc.lane < a.k) *reinterpret_cast<uint4*>(dst) = q;
-        if (even && t.seg * (kTaskVals / 16) + 2 * lc.lane < a.scale_cols) *sw = word;
-    }
+    store_task<FULL, GROUPED>(a, q, pair, t, lc);
 }
 template <bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void quantize_any(const FusedArgs& a, const uint4 (&u)[4], const DstCursor<GROUPED>& t,
@@ -939,10 +990,96 @@ struct Pass2Q {
 // order, so the later ones are the likeliest to be still in L2.  Order: the
 // slot tasks (each one's slot then takes the next refill), the
 // tensor-memory tasks (while the refills are in flight), the refills.
+// One tensor (not pre-scaled): the block amaxes of the tasks kept on chip,
+// computed in pass 1, and the per-CTA quotient table.  bm points at this
+// lane's word of on-chip task 0; task j's is kFWarps * 32 words further.
+struct OnChip {
+    const uint32_t* bm;
+    const int32_t* qtab;
+};
+template <bool GROUPED, bool SMOOTH>
+__device__ __forceinline__ void quantize_onchip(const FusedArgs& a, const uint4 (&u)[4], int j, const OnChip& oc,
+                                                const DstCursor<GROUPED>& t, const LaneC& lc, const GroupQ& gq,
+                                                const uint64_t* rtab, const float* ssm) {
+    if constexpr (!GROUPED && !SMOOTH) {
+        if (!gq.tiny) {   // warp-uniform
+            const uint32_t m = oc.bm[j * kFWarps * 32];
+            if (t.valid() && t.seg < a.full_segs)
+                quantize_plain<true>(a, u, m, t, lc, rtab, oc.qtab);
+            else
+                quantize_plain<false>(a, u, m, t, lc, rtab, oc.qtab);
+            return;
+        }
+    }
+    quantize_any<GROUPED, SMOOTH>(a, u, t, lc, gq, rtab, ssm);
+}
+
+// Pass 2 of the one-tensor form (g >= 2^-64) when every task of the warp is
+// on chip: tasks 0 .. nt - 1 in tensor memory, tasks nt .. n - 1 in slot
+// i % kStage, where pass 1 left them.  One loop in task order with little
+// live state: the values, the block amaxes from pass 1, the scale bytes from
+// the quotient table, and a destination cursor advanced in place.
+__device__ __forceinline__ void plain_pass2(const FusedArgs& a, const Ring& r, const LaneC& lc, int tw, int n, int nt,
+                                            uint32_t tcol, const uint32_t* bm, const uint64_t* rtab,
+                                            const int32_t* qtab) {
+    int row = tw / a.nseg, seg = tw - row * a.nseg;
+    const uint32_t kb2 = (uint32_t)(a.k >> 1);
+    auto scale_off = [&](int rw, int sg) {
+        const uint32_t rr = (uint32_t)rw;
+        return (rr >> 7) * a.sc4x512 + (rr & 31u) * 16u + ((rr >> 5) & 3u) * 4u + ((uint32_t)sg << 13);
+    };
+    uint32_t co = (uint32_t)row * kb2 + ((uint32_t)seg << 9);
+    uint32_t so = scale_off(row, seg);
+    uint8_t* const cbase = a.codes + 16 * lc.lane;
+    uint8_t* const sbase = a.scales + lc.s_off;
+    const bool even = (lc.lane & 1) == 0;
+    int s = nt % kStage;
+    for (int i = 0; i < n; ++i) {
+        uint4 u[4];
+        uint32_t m;
+        if (i < nt) {   // warp-uniform
+            load_tmem(tcol + 16u * (uint32_t)i, u);
+            m = bm[i * kFWarps * 32];
+        } else {
+            load_slot(r.slot(s), lc, u);
+            m = bm[(kTmTasks + i - nt) * kFWarps * 32];
+            s = (s + 1 == kStage) ? 0 : s + 1;
+        }
+        const uint32_t pair = block_sf2_tab(m, qtab);
+        const uint64_t rr0 = rtab[pair & 0xFFu];
+        const uint64_t rr1 = rtab[pair >> 8];
+        uint4 q;
+        q.x = quant8(u[0], rr0);
+        q.y = quant8(u[1], rr0);
+        q.z = quant8(u[2], rr1);
+        q.w = quant8(u[3], rr1);
+        const uint32_t word = __byte_perm(pair, __shfl_down_sync(kFull, pair, 1), 0x5410);
+        if (row < a.rows && seg < a.full_segs) {
+            *reinterpret_cast<uint4*>(cbase + co) = q;
+            if (even) *reinterpret_cast<uint32_t*>(sbase + so) = word;
+        } else {
+            // padding rows and values past k: no codes; zero scale bytes in the padded tile
+            if (row < a.rows && seg * kTaskVals + 32 * lc.lane < a.k) *reinterpret_cast<uint4*>(cbase + co) = q;
+            if (even && seg * (kTaskVals / 16) + 2 * lc.lane < a.scale_cols)
+                *reinterpret_cast<uint32_t*>(sbase + so) = word;
+        }
+        if (++seg == a.nseg) {
+            seg = 0;
+            ++row;
+            co = (uint32_t)row * kb2;
+            so = scale_off(row, 0);
+        } else {
+            co += kTaskVals / 2;
+            so += 8192u;   // 16 scale tiles of 512 bytes per segment
+        }
+    }
+}
+
 template <bool GROUPED, bool SMOOTH>
 __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const FusedArgs& a, const GroupTab& gt, Ring& r,
                                             const uint64_t* rtab, Pass2Q<GROUPED>& pq, uint32_t gen, int tw, int n,
-                                            int nt, uint32_t tcol, const LaneC& lc, const float* ssm) {
+                                            int nt, uint32_t tcol, const LaneC& lc, const float* ssm,
+                                            const OnChip& oc) {
     const uint64_t pol = l2_policy_evict_first();   // last use
     const int nres = n < kStage ? n : kStage;
     const int nl = n - nres - nt;
@@ -962,7 +1099,7 @@ __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const Fused
             stage<GROUPED>(tmap, a, r, s, lp, pol, lc.lane);
             lp.prev(a, gt);
         }
-        quantize_any<GROUPED, SMOOTH>(a, u, rp, lc, pq.at(a, rp, gen), rtab, ssm);
+        quantize_onchip<GROUPED, SMOOTH>(a, u, kTmTasks + k, oc, rp, lc, pq.at(a, rp, gen), rtab, ssm);
         rp.next(a, gt);
         s = (s + 1 == kStage) ? 0 : s + 1;
     }
@@ -971,7 +1108,7 @@ __device__ __forceinline__ void fused_pass2(const CUtensorMap* tmap, const Fused
         tp.init(a, gt, tw);
         for (int j = 0; j < nt; ++j) {
             load_tmem(tcol + 16u * (uint32_t)j, u);
-            quantize_any<GROUPED, SMOOTH>(a, u, tp, lc, pq.at(a, tp, gen), rtab, ssm);
+            quantize_onchip<GROUPED, SMOOTH>(a, u, j, oc, tp, lc, pq.at(a, tp, gen), rtab, ssm);
             tp.next(a, gt);
         }
     }
@@ -1003,6 +1140,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __shared__ __align__(16) float s_smooth[SMOOTH ? kMaxSmoothK : 4];
     __shared__ uint32_t s_amax, s_gen, s_tmem;
     __shared__ int s_ok;
+    constexpr bool kPlain = !GROUPED && !SMOOTH;
+    // one tensor: packed block amaxes of the tasks kept on chip, [task][warp][lane]
+    // (tensor-memory tasks 0 .. kTmTasks - 1, then the slot tasks)
+    __shared__ uint32_t s_bm[kPlain ? (kTmTasks + kStage) * kFWarps * 32 : 1];
+    __shared__ int32_t s_qtab[kPlain ? 128 : 1];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x;
     const int t0 = (int)((int64_t)a.tasks * blockIdx.x / G);
@@ -1010,7 +1152,39 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // Warp w takes a contiguous run of the CTA's tasks.
     const int tw = t0 + cnt * warp / kFWarps;
     int n = t0 + cnt * (warp + 1) / kFWarps - tw;
-    if (tid == 0) s_gen = (uint32_t)(ld_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x) >> 32) + 1u;
+    // this CTA's word: the generation of its last call (read early, used late)
+    const uint64_t gen_word = tid == 0 ? ld_relaxed_gpu_u64(a.part + kPartStrideWords * blockIdx.x) : 0ull;
+    GroupTab gt;
+    gt.off = s_off;
+    gt.blk = s_blk;
+    gt.G = a.groups;
+    Ring r;
+    r.base = reinterpret_cast<char*>(dsm) + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u);   // 128-byte swizzle: 1 KB aligned
+    r.bar = &sbar[warp * kStage];
+    r.warp = warp;
+    r.phase = 0;
+    r.box_bytes = box_bytes;
+    const LaneC lc = make_lanec(lane);
+    const uint64_t pol_keep = l2_policy_evict_normal();   // read again in pass 2
+    const uint64_t pol_last = l2_policy_evict_first();    // stays on chip: not read again
+    SrcCursor<GROUPED> sp, lp;                            // pass 1: next task to copy; next task to land
+    int nt = 0;   // this warp's first nt tasks stay in tensor memory
+    // The first kStage copies of pass 1 (one commit group each, empty past n).
+    // One tensor: issued before the set-up below, which they overlap.
+    auto first_copies = [&]() {
+        nt = max(0, min(a.tm_tasks, n - kStage));
+        sp.init(a, gt, tw);
+        lp.init(a, gt, tw);
+#pragma unroll
+        for (int i = 0; i < kStage; ++i) {
+            if (i < n) {
+                stage_cp<GROUPED>(a, r, i, sp, lc, (i < nt || i >= n - kStage) ? pol_last : pol_keep);
+                sp.next(a, gt);
+            }
+            cp_async_commit();
+        }
+    };
+    if constexpr (!GROUPED) first_copies();
     if (tid < kStage * kFWarps) mbar_init(&sbar[tid], 1);
     // Tensor memory (all 512 columns: 64 per warp, in the warp's own lane
     // quarter) when some warp has more tasks than shared-memory slots.
@@ -1018,10 +1192,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
         tmem_alloc(&s_tmem, 512);
         tmem_relinquish();
     }
-    GroupTab gt;
-    gt.off = s_off;
-    gt.blk = s_blk;
-    gt.G = a.groups;
     if constexpr (GROUPED) {
         // offsets and the exclusive prefix of the groups' 128-row block counts
         // (a.groups <= kMaxFusedGroups = kFThreads)
@@ -1055,23 +1225,20 @@ __global__ void __launch_bounds__(kFThreads, 1)
             s_smooth[seg * kTaskVals + pu * 4 + (i & 3)] = i < a.k ? a.smooth[i] : 0.0f;
         }
     }
+    if (GROUPED && tid == 0) s_gen = (uint32_t)(gen_word >> 32) + 1u;   // grouped: every warp folds with it
     fence_mbar_init();
     __syncthreads();
-    const uint32_t gen = s_gen;
+    // one more than this CTA's last call's generation (the same in every CTA);
+    // one tensor: only thread 0 uses it
+    const uint32_t gen = GROUPED ? s_gen : (uint32_t)(gen_word >> 32) + 1u;
     if constexpr (GROUPED) {
         // the exact task count: tasks past it belong to no group
         const int real = 128 * s_blk[a.groups] * a.nseg;
         n = max(0, min(tw + n, real) - tw);
+        first_copies();
     }
-    Ring r;
-    r.base = reinterpret_cast<char*>(dsm) + ((1024u - (smem_u32(dsm) & 1023u)) & 1023u);   // 128-byte swizzle: 1 KB aligned
-    r.bar = &sbar[warp * kStage];
-    r.warp = warp;
-    r.phase = 0;
-    r.box_bytes = box_bytes;
     if (lane == 0) prefetch_tmap(&tmap);
-    // this warp's first nt tasks stay in tensor memory, at columns tcol + 16 j
-    const int nt = max(0, min(a.tm_tasks, n - kStage));
+    // the first nt tasks stay in tensor memory, at columns tcol + 16 j
     uint32_t tcol = 0;
     if (a.tm_tasks > 0) {
         tc_fence_after();
@@ -1080,24 +1247,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
 
     // ---- pass 1: amax through the slot ring; the first nt tasks are parked in
     // tensor memory, the last kStage stay in their slots
-    const LaneC lc = make_lanec(lane);
     uint32_t acc = 0;      // packed BF16 running max |x|
     float accf = 0.0f;     // pre-scaled form: running max |x s|
     {
-        const uint64_t pol_keep = l2_policy_evict_normal();   // read again in pass 2
-        const uint64_t pol_last = l2_policy_evict_first();    // stays on chip: not read again
-        SrcCursor<GROUPED> sp, lp;                            // next task to copy; next task to land
-        sp.init(a, gt, tw);
-        lp.init(a, gt, tw);
         int cur = lp.m.e;                                     // grouped: the group acc belongs to
-#pragma unroll
-        for (int i = 0; i < kStage; ++i) {
-            if (i < n) {
-                stage_cp<GROUPED>(a, r, i, sp, lc, (i < nt || i >= n - kStage) ? pol_last : pol_keep);
-                sp.next(a, gt);
-            }
-            cp_async_commit();
-        }
         // One commit group per step (empty once nothing is left): with at most
         // kStage - 1 groups pending, the oldest copy has landed.
         int s = 0;
@@ -1127,9 +1280,21 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 for (int q = 0; q < 4; ++q)
                     accf = fmaxf(accf, absmax8_smooth(u[q], smooth_unit(sb2, lane, 2 * q),
                                                       smooth_unit(sb2, lane, 2 * q + 1)));
-            } else {
+            } else if constexpr (GROUPED) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) acc = bmax_abs(acc, absmax8_packed(u[q]));
+            } else {
+                // block maxima (blocks 2 lane, 2 lane + 1), kept for the tasks
+                // that stay on chip, then folded into the running maximum
+                const uint32_t m0 = bmax_abs(absmax8_packed(u[0]), absmax8_packed(u[1]));
+                const uint32_t m1 = bmax_abs(absmax8_packed(u[2]), absmax8_packed(u[3]));
+                acc = bmax_abs(acc, bmax_abs(m0, m1));
+                const int res0 = n - min(n, kStage);   // first slot task
+                if (i < nt || i >= res0) {
+                    const int j = i < nt ? i : kTmTasks + (i - res0);
+                    s_bm[(j * kFWarps + warp) * 32 + lane] =
+                        bmax_abs(__byte_perm(m0, m1, 0x5410), __byte_perm(m0, m1, 0x7632));
+                }
             }
             if (i < nt) {
                 const uint32_t w[16] = {u[0].x, u[0].y, u[0].z, u[0].w, u[1].x, u[1].y, u[1].z, u[1].w,
@@ -1192,9 +1357,18 @@ __global__ void __launch_bounds__(kFThreads, 1)
             pq.q = make_groupq(s_amax);
             if (blockIdx.x == 0 && tid == 0) a.gscale[0] = pq.q.g;
             fill_rtab(rtab, pq.q.g, tid);
+            if (kPlain && !pq.q.tiny) fill_qtab(s_qtab, pq.q.c.k6, tid - 128);
             __syncthreads();
         }
-        fused_pass2<GROUPED, SMOOTH>(&tmap, a, gt, r, rtab, pq, gen, tw, n, nt, tcol, lc, s_smooth);
+        const OnChip oc{s_bm + warp * 32 + lane, s_qtab};
+        bool done = false;
+        if constexpr (kPlain) {
+            if (!pq.q.tiny && n - min(n, kStage) - nt == 0) {   // warp-uniform: every task on chip
+                plain_pass2(a, r, lc, tw, n, nt, tcol, oc.bm, rtab, s_qtab);
+                done = true;
+            }
+        }
+        if (!done) fused_pass2<GROUPED, SMOOTH>(&tmap, a, gt, r, rtab, pq, gen, tw, n, nt, tcol, lc, s_smooth, oc);
     }
     if (a.tm_tasks > 0) {   // every warp's tensor-memory reads are done (tcgen05.wait::ld after each)
         tc_fence_before();

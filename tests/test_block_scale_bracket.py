@@ -54,3 +54,44 @@ def test_bracket_rule_subnormal_global_scale_always_divides():
     # amax at the bottom of the BF16 range: 6 g is subnormal in FP32
     n, _ = _check_amax(0x0001)
     assert n == 2
+
+
+# ---- the quotient table of the one-tensor kernel ---------------------------------------
+#
+# For a BF16 block amax b = m_b 2^(e_b - 127) (m_b = 1 + i/128) and a normal
+# 6g = m_k 2^(e_k - 127), the kernel takes the bits of RN(b / 6g) as
+# qtab[i] + (e_b << 23), qtab[i] = bits(RN((1 + i/128) / m_k)) - (e_k << 23),
+# clamped at 0 as a signed integer.  Restated here in float32 numpy and checked
+# against e4m3 of the correctly rounded quotient for every BF16 block amax up
+# to the tensor amax (zero, BF16 subnormals and quotients below 2^-126
+# included), at tensor amaxes whose g is at least 2^-64.
+
+def _table_rule(b_bits, k6):
+    kb = np.array([k6], np.float32).view(np.uint32)[0]
+    mk = np.array([(kb & 0x807FFFFF) | (127 << 23)], np.uint32).view(np.float32)[0]
+    num = ((np.uint32(127) << 23) | (np.arange(128, dtype=np.uint32) << 16)).view(np.float32)
+    q = (num / mk).astype(np.float32)                                  # correctly rounded
+    qtab = q.view(np.uint32).astype(np.int64) - int(kb & 0x7F800000)
+    f = (np.asarray(b_bits, np.uint32) << 16)                           # FP32 bits of the BF16 amax
+    bits = qtab[(f >> 16) & 0x7F] + (f & 0x7F800000).astype(np.int64)
+    bits = np.maximum(bits, 0).astype(np.uint32)
+    return O.e4m3_encode_array(bits.view(np.float32))
+
+
+def test_quotient_table_matches_correctly_rounded_quotient():
+    rng = np.random.default_rng(2025)
+    amaxes = list(rng.integers(0x2600, 0x7F80, size=120)) + [0x2600, 0x3F80, 0x40C0, 0x4340, 0x43E0, 0x7F7F,
+                                                             0x3C00, 0x3B4D, 0x40AF, 0x2580]
+    total = 0
+    for ab in amaxes:
+        amax = _bf16([ab])[0]
+        g = F32(amax / F32(2688.0))
+        assert g >= 2.0 ** -64
+        k6 = F32(F32(6.0) * g)
+        bits = np.arange(0, int(ab) + 1, dtype=np.uint32)              # every block amax <= amax
+        exact = O.e4m3_encode_array((_bf16(bits) / k6).astype(np.float32))
+        got = _table_rule(bits, k6)
+        bad = np.nonzero(got != exact)[0]
+        assert bad.size == 0, f"amax {amax:a}: table rule differs at b={_bf16(bits[bad[:1]])[0]:a}"
+        total += bits.size
+    assert total > 1_000_000
