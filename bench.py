@@ -733,9 +733,17 @@ def measure_decode(nv, torch, dev, cs, sampler, peaks, with_cpu, ms=(1, 8, 32, 6
             j = i % wl.R
             nv.gemm_w4a16(wl.a[j], wl.w[j], out=wl.c[j])
         t16, clk16 = timed_loop(torch, cs, w16, wl.R, KERNEL_ITERS, sampler)
+
+        def fused(i):
+            j = i % wl.R
+            nv.quantize_gemm(wl.a[j], wl.w[j], out=wl.c[j], qa=wl.qa[j])
+        tf, clkf = timed_loop(torch, cs, fused, wl.R, n, sampler)
         gbytes = wl.wbytes + wl.abytes + wl.cbytes
         g_gbs = gbytes / g_s / 1e9
-        r = {"step_ms": step_s * 1e3, "steps_timed": n, "quantize_ms": q_s * 1e3, "gemm_ms": g_s * 1e3,
+        r = {"step_ms": step_s * 1e3, "steps_timed": n,
+             "fused_step_ms": tf * 1e3, "fused_step_weight_stream_gbs": wl.wbytes / tf / 1e9,
+             "fused_step_weight_stream_frac_hbm": wl.wbytes / tf / 1e9 / hbm, "fused_step_clocks": clkf,
+             "quantize_ms": q_s * 1e3, "gemm_ms": g_s * 1e3,
              "gemm_tflops": wl.flops / g_s / 1e12, "gemm_frac_fp4": wl.flops / g_s / 1e12 / fp4_peak,
              "weight_stream_gbs": wl.wbytes / g_s / 1e9, "weight_stream_frac_hbm": wl.wbytes / g_s / 1e9 / hbm,
              "step_weight_stream_gbs": wl.wbytes / step_s / 1e9,
@@ -748,7 +756,7 @@ def measure_decode(nv, torch, dev, cs, sampler, peaks, with_cpu, ms=(1, 8, 32, 6
         if with_cpu:
             r["cpu_baseline"] = cpu_baseline_decode(wl.a_host, wh, wl.n, wl.k)
         out["per_m"][str(m)] = r
-        del wl, w16
+        del wl, w16, fused
         torch.cuda.empty_cache()
     return out
 

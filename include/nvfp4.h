@@ -98,7 +98,7 @@ size_t nvfp4_grouped_scale_bytes(int64_t total_rows, int num_groups, int64_t k);
 
 /* Workspace bytes an operation needs (operations below); 0 if none. */
 enum { NVFP4_OP_QUANTIZE_ACT = 0, NVFP4_OP_QUANTIZE_WEIGHT_2D = 1, NVFP4_OP_GEMM = 2,
-       NVFP4_OP_GROUPED_GEMM = 3, NVFP4_OP_GEMM_EMIT_SCALE = 4 };
+       NVFP4_OP_GROUPED_GEMM = 3, NVFP4_OP_GEMM_EMIT_SCALE = 4, NVFP4_OP_QUANTIZE_GEMM = 5 };
 size_t nvfp4_workspace_bytes(int op, int64_t rows, int64_t n, int64_t k, int num_groups);
 
 /* Zero a workspace before its first use (cudaMemsetAsync on stream). */
@@ -241,6 +241,32 @@ nvfp4_status_t nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const
                           const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global,
                           void* c, int64_t ldc, int64_t m, int64_t n, int64_t k,
                           void* workspace, void* stream);
+
+/* nvfp4_quantize_gemm -- one W4A4 layer step: dynamic quantization of the
+ * BF16 activations x (exactly as nvfp4_quantize_act, one tensor), then
+ * C = A_q * B^T as nvfp4_gemm ("NVFP4 Dynamic Quantization in Practice",
+ * W4A4: activations quantized on the fly against pre-quantized weights).
+ * Results are bit-identical to calling the two entry points in turn.
+ * For decode-sized activations (m <= 64) the weights' stream starts while the
+ * activations are still being quantized: decode is bound by reading the
+ * weights ("W4A8 vs NVFP4 quantization on GPUs", "Batch size can change the
+ * winner"), and this call knows that none of its own kernels writes them.
+ * So b_codes and b_scales must not be written by the kernel that runs just
+ * before this call on the stream (as for any kernel input, the caller orders
+ * their producer before the call).
+ *   x: device BF16 [m, k], row stride ldx (ldx >= k, ldx % 8 == 0); k % 64 == 0.
+ *   b_codes, b_scales, b_global, n, c, ldc: as nvfp4_gemm.
+ *   a_codes, a_scales, a_global: receive the quantized activations, as the
+ *   outputs of nvfp4_quantize_act (codes [m, k/2], nvfp4_scale_bytes(m, k)
+ *   scale bytes, one FP32 global scale).
+ *   workspace: nvfp4_workspace_bytes(NVFP4_OP_QUANTIZE_GEMM, m, n, k, 0)
+ *   bytes, 16-byte aligned, zeroed before first use; the quantizer's part
+ *   first, then the GEMM's.  Calls on one workspace must not overlap.
+ *   m == 0 returns NVFP4_OK without launching anything. */
+nvfp4_status_t nvfp4_quantize_gemm(const void* x, int64_t m, int64_t k, int64_t ldx, const uint8_t* b_codes,
+                                   const uint8_t* b_scales, const float* b_global, int64_t n, void* c, int64_t ldc,
+                                   uint8_t* a_codes, uint8_t* a_scales, float* a_global, void* workspace,
+                                   void* stream);
 
 /* nvfp4_gemm_emit_scale -- nvfp4_gemm that also takes the amax of its BF16
  * output in the epilogue and writes the global scale the next layer's

@@ -29,14 +29,14 @@ __all__ = [
     "quantize_act", "quantize_weight_2d", "gemm", "grouped_gemm", "check_device_error",
     "gemm_emit_scale", "quantize_act_scaled", "quantize_act_smooth",
     "mxfp4_scale_bytes", "mxfp4_quantize_act", "mxfp4_gemm", "MXFP4Tensor", "quantize_mx", "gemm_mx",
-    "w4a16_gemm", "gemm_w4a16",
+    "w4a16_gemm", "gemm_w4a16", "nvfp4_quantize_gemm", "quantize_gemm", "OP_QUANTIZE_GEMM",
     "OP_QUANTIZE_ACT", "OP_QUANTIZE_WEIGHT_2D", "OP_GEMM", "OP_GROUPED_GEMM", "OP_GEMM_EMIT_SCALE",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libnvfp4.so")
 
-OP_QUANTIZE_ACT, OP_QUANTIZE_WEIGHT_2D, OP_GEMM, OP_GROUPED_GEMM, OP_GEMM_EMIT_SCALE = 0, 1, 2, 3, 4
+OP_QUANTIZE_ACT, OP_QUANTIZE_WEIGHT_2D, OP_GEMM, OP_GROUPED_GEMM, OP_GEMM_EMIT_SCALE, OP_QUANTIZE_GEMM = 0, 1, 2, 3, 4, 5
 STATUS = {0: "OK", 1: "INVALID_ARGUMENT", 2: "UNSUPPORTED_SHAPE", 3: "MISALIGNED", 4: "CUDA",
           5: "TIMEOUT", 6: "NO_DEVICE"}
 
@@ -67,6 +67,7 @@ _SIGNATURES = {
     "nvfp4_quantize_act_scaled": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]),
     "nvfp4_quantize_act_smooth": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp]),
     "nvfp4_grouped_gemm": (_i32, [_vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp]),
+    "nvfp4_quantize_gemm": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _vp]),
     "mxfp4_scale_bytes": (_sz, [_i64, _i64]),
     "mxfp4_quantize_act": (_i32, [_vp, _i64, _i64, _i64, _vp, _vp, _vp]),
     "mxfp4_gemm": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _vp]),
@@ -186,6 +187,12 @@ def nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_code
                        total_rows, workspace=None, stream=0) -> int:
     return lib().nvfp4_grouped_gemm(a_codes, a_scales, a_global, offsets, num_experts, b_codes, b_scales,
                                     b_global, c, n, k, total_rows, workspace, stream)
+
+
+def nvfp4_quantize_gemm(x, m, k, ldx, b_codes, b_scales, b_global, n, c, ldc, a_codes, a_scales, a_global,
+                        workspace, stream=0) -> int:
+    return lib().nvfp4_quantize_gemm(x, m, k, ldx, b_codes, b_scales, b_global, n, c, ldc, a_codes, a_scales,
+                                     a_global, workspace, stream)
 
 
 def mxfp4_scale_bytes(rows: int, k: int) -> int:
@@ -517,6 +524,37 @@ def _reset_workspaces(device_index: int) -> None:
         for ws in mine:
             ws.zero_()
         torch.cuda.synchronize()
+
+
+def quantize_gemm(x, b: NVFP4Tensor, out=None, qa: Optional[NVFP4Tensor] = None):
+    """One W4A4 step: quantize the BF16 [m, k] activations x dynamically and
+    multiply by the NVFP4 weights b; returns (C, the quantized activations).
+    For m <= 64 the weights start streaming while x is being quantized."""
+    import torch
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise TypeError("x must be a 2-D bfloat16 CUDA tensor")
+    if x.stride(1) != 1:
+        raise ValueError("x must have unit stride along k")
+    m, k = x.shape
+    if k != b.k:
+        raise ValueError("k mismatch")
+    dev = x.device
+    c = out if out is not None else torch.empty((m, b.rows), dtype=torch.bfloat16, device=dev)
+    if qa is None:
+        qa = NVFP4Tensor(torch.empty((m, k // 2), dtype=torch.uint8, device=dev),
+                         torch.empty(nvfp4_scale_bytes(m, k), dtype=torch.uint8, device=dev),
+                         torch.empty(1, dtype=torch.float32, device=dev), m, k)
+    nbytes = nvfp4_workspace_bytes(OP_QUANTIZE_GEMM, m, b.rows, k, 0)
+    key = (dev.index, OP_QUANTIZE_GEMM, 0, torch.cuda.current_stream(dev).cuda_stream)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+        _ws_cache[key] = ws
+    st = nvfp4_quantize_gemm(_ptr(x), m, k, x.stride(0), _ptr(b.codes), _ptr(b.scales), _ptr(b.global_scale),
+                             b.rows, _ptr(c), c.stride(0), _ptr(qa.codes), _ptr(qa.scales), _ptr(qa.global_scale),
+                             _ptr(ws), _stream_ptr(torch, dev))
+    _check(st, "nvfp4_quantize_gemm")
+    return c, qa
 
 
 def check_device_error(stream: int = 0) -> None:

@@ -124,6 +124,7 @@ extern "C" size_t nvfp4_workspace_bytes(int op, int64_t rows, int64_t n, int64_t
         case NVFP4_OP_GEMM: return gemm_workspace_bytes(rows, n, k);
         case NVFP4_OP_GEMM_EMIT_SCALE: return (size_t)kEmitScaleWsBytes + gemm_workspace_bytes(rows, n, k);
         case NVFP4_OP_GROUPED_GEMM: return 0;
+        case NVFP4_OP_QUANTIZE_GEMM: return (size_t)quant_ws_bytes(1) + gemm_workspace_bytes(rows, n, k);
     }
     return 0;
 }

@@ -93,6 +93,11 @@ struct GemmArgs {
     // optional: the amax of the BF16 output, as the next quantizer's global scale
     uint32_t* c_amax;          // [0] running max |C| (BF16 bits), [1] CTAs done; both 0 between calls
     float* c_gscale;           // receives amax(C) / 2688 (1 when amax is 0)
+    // single-SM kernel, plain form: B (codes and scales) was not written by the
+    // kernel this one depends on, so the producer may load the first stages'
+    // B tiles before griddepcontrol.wait (the weight stream starts while the
+    // activations are still being quantized)
+    int b_early;
 };
 
 // The largest |value| of packed BF16 pairs, as a 16-bit pattern.
@@ -264,6 +269,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_tmap(&tmB);
         prefetch_tmap(&tmC);
     }
+    // b_early: thread 0 (the producer) sends the B half -- codes and scales --
+    // of its first tile's first `pre` stages (the ring is fresh: stage kt)
+    // before any wait, so that the weights stream while the kernel this one
+    // depends on is still running; the A half follows in the producer loop.
+    const bool b_early = !GROUPED && p.b_early != 0;
+    int pre = 0;
+    auto b_half = [&](const TileInfo& ti, int kt, uint64_t* bar, uint8_t* sB, uint8_t* sSFB, uint32_t nch, int nsfb) {
+        const uint8_t* sfb_src =
+            p.sfb + (int64_t)ti.group * p.sfb_group_stride + (int64_t)(ti.b_col0 / 128) * p.sfb_rb_stride;
+        tma_load_2d(sB, &tmB, bar, kt * 128, ti.b_row0);
+        for (int rb = 0; rb < nsfb; ++rb)
+            bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * SF_KT, nch * 512u,
+                      bar);
+    };
+    const bool first_tile = !GROUPED && threadIdx.x == 0 && (int)blockIdx.x < p.tiles_m * p.tiles_n;
+    if (b_early && first_tile) {
+        const TileInfo ti = tile_info<BN, GROUPED>(p, tail, blockIdx.x);
+        const int nsfb = min(NSFB, p.sfb_rb_per_group - ti.b_col0 / 128);
+        pre = min(STAGES, p.num_kt);
+        for (int kt = 0; kt < pre; ++kt) {
+            const int nat = min(4, p.num_ks - kt * 4);
+            const uint32_t nch = MX ? (uint32_t)(nat + 1) / 2 : (uint32_t)nat;
+            uint8_t* sA = smem + kt * C::STAGE_BYTES;
+            uint8_t* sSFA = sA + C::A_BYTES + C::B_BYTES;
+            uint64_t* bar = &tail->full[kt];
+            mbar_arrive_expect_tx(bar, C::A_BYTES + C::B_BYTES + nch * 512u * (1u + (uint32_t)nsfb));
+            b_half(ti, kt, bar, sA + C::A_BYTES, sSFA + C::SFA_BYTES, nch, nsfb);
+        }
+    }
     if (warp == 1) {
         tmem_alloc(&tail->tmem_base, kTmemCols);
         tmem_relinquish();
@@ -326,8 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
                 const TileInfo ti = tile_info<BN, GROUPED>(p, tail, t);
                 const uint8_t* sfa_src = p.sfa + (int64_t)ti.sfa_rb * p.sfa_rb_stride;
-                const uint8_t* sfb_src = p.sfb + (int64_t)ti.group * p.sfb_group_stride +
-                                         (int64_t)(ti.b_col0 / 128) * p.sfb_rb_stride;
                 const int nsfb = min(NSFB, p.sfb_rb_per_group - ti.b_col0 / 128);
                 for (int kt = 0; kt < p.num_kt; ++kt) {
                     if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
@@ -341,13 +373,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint8_t* sSFA = sB + C::B_BYTES;
                     uint8_t* sSFB = sSFA + C::SFA_BYTES;
                     uint64_t* bar = &tail->full[stage];
-                    mbar_arrive_expect_tx(bar, C::A_BYTES + C::B_BYTES + nch * 512u * (1u + (uint32_t)nsfb));
+                    const bool b_done = t == (int)blockIdx.x && kt < pre;   // B half already issued
+                    if (!b_done) {
+                        mbar_arrive_expect_tx(bar, C::A_BYTES + C::B_BYTES + nch * 512u * (1u + (uint32_t)nsfb));
+                        b_half(ti, kt, bar, sB, sSFB, nch, nsfb);
+                    }
                     tma_load_2d(sA, &tmA, bar, kt * 128, ti.a_row0);
-                    tma_load_2d(sB, &tmB, bar, kt * 128, ti.b_row0);
                     bulk_load(sSFA, sfa_src + (int64_t)kt * SF_KT, nch * 512u, bar);
-                    for (int rb = 0; rb < nsfb; ++rb)
-                        bulk_load(sSFB + rb * 2048, sfb_src + (int64_t)rb * p.sfb_rb_stride + (int64_t)kt * SF_KT,
-                                  nch * 512u, bar);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
@@ -1420,7 +1452,7 @@ __global__ void set_one_kernel(float* g) { g[0] = 1.0f; }
 nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                          const uint8_t* b_codes, const uint8_t* b_scales, const float* b_global, void* c, int64_t ldc,
                          int64_t m, int64_t n, int64_t k, void* workspace, uint32_t* c_amax, float* c_gscale,
-                         void* stream, bool mx = false) {
+                         void* stream, bool mx = false, bool b_early = false) {
     if (m < 0 || n <= 0 || k <= 0 || ldc < n) return NVFP4_ERR_INVALID_ARGUMENT;
     if (k % 64 != 0 || m >= ((int64_t)1 << 31) || n >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
         return NVFP4_ERR_UNSUPPORTED_SHAPE;
@@ -1476,6 +1508,7 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
         p.rows_b = (int)n;
         p.tiles_m = 1;
         p.tiles_n = (int)((n + CfgDecW::BN - 1) / CfgDecW::BN);
+        p.b_early = b_early ? 1 : 0;
         const int grid = (int)std::min<int64_t>((int64_t)p.tiles_n, sms);
         if (mx) return launch<CfgDecW, false, false, true>(ta, tb, tc, p, grid, s);
         return c_amax ? launch<CfgDecW, false, true>(ta, tb, tc, p, grid, s) : launch<CfgDecW, false>(ta, tb, tc, p, grid, s);
@@ -1622,4 +1655,42 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     const int64_t max_tiles = (total_rows / 128 + num_experts) * (int64_t)p.tiles_n;
     const int grid = (int)std::min<int64_t>(max_tiles, sms);
     return launch<CfgWide, true>(ta, tb, tc, p, grid, s);
+}
+
+// Dynamic activation quantization followed by the GEMM, in one call.  For
+// decode-sized activations (m <= 64) the quantizer runs as the two-kernel
+// form, whose small CTAs leave room on every SM, and the GEMM is launched as
+// its programmatic dependent with b_early: its CTAs start streaming the
+// weights (which no kernel of this call writes) while the activations are
+// still being quantized, and wait only before reading them.  Larger m: the
+// one-launch quantizer, then the GEMM.
+extern "C" nvfp4_status_t nvfp4_quantize_gemm(const void* x, int64_t m, int64_t k, int64_t ldx, const uint8_t* b_codes,
+                                              const uint8_t* b_scales, const float* b_global, int64_t n, void* c,
+                                              int64_t ldc, uint8_t* a_codes, uint8_t* a_scales, float* a_global,
+                                              void* workspace, void* stream) {
+    if (m < 0 || n <= 0 || k <= 0 || ldx < k || ldc < n) return NVFP4_ERR_INVALID_ARGUMENT;
+    if (m == 0) return NVFP4_OK;
+    if (!x || !b_codes || !b_scales || !b_global || !c || !a_codes || !a_scales || !a_global || !workspace)
+        return NVFP4_ERR_INVALID_ARGUMENT;
+    if (k % 64 != 0 || m >= ((int64_t)1 << 31) || n >= ((int64_t)1 << 31) || k >= ((int64_t)1 << 31))
+        return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    if (!ptr_ok(x) || !ptr_ok(workspace) || ldx % 8 != 0) return NVFP4_ERR_MISALIGNED;
+    uint8_t* gemm_ws = reinterpret_cast<uint8_t*>(workspace) + quant_ws_bytes(1);
+    if (m > 64) {
+        const nvfp4_status_t st =
+            nvfp4_quantize_act(x, m, k, ldx, nullptr, 0, a_codes, a_scales, a_global, workspace, stream);
+        if (st != NVFP4_OK) return st;
+        return nvfp4_gemm(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k,
+                          gemm_workspace_bytes(m, n, k) ? gemm_ws : nullptr, stream);
+    }
+    // argument checks of both halves before anything is launched
+    if (!ptr_ok(a_codes) || !ptr_ok(a_scales) || !ptr_ok(b_codes) || !ptr_ok(b_scales) || !ptr_ok(c) ||
+        (reinterpret_cast<uintptr_t>(a_global) & 3u) || (reinterpret_cast<uintptr_t>(b_global) & 3u) || ldc % 8 != 0)
+        return NVFP4_ERR_MISALIGNED;
+    if (num_sms() <= 0) return NVFP4_ERR_NO_DEVICE;
+    const nvfp4_status_t st = run_two_kernel(reinterpret_cast<const uint16_t*>(x), m, k, ldx, nullptr, 1, a_codes,
+                                             a_scales, a_global, workspace, reinterpret_cast<cudaStream_t>(stream));
+    if (st != NVFP4_OK) return st;
+    return gemm_impl(a_codes, a_scales, a_global, b_codes, b_scales, b_global, c, ldc, m, n, k, nullptr, nullptr,
+                     nullptr, stream, false, true);
 }

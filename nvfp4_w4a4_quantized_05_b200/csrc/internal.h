@@ -43,6 +43,14 @@ inline bool smem_attr_on_device(const void* kernel, int bytes, std::atomic<unsig
 // Current limit of the bounded waits, in ns.
 uint64_t wait_limit_ns();
 
+// Dynamic 1D quantization of one tensor (offsets == nullptr, groups == 1) or of
+// row groups by the two-kernel form: the amax kernel, then the quantize kernel
+// as its programmatic dependent.  Arguments as nvfp4_quantize_act, already
+// checked by the caller.
+nvfp4_status_t run_two_kernel(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, const int32_t* group_offsets,
+                              int groups, uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
+                              cudaStream_t s);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 constexpr int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }

@@ -343,7 +343,13 @@ struct AmaxArgs {
 
 constexpr int kAmaxUnroll = 8;
 
+// The kernels below let the next kernel in the stream launch as soon as all
+// their CTAs run (griddepcontrol.launch_dependents at the start): a dependent
+// kernel's griddepcontrol.wait still waits for this grid's completion and
+// writes, so it may only do independent work earlier (prefetch its own
+// inputs that this kernel does not write).
 __global__ void __launch_bounds__(kThreads, 4) amax_kernel(AmaxArgs a) {
+    pdl_launch_dependents();
     const int e = blockIdx.y;
     int r0, r1;
     a.groups.range(e, r0, r1);
@@ -398,7 +404,6 @@ __global__ void __launch_bounds__(kThreads, 4) amax_kernel(AmaxArgs a) {
         if (a.pad_rows) write_pad_rows(a.groups, a.num_groups, a.pad_rows);
         if (threadIdx.x == 0) a.ws[0] = 0;
     }
-    pdl_launch_dependents();
 }
 
 // ---- kernel 2: 1D 16-element blocks (one tensor or row groups) ---------------------
@@ -445,6 +450,7 @@ __device__ __forceinline__ void load_block16(const Quant1dArgs& a, int r0, int n
 // MX: the MXFP4 task (one tensor, no global scale; gscale unused).
 template <bool MX = false>
 __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
+    pdl_launch_dependents();
     const int e = blockIdx.y;
     int r0, r1;
     a.groups.range(e, r0, r1);
@@ -505,7 +511,6 @@ __global__ void __launch_bounds__(kThreads, 4) quant1d_kernel(Quant1dArgs a) {
             load_block16(a, r0, nrows, tp[u], lane, pol, v[u][0], v[u][1]);
         }
     }
-    pdl_launch_dependents();
 }
 
 // ---- one launch for one tensor: amax, grid barrier, quantize ---------------------
@@ -1348,6 +1353,10 @@ __global__ void __launch_bounds__(kFThreads, 1)
     }
     __syncthreads();
     const bool ok = s_ok != 0;
+    // The next kernel in the stream may launch now: its CTAs cannot share an
+    // SM with these (shared memory), so they start as each SM frees, and its
+    // wait still covers this grid's completion and writes.
+    pdl_launch_dependents();
     if (ok) {
         Pass2Q<GROUPED> pq;
         if constexpr (GROUPED) {
@@ -1375,7 +1384,6 @@ __global__ void __launch_bounds__(kFThreads, 1)
         __syncthreads();
         if (warp == 0) tmem_dealloc(s_tmem, 512);
     }
-    pdl_launch_dependents();
 }
 
 // ---- kernel 2 (weights): 16 x 16 blocks -------------------------------------------
@@ -1390,6 +1398,7 @@ struct Quant2dArgs {
 };
 
 __global__ void __launch_bounds__(kThreads) quant2d_kernel(Quant2dArgs a) {
+    pdl_launch_dependents();
     pdl_wait();
     const float g = a.gscale[0];
     const float k6 = __fmul_rn(6.0f, g);
@@ -1437,7 +1446,6 @@ __global__ void __launch_bounds__(kThreads) quant2d_kernel(Quant2dArgs a) {
                 *reinterpret_cast<uint32_t*>(a.scales + sf_tile_offset(tr * 16 + i, scol, a.scale_cols)) = word;
         }
     }
-    pdl_launch_dependents();
 }
 
 // ---- format probe -------------------------------------------------------------------
@@ -1599,6 +1607,39 @@ nvfp4_status_t run_amax(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, 
 }
 
 }  // namespace
+
+// The two-kernel form: the amax kernel, then the quantize kernel launched as
+// its programmatic dependent (its first loads of x precede its wait).  Small
+// CTAs (256 threads): a dependent GEMM's CTAs fit beside them on every SM.
+nvfp4_status_t run_two_kernel(const uint16_t* xb, int64_t rows, int64_t k, int64_t ld, const int32_t* group_offsets,
+                              int groups, uint8_t* codes, uint8_t* scales, float* global_scale, void* workspace,
+                              cudaStream_t s) {
+    nvfp4_status_t st = run_amax(xb, rows, k, ld, group_offsets, groups, workspace, global_scale, s);
+    if (st != NVFP4_OK) return st;
+
+    Quant1dArgs q;
+    q.x = xb;
+    q.ld = ld;
+    q.k = (int)k;
+    q.nseg = (int)((k + 511) / 512);
+    q.scale_cols = (int)(round_up(k / 16, 4));
+    q.groups.offsets = group_offsets;
+    q.groups.rows = (int)rows;
+    q.pad_rows = group_offsets ? reinterpret_cast<const int32_t*>(reinterpret_cast<uint8_t*>(workspace) +
+                                                                 quant_ws_pad_off(groups))
+                               : nullptr;
+    q.gscale = global_scale;
+    q.codes = codes;
+    q.scales = scales;
+    const int64_t tasks = (round_up(rows, 128) + (group_offsets ? 127 * (int64_t)groups : 0)) * q.nseg;
+    const int64_t per_group = (tasks + groups - 1) / groups;
+    const int qx = clamp_grid((per_group + kWarps * kQuantUnroll - 1) / (kWarps * kQuantUnroll),
+                              (int64_t)num_sms() * 4 / groups);
+    void* args[] = {&q};
+    return cuda_status(launch_pdl(reinterpret_cast<const void*>(&quant1d_kernel<false>), dim3(qx, groups), dim3(kThreads),
+                                  args, s));
+}
+
 }  // namespace nvfp4
 
 using namespace nvfp4;
@@ -1630,30 +1671,7 @@ extern "C" nvfp4_status_t nvfp4_quantize_act(const void* x, int64_t rows, int64_
             run_fused(xb, rows, k, ld, group_offsets, groups, codes, scales, global_scale, workspace, s);
         if (fs != NVFP4_ERR_UNSUPPORTED_SHAPE) return fs;
     }
-    nvfp4_status_t st = run_amax(xb, rows, k, ld, group_offsets, groups, workspace, global_scale, s);
-    if (st != NVFP4_OK) return st;
-
-    Quant1dArgs q;
-    q.x = xb;
-    q.ld = ld;
-    q.k = (int)k;
-    q.nseg = (int)((k + 511) / 512);
-    q.scale_cols = (int)(round_up(k / 16, 4));
-    q.groups.offsets = group_offsets;
-    q.groups.rows = (int)rows;
-    q.pad_rows = group_offsets ? reinterpret_cast<const int32_t*>(reinterpret_cast<uint8_t*>(workspace) +
-                                                                 quant_ws_pad_off(groups))
-                               : nullptr;
-    q.gscale = global_scale;
-    q.codes = codes;
-    q.scales = scales;
-    const int64_t tasks = (round_up(rows, 128) + (group_offsets ? 127 * (int64_t)groups : 0)) * q.nseg;
-    const int64_t per_group = (tasks + groups - 1) / groups;
-    const int qx = clamp_grid((per_group + kWarps * kQuantUnroll - 1) / (kWarps * kQuantUnroll),
-                              (int64_t)num_sms() * 4 / groups);
-    void* args[] = {&q};
-    return cuda_status(launch_pdl(reinterpret_cast<const void*>(&quant1d_kernel<false>), dim3(qx, groups), dim3(kThreads),
-                                  args, s));
+    return run_two_kernel(xb, rows, k, ld, group_offsets, groups, codes, scales, global_scale, workspace, s);
 }
 
 extern "C" nvfp4_status_t nvfp4_quantize_weight_2d(const void* w, int64_t n, int64_t k, int64_t ld, uint8_t* codes,

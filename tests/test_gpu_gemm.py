@@ -259,3 +259,30 @@ def test_scale_layout_read_by_library_block_scaled_gemm(m, n, k):
     torch.cuda.synchronize()
     ref, absref = gemm_refs(O.dequantize(ac, asf, 1.0), O.dequantize(wc, wsf, 1.0))
     assert_gemm_close(to_host_f64(c), ref, absref, k, f"library GEMM on our scale bytes {m}x{n}x{k}")
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 25600, 5120), (8, 208, 320), (33, 416, 1024), (64, 25600, 5120), (64, 200, 64),
+                                   (200, 528, 576)])
+def test_quantize_gemm_equals_separate_calls(m, n, k):
+    """nvfp4_quantize_gemm (dynamic quantization, then the GEMM, the weights
+    streaming early for m <= 64) gives the same quantized activations and the
+    same output bits as nvfp4_quantize_act followed by nvfp4_gemm, twice in a
+    row on one workspace, and the oracle's product within the bound."""
+    import torch
+    a = W.gaussian_bf16((m, k), 0, 1400 + m, 1.0, outlier_frac=0.01)
+    w = W.gaussian_bf16((n, k), 0, 1401 + n, 0.02)
+    wq = O.quantize_2d(w) if n % 16 == 0 else O.quantize_1d(w)
+    tw = nvfp4_from_host(*wq)
+    x = bf16_to_device(a)
+    for _ in range(2):
+        c1, qa1 = nv.quantize_gemm(x, tw)
+        qa2 = nv.quantize_act(x)
+        c2 = nv.gemm(qa2, tw)
+        _sync()
+        assert torch.equal(qa1.codes, qa2.codes) and torch.equal(qa1.scales, qa2.scales)
+        assert torch.equal(qa1.global_scale, qa2.global_scale)
+        assert torch.equal(c1, c2)
+    ac, asf, ga = O.quantize_1d(a)
+    assert np.array_equal(qa1.codes.cpu().numpy(), ac)
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(*wq))
+    assert_gemm_close(to_host_f64(c1), ref, absref, k, f"quantize_gemm {m}x{n}x{k}")
