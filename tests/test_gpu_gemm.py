@@ -262,7 +262,7 @@ def test_scale_layout_read_by_library_block_scaled_gemm(m, n, k):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 25600, 5120), (8, 208, 320), (33, 416, 1024), (64, 25600, 5120), (64, 200, 64),
-                                   (200, 528, 576)])
+                                   (4, 28608, 128), (200, 528, 576)])
 def test_quantize_gemm_equals_separate_calls(m, n, k):
     """nvfp4_quantize_gemm (dynamic quantization, then the GEMM, the weights
     streaming early for m <= 64) gives the same quantized activations and the
@@ -286,3 +286,67 @@ def test_quantize_gemm_equals_separate_calls(m, n, k):
     assert np.array_equal(qa1.codes.cpu().numpy(), ac)
     ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(*wq))
     assert_gemm_close(to_host_f64(c1), ref, absref, k, f"quantize_gemm {m}x{n}x{k}")
+
+
+def _check_qa_against_oracle(a_host, qa):
+    oc, osf, og = O.quantize_1d(a_host)
+    assert np.array_equal(qa.codes.cpu().numpy(), oc)
+    assert np.array_equal(qa.scales.cpu().numpy(), osf)
+    assert qa.global_scale.cpu().numpy().view(np.uint32)[0] == np.array([np.float32(og)]).view(np.uint32)[0]
+    return oc, osf, og
+
+
+@pytest.mark.parametrize("m,n,k", [(64, 208, 8192), (5, 400, 4096), (64, 416, 64), (40, 27008, 1024)])
+def test_quantize_gemm_decode_shapes(m, n, k):
+    """Decode-sized nvfp4_quantize_gemm (two-kernel quantizer, then the GEMM
+    streaming its first weight stages early) on long k (8192: 32 k-tiles,
+    more stages than the early weight stream covers), one partial k-tile
+    (k = 64), a two-tile n and a 141-tile n.  Codes, scale bytes (pad rows
+    zero) and g are the oracle's bit for bit; C is within the bound."""
+    a = W.gaussian_bf16((m, k), 2, 1500 + m, 1.0, outlier_frac=0.01)
+    w = W.gaussian_bf16((n, k), 2, 1501 + n, 0.02)
+    wq = O.quantize_2d(w)
+    tw = nvfp4_from_host(*wq)
+    c, qa = nv.quantize_gemm(bf16_to_device(a), tw)
+    _sync()
+    ac, asf, ga = _check_qa_against_oracle(a, qa)
+    ref, absref = gemm_refs(O.dequantize(ac, asf, ga), O.dequantize(*wq))
+    assert_gemm_close(to_host_f64(c), ref, absref, k, f"quantize_gemm {m}x{n}x{k}")
+
+
+def test_quantize_gemm_decode_call_sequence_on_one_workspace():
+    """One workspace through calls whose GEMM grids differ (n = 208: 2 CTAs,
+    n = 25600: 134), whose m changes, and whose amax goes up, down, to a tiny
+    global scale (g < 2^-64, the scaled reciprocal) and to zero (g = 1): the
+    quantizer's amax words come back to zero after every call, so each
+    call's quantization is the oracle's for its own x, and C equals
+    nvfp4_gemm on those codes."""
+    import torch
+    k = 1024
+    weights = {n: nvfp4_from_host(*O.quantize_2d(W.gaussian_bf16((n, k), 3, 1600 + n, 0.02))) for n in (208, 25600)}
+    seq = [(64, 25600, 1.0), (1, 208, 4.0), (17, 25600, 0.25), (64, 208, 1e-20), (8, 25600, 0.0), (64, 25600, 2.0)]
+    for i, (m, n, scale) in enumerate(seq):
+        if scale == 0.0:
+            a = np.zeros((m, k), np.uint16)
+        else:
+            a = W.gaussian_bf16((m, k), 3, 1700 + i, scale, outlier_frac=0.01)
+        c, qa = nv.quantize_gemm(bf16_to_device(a), weights[n])
+        c2 = nv.gemm(qa, weights[n])
+        _sync()
+        _check_qa_against_oracle(a, qa)
+        assert torch.equal(c, c2), f"call {i}"
+
+
+def test_quantize_gemm_decode_strided_activations():
+    """x as a view with a row stride above k (ldx = k + 64)."""
+    import torch
+    m, n, k = 48, 1040, 2048
+    a = W.gaussian_bf16((m, k + 64), 4, 1800, 1.0, outlier_frac=0.01)
+    xw = bf16_to_device(a)
+    x = xw[:, :k]
+    assert x.stride(0) == k + 64
+    tw = nvfp4_from_host(*O.quantize_2d(W.gaussian_bf16((n, k), 4, 1801, 0.02)))
+    c, qa = nv.quantize_gemm(x, tw)
+    _sync()
+    _check_qa_against_oracle(np.ascontiguousarray(a[:, :k]), qa)
+    assert torch.equal(c, nv.gemm(qa, tw))
