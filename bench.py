@@ -473,16 +473,28 @@ class Moe:
         return self.c[i % self.R]
 
     def gemm_label(self):
+        if self.n % 256 == 0:
+            return ("moe_swap_kernel (tcgen05 mxf4nvf4, cta_group::2; 256 weight rows x up to 256 tokens "
+                    "per tile)")
         return "gemm_pair_kernel<grouped> (tcgen05 mxf4nvf4, cta_group::2; 256 x 256 tiles per expert)"
 
     def padding(self):
-        """Rows of tensor-core work per expert, as the grouped GEMM tiles them
-        (experts of >= 192 rows on average take 256-row pair tiles), against
-        the rows that hold tokens."""
+        """Token columns of tensor-core work per expert, as the grouped GEMM
+        tiles them, against the rows that hold tokens.  With n a multiple of
+        256 the swapped kernel runs: tokens on the MMA's N side in tiles of
+        256, the last part rounded up to a multiple of 32 (riding on the tile
+        before it when it holds at most 64 tokens)."""
         sizes = np.diff(self.off.cpu().numpy().astype(np.int64))
-        tile = 256 if sizes.sum() >= 192 * len(sizes) else 128
-        padded = int(np.sum(-(-sizes // tile) * tile))
-        return {"token_rows": int(sizes.sum()), "mma_rows": padded, "tile_rows": tile,
+        if self.n % 256 == 0:
+            full = sizes // 256
+            last = sizes - 256 * full
+            padded = int(np.sum(256 * full + (-(-last // 32)) * 32))
+            tiling = "tokens on N: 256-token tiles, the last part rounded up to 32"
+        else:
+            tile = 256 if sizes.sum() >= 192 * len(sizes) else 128
+            padded = int(np.sum(-(-sizes // tile) * tile))
+            tiling = f"tokens on the MMA's M side in {tile}-row tiles"
+        return {"token_rows": int(sizes.sum()), "mma_rows": padded, "tiling": tiling,
                 "padding_frac": 1.0 - sizes.sum() / padded if padded else 0.0}
 
     def config(self):

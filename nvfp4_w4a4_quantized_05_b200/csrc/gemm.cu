@@ -1269,6 +1269,454 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     }
 }
 
+// ---- grouped GEMM with the operands swapped (MoE) ----------------------------------
+//
+// Per expert e (rows [r0, r0 + n_e) of A, weights W_e [n, k]) the pair kernel
+// above puts the tokens on the MMA's 256-row side, so an expert of 257 rows
+// takes two 256-row tiles.  Here the weights take the 256-row side (n % 256
+// == 0: M = 256 over the CTA pair, 128 weight rows per CTA) and the expert's
+// tokens the N side, in tiles of 256 tokens.  A last part of at most 64
+// tokens rides on the tile before it as a second MMA into a second
+// accumulator, against the same weight stages; any other last part is a tile
+// of its own.  Each part's N is its token count rounded up to a multiple of
+// 32 (cta_group::2 MMAs take N in steps of 16), so an expert pads fewer than
+// 32 rows.  Each CTA loads N / 2 token rows of a part (tensor maps with
+// boxes of 16, 32, 64 and 128 rows; the smallest that holds them) and stages
+// the scales of all token columns; token tiles start at multiples of 256
+// rows of the expert, i.e. at row 0 of a 128-row scale block.  Tiles of
+// expert e run (weight tile, token tile) with the token tile fastest, so the
+// CTAs working on one weight tile at the same time share it through L2.
+//
+// The accumulators hold weight rows in tensor-memory lanes and tokens in
+// columns (the second part's from column 256), so the epilogue writes C
+// transposed: each warp reads 32 token columns of its 32 lanes (one weight
+// row per thread) and converts them to BF16; neighbouring lanes swap values
+// so that each holds two adjacent output columns of one token, and one warp
+// store writes 64 contiguous bytes of each of two token rows of C.  Stores
+// stop at the expert's last token (the next rows of C belong to the next
+// expert).
+//
+// Warps: 0 producer, 1 MMA (leader), 2-9 epilogue (two per tensor-memory lane
+// quarter, alternate 32-column chunks), 10-13 scale staging.  Tensor memory
+// per CTA: the 256 + 64 accumulator columns, three scale buffers of 56.
+struct SwapCfg {
+    static constexpr int STAGES = 5;
+    static constexpr int NSB = 3;                          // scale buffers in tensor memory
+    static constexpr int N2_MAX = 64;                      // tokens of a second part
+    static constexpr uint32_t A_BYTES = 128 * 128;         // 128 weight rows x 256 FP4
+    static constexpr uint32_t B_BYTES = 128 * 128;         // up to 128 token rows x 256 FP4
+    static constexpr uint32_t B2_BYTES = (N2_MAX / 2) * 128;   // a second part's token rows
+    static constexpr uint32_t SFA_BYTES = 4 * 512;         // the CTA's 128 weight rows
+    static constexpr uint32_t SFB_BYTES = 3 * 4 * 512;     // <= 320 token rows from row 0 of a block: 3 blocks
+    static constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + B2_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int NBC = (256 + N2_MAX) / 32;        // token scale columns per k-step
+    static constexpr uint32_t SF_COLS = 16 + 4 * NBC;
+    static constexpr uint32_t SF_STRIDE = SF_COLS;
+    static constexpr uint32_t SF_BASE = 256 + N2_MAX;      // after the accumulators
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int THREADS = 32 * (2 + EPI_WARPS + 4);
+    static constexpr int NUM_BOXES = 4;                    // token maps with boxes of 16, 32, 64, 128 rows
+    static constexpr int MAX_CHUNKS = NBC;                 // 32-column accumulator chunks
+    static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+    static_assert((A_BYTES + B_BYTES) % 1024 == 0, "second token box alignment (128-byte swizzle)");
+    static_assert(SF_BASE + NSB * SF_STRIDE <= kTmemCols, "tensor memory budget");
+    static_assert(SF_BASE % 8 == 0 && SF_STRIDE % 8 == 0, "8-column stores start at a multiple of 8");
+};
+
+struct alignas(8) SwapTail {
+    uint64_t full[SwapCfg::STAGES];      // leader: both CTAs' weight and token bytes
+    uint64_t empty[SwapCfg::STAGES];     // each CTA: released by the leader's MMA commit
+    uint64_t sfl[SwapCfg::STAGES];       // each CTA: its own scale bytes landed
+    uint64_t acc_full;                   // each CTA: accumulators ready
+    uint64_t acc_empty;                  // leader: the epilogue warps of both CTAs read them
+    uint64_t sf_ready[SwapCfg::NSB];     // leader: 8 scale warps staged a buffer
+    uint64_t sf_free[SwapCfg::NSB];      // each CTA: MMAs reading a scale buffer done
+    uint32_t tmem_base;
+    volatile int abort_flag;
+    int total_tiles;
+    int tile_prefix[kMaxGroups + 1];     // first tile of expert e
+    int blk_prefix[kMaxGroups + 1];      // first 128-row token scale block of expert e
+};
+constexpr size_t kSwapSmem = 1024 + (size_t)SwapCfg::STAGES * SwapCfg::STAGE_BYTES + sizeof(SwapTail);
+static_assert(kSwapSmem <= 232448, "shared memory");
+
+// Token maps: one per box height (16 << i rows).
+struct SwapMaps {
+    CUtensorMap x[SwapCfg::NUM_BOXES];
+};
+
+// Token tiles of an expert of n_e rows: 256 each; a last part of at most 64
+// tokens joins the tile before it.
+__device__ __forceinline__ int swap_token_tiles(int n_e) {
+    const int full = n_e >> 8, rem = n_e & 255;
+    return full + ((rem > 0 && (full == 0 || rem > SwapCfg::N2_MAX)) ? 1 : 0);
+}
+__device__ __forceinline__ int swap_box(int rows) { return rows <= 16 ? 0 : rows <= 32 ? 1 : rows <= 64 ? 2 : 3; }
+
+// Where tile t lies.
+struct SwapTile {
+    int e;
+    int w_row;      // first weight tensor-map row of this CTA's 128
+    int tok0;       // first token row of the tile (A / C row)
+    int ntok;       // valid tokens of the tile (<= 256 + 64)
+    int N1, N2;     // MMA N of the two parts (tokens rounded up to 32; N2 = 0: one part)
+    int x1_row;     // first token row of this CTA's half of part 1
+    int x2_row;     // ... of part 2
+    int box1, box2; // token map of each part: 16 << box >= N / 2
+    int sfw_blk;    // weight scale block (128 rows) of this CTA, within the expert's weights
+    int sfx_blk;    // first token scale block of the tile
+    int nsfx;       // token scale blocks the tile touches (1 to 3)
+    int wcol0;      // first output column of this CTA's 128 weight rows
+};
+__device__ __forceinline__ SwapTile swap_tile(const GemmArgs& p, const SwapTail* tail, int t, uint32_t rank) {
+    int lo = 0, hi = p.num_groups;   // largest e with tile_prefix[e] <= t
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (tail->tile_prefix[mid] <= t) lo = mid; else hi = mid;
+    }
+    SwapTile s;
+    const int e = lo;
+    const int r0 = p.offsets[e], n_e = p.offsets[e + 1] - r0;
+    const int T = swap_token_tiles(n_e);
+    const int local = t - tail->tile_prefix[e];
+    const int wt = local / T, j = local - wt * T;
+    s.e = e;
+    s.ntok = j < T - 1 ? 256 : n_e - 256 * j;
+    s.N1 = (min(s.ntok, 256) + 31) & ~31;
+    s.N2 = s.ntok > 256 ? (s.ntok - 256 + 31) & ~31 : 0;
+    s.tok0 = r0 + 256 * j;
+    s.x1_row = s.tok0 + (s.N1 >> 1) * (int)rank;
+    s.x2_row = s.tok0 + 256 + (s.N2 >> 1) * (int)rank;
+    s.box1 = swap_box(s.N1 >> 1);
+    s.box2 = swap_box(s.N2 >> 1);
+    s.wcol0 = wt * 256 + 128 * (int)rank;
+    s.w_row = e * p.rows_b + s.wcol0;
+    s.sfw_blk = 2 * wt + (int)rank;
+    s.sfx_blk = tail->blk_prefix[e] + 2 * j;
+    s.nsfx = (s.N1 + s.N2 + 127) / 128;
+    return s;
+}
+
+__global__ void __launch_bounds__(SwapCfg::THREADS, 1)
+    moe_swap_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ SwapMaps tmX,
+                    const __grid_constant__ CUtensorMap tmC, const GemmArgs p) {
+    using P = SwapCfg;
+    constexpr int STAGES = P::STAGES, NBC = P::NBC;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    SwapTail* tail = reinterpret_cast<SwapTail*>(smem + STAGES * P::STAGE_BYTES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1;
+    const int P2 = (int)(gridDim.x >> 1);
+    const uint64_t limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&tail->full[s], 1);
+            mbar_init(&tail->empty[s], 1);
+            mbar_init(&tail->sfl[s], 1);
+        }
+        mbar_init(&tail->acc_full, 1);
+        mbar_init(&tail->acc_empty, 2 * P::EPI_WARPS);
+        for (int b = 0; b < P::NSB; ++b) {
+            mbar_init(&tail->sf_ready[b], 8);
+            mbar_init(&tail->sf_free[b], 1);
+        }
+        tail->abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmW);
+        for (int i = 0; i < P::NUM_BOXES; ++i) prefetch_tmap(&tmX.x[i]);
+        prefetch_tmap(&tmC);
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(&tail->tmem_base, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    pdl_wait();
+    if (warp == 2) {
+        // per-expert prefixes of tiles and token scale blocks (the offsets may
+        // come from the previous kernel)
+        const int E = p.num_groups, W = p.rows_b / 256;
+        const int per = (E + 31) / 32;
+        int t_loc = 0, b_loc = 0;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                const int n_e = p.offsets[e + 1] - p.offsets[e];
+                t_loc += swap_token_tiles(n_e) * W;
+                b_loc += (n_e + 127) / 128;
+            }
+        }
+        int t_inc = t_loc, b_inc = b_loc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int tv = __shfl_up_sync(0xFFFFFFFFu, t_inc, o);
+            const int bv = __shfl_up_sync(0xFFFFFFFFu, b_inc, o);
+            if (lane >= o) {
+                t_inc += tv;
+                b_inc += bv;
+            }
+        }
+        int t_run = t_inc - t_loc, b_run = b_inc - b_loc;
+        for (int i = 0; i < per; ++i) {
+            const int e = lane * per + i;
+            if (e < E) {
+                tail->tile_prefix[e] = t_run;
+                tail->blk_prefix[e] = b_run;
+                const int n_e = p.offsets[e + 1] - p.offsets[e];
+                t_run += swap_token_tiles(n_e) * W;
+                b_run += (n_e + 127) / 128;
+            }
+        }
+        if (lane == 31) {
+            tail->tile_prefix[E] = t_inc;
+            tail->blk_prefix[E] = b_inc;
+            tail->total_tiles = t_inc;
+        }
+    }
+    tc_fence_before();
+    cluster_sync();          // both CTAs' barriers initialized, tensor memory allocated, prefixes written
+    tc_fence_after();
+    const uint32_t tmem = tail->tmem_base;
+    const int total_tiles = tail->total_tiles;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------- TMA producer (both CTAs) ----------------
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int t = cluster; t < total_tiles && ok; t += P2) {
+                const SwapTile st = swap_tile(p, tail, t, rank);
+                const uint32_t xbytes = (16u << st.box1) * 128u + (st.N2 ? (16u << st.box2) * 128u : 0u);
+                const uint8_t* sfw_src =
+                    p.sfb + (int64_t)st.e * p.sfb_group_stride + (int64_t)st.sfw_blk * p.sfb_rb_stride;
+                const uint8_t* sfx_src = p.sfa + (int64_t)st.sfx_blk * p.sfa_rb_stride;
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait(&tail->empty[stage], phase ^ 1u, limit) || tail->abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    const int nat = min(4, p.num_ks - kt * 4);
+                    uint8_t* sA = smem + stage * P::STAGE_BYTES;
+                    uint8_t* sB = sA + P::A_BYTES;
+                    uint8_t* sB2 = sB + P::B_BYTES;
+                    uint8_t* sSFA = sB2 + P::B2_BYTES;
+                    uint8_t* sSFB = sSFA + P::SFA_BYTES;
+                    const uint32_t full0 = mapa_shared(smem_u32(&tail->full[stage]), 0);
+                    if (leader) mbar_arrive_expect_tx(&tail->full[stage], 2u * (P::A_BYTES + xbytes));
+                    tma_load_2d_pair(sA, &tmW, full0, kt * 128, st.w_row);
+                    tma_load_2d_pair(sB, &tmX.x[st.box1], full0, kt * 128, st.x1_row);
+                    if (st.N2) tma_load_2d_pair(sB2, &tmX.x[st.box2], full0, kt * 128, st.x2_row);
+                    uint64_t* sbar = &tail->sfl[stage];
+                    const uint32_t nch = (uint32_t)nat;
+                    mbar_arrive_expect_tx(sbar, nch * 512u * (1u + (uint32_t)st.nsfx));
+                    bulk_load(sSFA, sfw_src + (int64_t)kt * 2048, nch * 512u, sbar);
+                    for (int rb = 0; rb < st.nsfx; ++rb)
+                        bulk_load(sSFB + rb * 2048, sfx_src + (int64_t)rb * p.sfa_rb_stride + (int64_t)kt * 2048,
+                                  nch * 512u, sbar);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (!ok) {
+                tail->abort_flag = 1;
+                if (p.err) atomicOr(p.err, 1u);
+            }
+        }
+    } else if (warp == 1) {
+        if (leader && lane == 0) {
+            // ---------------- MMA issuer (pair leader) ----------------
+            uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
+            int it = 0;
+            bool ok = true;
+            for (int t = cluster; t < total_tiles && ok; t += P2, ++it) {
+                const SwapTile st = swap_tile(p, tail, t, rank);
+                const uint32_t idesc1 = idesc_mxf4nvf4(256, st.N1);
+                const uint32_t idesc2 = idesc_mxf4nvf4(256, st.N2 ? st.N2 : 32);
+                if (!mbar_wait(&tail->acc_empty, ((uint32_t)it & 1u) ^ 1u, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                for (int kt = 0; kt < p.num_kt; ++kt) {
+                    if (!mbar_wait(&tail->full[stage], phase, limit) ||
+                        !mbar_wait(&tail->sf_ready[sb], sph, limit) || tail->abort_flag) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nat = min(4, p.num_ks - kt * 4);
+                    const uint32_t sA = smem_u32(smem + stage * P::STAGE_BYTES);
+                    const uint32_t sB = sA + P::A_BYTES;
+                    const uint32_t sB2 = sB + P::B_BYTES;
+                    const uint32_t sf = tmem + P::SF_BASE + sb * P::SF_STRIDE;
+                    for (int j = 0; j < nat; ++j) {
+                        const uint64_t da = sdesc_kmajor_sw128(sA + j * 32);
+                        const uint32_t acc = (kt > 0 || j > 0) ? 1u : 0u;
+                        mma_mxf4nvf4_pair(tmem, da, sdesc_kmajor_sw128(sB + j * 32), idesc1, sf + j * 4,
+                                          sf + 16 + j * NBC, acc);
+                        if (st.N2)   // the second part: tokens 256.. (scale columns 8..)
+                            mma_mxf4nvf4_pair(tmem + 256, da, sdesc_kmajor_sw128(sB2 + j * 32), idesc2, sf + j * 4,
+                                              sf + 16 + j * NBC + 8, acc);
+                    }
+                    tc_commit_pair(&tail->empty[stage], 0x3);
+                    tc_commit_pair(&tail->sf_free[sb], 0x3);
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                    if (++sb == (uint32_t)P::NSB) {
+                        sb = 0;
+                        sph ^= 1u;
+                    }
+                }
+                if (ok) tc_commit_pair(&tail->acc_full, 0x3);
+            }
+            if (!ok) {
+                tail->abort_flag = 1;
+                if (p.err) atomicOr(p.err, 1u);
+            }
+        }
+    } else if (warp >= 2 + P::EPI_WARPS) {
+        // ---------------- scale staging (both CTAs; warps 10..13, one lane quarter each) ----------------
+        const int q = warp & 3;
+        const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + P::SF_BASE;
+        const uint32_t ready0 = mapa_shared(smem_u32(&tail->sf_ready[0]), 0);
+        const uint32_t ready_step = (uint32_t)(smem_u32(&tail->sf_ready[1]) - smem_u32(&tail->sf_ready[0]));
+        uint32_t stage = 0, phase = 0, sb = 0, sph = 0;
+        bool ok = true;
+        for (int t = cluster; t < total_tiles && ok; t += P2) {
+            for (int kt = 0; kt < p.num_kt; ++kt) {
+                if (!mbar_wait(&tail->sfl[stage], phase, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t sSFA =
+                    smem_u32(smem + stage * P::STAGE_BYTES) + P::A_BYTES + P::B_BYTES + P::B2_BYTES;
+                const uint32_t sSFB = sSFA + P::SFA_BYTES;
+                // one k-tile of scales, in tensor-memory column order: weight
+                // k-step j at 4j, token k-step j at 16 + NBC * j (column c =
+                // tokens 32c..32c+31; columns past a part's N are not read)
+                uint32_t w[P::SF_COLS];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const uint4 v = ld_shared_v4(sSFA + j * 512 + lane * 16);
+                    w[4 * j + 0] = v.x;
+                    w[4 * j + 1] = v.y;
+                    w[4 * j + 2] = v.z;
+                    w[4 * j + 3] = v.w;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+#pragma unroll
+                    for (int c = 0; c < NBC; ++c) {
+                        const int rr = 32 * c + lane;   // token row of the tile
+                        const uint32_t addr =
+                            sSFB + (uint32_t)((rr >> 7) * 2048 + j * 512 + (rr & 31) * 16 + ((rr >> 5) & 3) * 4);
+                        asm volatile("ld.shared.b32 %0, [%1];" : "=r"(w[16 + NBC * j + c]) : "r"(addr));
+                    }
+                if (!mbar_wait(&tail->sf_free[sb], sph ^ 1u, limit) || tail->abort_flag) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t dst = tq + sb * P::SF_STRIDE;
+#pragma unroll
+                for (int i = 0; i < (int)P::SF_COLS / 8; ++i) tmem_st_32x32b_x8(dst + 8 * i, w + 8 * i);
+                tmem_st_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(ready0 + sb * ready_step);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+                if (++sb == (uint32_t)P::NSB) {
+                    sb = 0;
+                    sph ^= 1u;
+                }
+            }
+        }
+        if (!ok && lane == 0) {
+            tail->abort_flag = 1;
+            if (p.err) atomicOr(p.err, 1u);
+        }
+    } else if (warp >= 2) {
+        // ---------------- epilogue (both CTAs; warps 2..9) ----------------
+        const int q = warp & 3;                       // tensor-memory lane quarter: weight rows 32q..32q+31
+        const int hh = (warp - 2) >> 2;               // this warp's chunks: hh, hh + 2, ...
+        const uint32_t empty0 = mapa_shared(smem_u32(&tail->acc_empty), 0);
+        const bool odd = lane & 1;
+        constexpr int WCH = (P::MAX_CHUNKS + 1) / 2;  // chunks per warp
+        int it = 0;
+        for (int t = cluster; t < total_tiles; t += P2, ++it) {
+            if (!mbar_wait(&tail->acc_full, (uint32_t)it & 1u, limit) || tail->abort_flag) {
+                if (lane == 0) {
+                    tail->abort_flag = 1;
+                    if (p.err) atomicOr(p.err, 1u);
+                }
+                break;
+            }
+            tc_fence_after();
+            const SwapTile st = swap_tile(p, tail, t, rank);
+            const float alpha = __fmul_rn(p.ga[st.e], p.gb[st.e]);
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+            // chunk c: accumulator columns (tokens) 32c..32c+31; part 1 fills
+            // chunks [0, N1 / 32), part 2 chunks [8, 8 + N2 / 32)
+            auto live = [&](int c) { return c < (st.N1 >> 5) || (c >= 8 && c < 8 + (st.N2 >> 5)); };
+            // all of this warp's chunks to registers as BF16 pairs of
+            // neighbouring tokens, then release the accumulators
+            uint32_t bf[WCH][16];
+#pragma unroll
+            for (int ci = 0; ci < WCH; ++ci) {
+                const int c = hh + 2 * ci;
+                if (live(c)) {   // uniform
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tq + (uint32_t)(c * 32), v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        bf[ci][i] = pack_bf16x2(__uint_as_float(v[2 * i]) * alpha, __uint_as_float(v[2 * i + 1]) * alpha);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(empty0);
+            // C[tok0 + 32c + i][col + lane]: lanes 2a, 2a + 1 (columns 2a,
+            // 2a + 1) swap halves, the even lane keeping even tokens and the
+            // odd lane odd ones, each as a BF16 pair of the two columns
+            __nv_bfloat16* cbase = p.c + (int64_t)st.tok0 * p.ldc + st.wcol0 + q * 32 + (lane & ~1);
+#pragma unroll
+            for (int ci = 0; ci < WCH; ++ci) {
+                const int c = hh + 2 * ci;
+                if (!live(c)) continue;                     // uniform
+                const int nt = min(32, st.ntok - 32 * c);   // valid tokens of the chunk
+#pragma unroll
+                for (int k = 0; k < 16; ++k) {
+                    const uint32_t own = bf[ci][k];
+                    const uint32_t nb = __shfl_xor_sync(0xFFFFFFFFu, own, 1);
+                    const uint32_t word = odd ? prmt_b32(nb, own, 0x7632) : prmt_b32(own, nb, 0x5410);
+                    const int row = 2 * k + (odd ? 1 : 0);
+                    if (row < nt)
+                        *reinterpret_cast<uint32_t*>(cbase + (int64_t)(32 * c + row) * p.ldc) = word;
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();          // no CTA leaves while its peer may still touch its shared memory
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem, kTmemCols);
+    }
+}
+
 // ---- host side -----------------------------------------------------------------
 
 // 2-D uint8 view [rows, row_bytes] of packed codes, 128-byte x box_rows boxes,
@@ -1587,6 +2035,55 @@ extern "C" nvfp4_status_t nvfp4_gemm_emit_scale(const uint8_t* a_codes, const ui
                      ws + kEmitScaleWsBytes, reinterpret_cast<uint32_t*>(ws), c_global_scale, stream);
 }
 
+namespace nvfp4 {
+namespace {
+cudaLaunchConfig_t swap_config(int clusters, cudaStream_t s, cudaLaunchAttribute (&attr)[2]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.blockDim = dim3(SwapCfg::THREADS);
+    cfg.dynamicSmemBytes = kSwapSmem;
+    cfg.stream = s;
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cfg;
+}
+// Pairs of moe_swap_kernel that can be resident at once, per device (0: unavailable).
+int swap_clusters_resident() {
+    static std::mutex mu;
+    static int cached[64] = {};
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= 64) return 0;
+    std::lock_guard<std::mutex> lk(mu);
+    if (cached[d] == 0) {
+        if (cudaFuncSetAttribute(moe_swap_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSwapSmem) !=
+            cudaSuccess)
+            return 0;
+        cudaLaunchAttribute attr[2];
+        cudaLaunchConfig_t cfg = swap_config(1, nullptr, attr);
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, moe_swap_kernel, &cfg) != cudaSuccess || n <= 0) return 0;
+        cached[d] = n;
+    }
+    return cached[d];
+}
+nvfp4_status_t launch_swap(const CUtensorMap& tw, const SwapMaps& tx, const CUtensorMap& tc, const GemmArgs& args,
+                           int clusters, cudaStream_t s) {
+    static std::atomic<unsigned long long> attr_done{0};
+    if (!smem_attr_on_device(reinterpret_cast<const void*>(moe_swap_kernel), (int)kSwapSmem, attr_done))
+        return NVFP4_ERR_CUDA;
+    cudaLaunchAttribute attr[2];
+    cudaLaunchConfig_t cfg = swap_config(clusters, s, attr);
+    return cuda_status(cudaLaunchKernelEx(&cfg, moe_swap_kernel, tw, tx, tc, args));
+}
+}  // namespace
+}  // namespace nvfp4
+
 extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8_t* a_scales, const float* a_global,
                                              const int32_t* offsets, int num_experts, const uint8_t* b_codes,
                                              const uint8_t* b_scales, const float* b_global, void* c, int64_t n,
@@ -1631,6 +2128,20 @@ extern "C" nvfp4_status_t nvfp4_grouped_gemm(const uint8_t* a_codes, const uint8
     p.err = device_error_word();
     if (!p.err) return NVFP4_ERR_CUDA;
     CUtensorMap ta, tb, tc;
+    // Weights in whole 256-row tiles: the swapped kernel (weights on the
+    // 256-row MMA side, each expert's tokens on N, padded to 32 at most).
+    const int swap_max = swap_clusters_resident();
+    if (n % 256 == 0 && swap_max > 0 && sms >= 2) {
+        SwapMaps tx;
+        if (!make_codes_map(&tb, b_codes, n * num_experts, k / 2, 128) || !make_out_map(&tc, c, total_rows, n, n))
+            return NVFP4_ERR_CUDA;
+        for (int i = 0; i < SwapCfg::NUM_BOXES; ++i)
+            if (!make_codes_map(&tx.x[i], a_codes, total_rows, k / 2, 16 << i)) return NVFP4_ERR_CUDA;
+        // upper bound of the tile count: sum_e ceil(n_e / 256) <= total_rows / 256 + num_experts
+        const int64_t max_tiles = (total_rows / 256 + num_experts) * (n / 256);
+        const int clusters = (int)std::min<int64_t>(max_tiles, std::min(swap_max, sms / 2));
+        return launch_swap(tb, tx, tc, p, clusters, s);
+    }
     // Experts of 192 rows or more on average (prefill-sized MoE): 256 x 256
     // pair tiles, every tile whole; smaller groups would mostly pad a 256-row
     // tile, so they take the 128 x 192 single-SM tiles.

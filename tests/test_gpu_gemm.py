@@ -165,7 +165,16 @@ def test_decode_workload_full(m, decode_weights):
     # rows (one valid row in the second half), of exactly 256, of 1, of 0, and
     # ragged n (last column tile 8 wide) with a partial last k-tile
     ([300, 0, 129, 256, 511, 1, 385, 200], 576, 520),
+    # n % 256 == 0: the swapped kernel (weights on the 256-row side, tokens
+    # on N in tiles of 256; a last part of <= 64 tokens rides on the tile
+    # before it as a second MMA, a larger one is a tile of its own, each
+    # rounded up to 32 tokens): experts of 0, 1, 16, 31, 32, 33 ... 700 rows
+    # (one, two and three token tiles; parts of every box height; riding
+    # parts of 1 and 44 tokens; partial last 32-token chunks), a partial last
+    # k-tile (k = 320) and two weight tiles
     ([256] * 3 + [255, 257], 1024, 256),
+    ([0, 1, 16, 31, 32, 33, 100, 128, 129, 255, 256, 257, 300, 511, 512, 513, 700, 0], 320, 512),
+    ([40, 97, 64], 2048, 1536),
 ])
 def test_grouped_gemm_ragged_experts(sizes, k, n):
     off = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32)
