@@ -98,6 +98,11 @@ struct GemmArgs {
     // B tiles before griddepcontrol.wait (the weight stream starts while the
     // activations are still being quantized)
     int b_early;
+    // 1: let the next kernel on the stream launch at this grid's start (its
+    // CTAs take SMs as these leave; it waits for this grid before reading
+    // what this one writes).  Off for decode-size and grouped shapes, whose
+    // steps measured slower with it.
+    int pdl_trigger;
 };
 
 // The largest |value| of packed BF16 pairs, as a 16-bit pattern.
@@ -249,6 +254,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     SmemTail* tail = reinterpret_cast<SmemTail*>(epi_smem + C::EPI_BYTES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint64_t limit = p.wait_limit_ns;
+    if (p.pdl_trigger) pdl_launch_dependents();
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -795,6 +801,7 @@ __global__ void __launch_bounds__(P::THREADS, 1)
     const bool leader = rank == 0;
     const int cluster = blockIdx.x >> 1;
     const uint64_t limit = p.wait_limit_ns;
+    if (p.pdl_trigger) pdl_launch_dependents();   // as in gemm_kernel
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -1411,6 +1418,9 @@ __global__ void __launch_bounds__(SwapCfg::THREADS, 1)
     const int cluster = blockIdx.x >> 1;
     const int P2 = (int)(gridDim.x >> 1);
     const uint64_t limit = p.wait_limit_ns;
+    // No early launch of the next kernel here: on the MoE step the next one is
+    // the grouped one-launch quantizer, and starting it while this grid's
+    // pairs finish unevenly cost ≈ 4 us per step (measured).
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -1981,6 +1991,7 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
         p.dp_tiles = sk ? pl.dp_tiles : (int)pl.tiles;
         p.sk_units = sk ? pl.sk_units : 0;
         p.sk_flags = sk ? reinterpret_cast<uint32_t*>(workspace) : nullptr;
+        p.pdl_trigger = 1;
         p.partial = sk ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(workspace) + kSkFlagsBytes) : nullptr;
         if (mx) return launch_pair<false, false, true>(ta, tb, tc, p, pl.clusters, s);
         return c_amax ? launch_pair<false, true>(ta, tb, tc, p, pl.clusters, s)
@@ -2001,6 +2012,7 @@ nvfp4_status_t gemm_impl(const uint8_t* a_codes, const uint8_t* a_scales, const 
     p.tiles_n = (int)((n + BN - 1) / BN);
     const int64_t tiles = (int64_t)p.tiles_m * p.tiles_n;
     if (tiles >= ((int64_t)1 << 31)) return NVFP4_ERR_UNSUPPORTED_SHAPE;
+    p.pdl_trigger = 1;
     const int grid = (int)std::min<int64_t>(tiles, sms);
     if (mx) return launch<CfgWide, false, false, true>(ta, tb, tc, p, grid, s);
     return c_amax ? launch<CfgWide, false, true>(ta, tb, tc, p, grid, s) : launch<CfgWide, false>(ta, tb, tc, p, grid, s);

@@ -344,11 +344,15 @@ struct AmaxArgs {
 constexpr int kAmaxUnroll = 8;
 
 // The kernels below let the next kernel in the stream launch as soon as all
-// their CTAs run (griddepcontrol.launch_dependents at the start): a dependent
-// kernel's griddepcontrol.wait still waits for this grid's completion and
-// writes, so it may only do independent work earlier (prefetch its own
-// inputs that this kernel does not write).
+// their CTAs run (griddepcontrol.launch_dependents): a dependent kernel's
+// griddepcontrol.wait still waits for this grid's completion and writes, so
+// it may only do independent work earlier (prefetch its own inputs that this
+// kernel does not write).  The amax kernel is itself launched as a
+// dependent (it may start while the kernel before it, perhaps the producer
+// of x, is finishing), so it waits before anything else and only then lets
+// its own dependent start: that one may read x before its wait.
 __global__ void __launch_bounds__(kThreads, 4) amax_kernel(AmaxArgs a) {
+    pdl_wait();
     pdl_launch_dependents();
     const int e = blockIdx.y;
     int r0, r1;
@@ -1150,6 +1154,9 @@ __global__ void __launch_bounds__(kFThreads, 1)
     // (tensor-memory tasks 0 .. kTmTasks - 1, then the slot tasks)
     __shared__ uint32_t s_bm[kPlain ? (kTmTasks + kStage) * kFWarps * 32 : 1];
     __shared__ int32_t s_qtab[kPlain ? 128 : 1];
+    // Launched as a programmatic dependent: everything below may read what
+    // the previous kernel wrote (x, this workspace).
+    pdl_wait();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int G = gridDim.x;
     const int t0 = (int)((int64_t)a.tasks * blockIdx.x / G);
@@ -1573,11 +1580,13 @@ nvfp4_status_t run_fused(const uint16_t* x, int64_t rows, int64_t k, int64_t ld,
     cfg.blockDim = dim3(kFThreads);
     cfg.dynamicSmemBytes = (size_t)(depth > 0 ? depth : 1) * kFWarps * kTaskBytes + 1024;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeCooperative;   // all CTAs resident at once (grid barrier)
     attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may launch early; waits first
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     void* args[] = {&tmap, &a, &box_bytes};
     const void* kern = grouped  ? reinterpret_cast<const void*>(&quant1d_fused_kernel<true>)
                        : smooth ? reinterpret_cast<const void*>(&quant1d_fused_kernel<false, true>)
@@ -1602,8 +1611,8 @@ nvfp4_status_t run_amax(const uint16_t* x, int64_t rows, int64_t k, int64_t ld, 
     const int64_t per_group = (chunks + groups - 1) / groups;
     const int gx = clamp_grid((per_group + kThreads * kAmaxUnroll - 1) / (kThreads * kAmaxUnroll),
                               (int64_t)num_sms() * 4 / groups);
-    amax_kernel<<<dim3(gx, groups), kThreads, 0, s>>>(a);
-    return cuda_status(cudaGetLastError());
+    void* args[] = {&a};
+    return cuda_status(launch_pdl(reinterpret_cast<const void*>(&amax_kernel), dim3(gx, groups), dim3(kThreads), args, s));
 }
 
 }  // namespace
