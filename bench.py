@@ -349,6 +349,20 @@ class Decode(Prefill):
         self.quantize(i)
         self.gemm(i)
 
+    def prepare_two_phase(self):
+        """Each buffer set's global scale, as the GEMM that produced the
+        activations would have emitted it (nvfp4_gemm_emit_scale); taken
+        before timing."""
+        self.g_given = [self.nv.quantize_act(a).global_scale.clone() for a in self.a]
+
+    def two_phase_step(self, i):
+        """The step when the producing layer has already emitted x's global
+        scale: the given-scale quantize pass, then the GEMM; no amax pass.
+        The codes and scales equal the dynamic step's."""
+        j = i % self.R
+        self.nv.quantize_act_scaled(self.a[j], self.g_given[j], out=self.qa[j])
+        self.gemm(i)
+
     def step_bytes(self):
         """Algorithmic HBM bytes of one step: x, the weights (codes, scales),
         A's codes and scales written and read once, C."""
@@ -763,6 +777,8 @@ def measure_decode(nv, torch, dev, cs, sampler, peaks, with_cpu, ms=(1, 8, 32, 6
             j = i % wl.R
             nv.gemm_w4a16(wl.a[j], wl.w[j], out=wl.c[j])
         t16, clk16 = timed_loop(torch, cs, w16, wl.R, KERNEL_ITERS, sampler)
+        wl.prepare_two_phase()
+        tp_s, tp_clk = timed_loop(torch, cs, wl.two_phase_step, wl.R, n, sampler)
         gbytes = wl.wbytes + wl.abytes + wl.cbytes
         g_gbs = gbytes / g_s / 1e9
         s_gbs = wl.step_bytes() / step_s / 1e9
@@ -772,6 +788,9 @@ def measure_decode(nv, torch, dev, cs, sampler, peaks, with_cpu, ms=(1, 8, 32, 6
              "step_roofline": _roofline("hbm", "the step's three kernels", s_gbs, hbm, "GB/s", None, step_s, clk,
                                         algorithmic_bytes=wl.step_bytes(), launches_timed=n),
              "separate_step_ms": sep_s * 1e3, "separate_step_clocks": sep_clk,
+             "two_phase_step_ms": tp_s * 1e3, "two_phase_step_clocks": tp_clk,
+             "two_phase_step_path": "global scale emitted by the producing GEMM: nvfp4_quantize_act_scaled "
+                                    "(quantize pass only), then nvfp4_gemm",
              "quantize_ms": q_s * 1e3, "gemm_ms": g_s * 1e3,
              "gemm_tflops": wl.flops / g_s / 1e12, "gemm_frac_fp4": wl.flops / g_s / 1e12 / fp4_peak,
              "weight_stream_gbs": wl.wbytes / g_s / 1e9, "weight_stream_frac_hbm": wl.wbytes / g_s / 1e9 / hbm,
